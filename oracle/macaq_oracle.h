@@ -1,0 +1,112 @@
+/*
+ * Test infrastructure: the CPU oracle of the MACaQ W4A4 linear layer.
+ *
+ * Only tests/, __graft_entry__.smoke() and bench.py's CPU-baseline leg may load this
+ * library. The product path (the CUDA library and its Python binding) never calls it,
+ * and the two share no code, header, table or constant generator.
+ *
+ * What it computes (MACaQ pages: "Quantization mechanism" of the zicq.com English
+ * article, equation y = xW^T and the garbled transformed form; openai-hub.com
+ * article, paragraphs on MXFP4 and on the block Hadamard "micro-rotation"):
+ *
+ *   y = x W^T = (x D^-1 Hb) (Hb D W^T),   D = diag(s),
+ *   Hb = block-diag(H32 / sqrt(32)), H32 the Sylvester Hadamard matrix,
+ *
+ * with both factors quantised to OCP MXFP4 (E2M1 elements, one E8M0 scale per 32).
+ *
+ * Precision: the quantisation steps run in IEEE fp32 with round-to-nearest-even,
+ * no FMA contraction, in the fixed butterfly order given below,
+ * because the fp32 result decides integer codes. The GEMM reference and the
+ * exact-algebra helpers run in fp64.
+ *
+ * Parity status: every function below is pinned by tests in tests/test_oracle_*.py
+ * against closed forms, library routines (scipy's Hadamard, numpy matmul) or brute
+ * force; none is "parity unpinned".
+ */
+#ifndef MACAQ_ORACLE_H
+#define MACAQ_ORACLE_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* (-1)^popcount(i & j): entry (i, j) of the natural-order Sylvester matrix H_n. */
+int oracle_hadamard_entry(int i, int j);
+
+/* Widen a bf16 bit pattern to fp32 (exact: bf16 is the upper half of an fp32). */
+float oracle_bf16_to_f32(uint16_t b);
+
+/* In-place 32-point Walsh-Hadamard butterfly in fp32, stages h = 1,2,4,8,16,
+ * pair (a, b) -> (a + b, a - b) with a at the lower index, then every element is
+ * multiplied by c = fp32(1/sqrt(32)) (bit pattern 0x3E3504F3). */
+void oracle_fwht32_f32(float v[32]);
+
+/* Shared-exponent rule: e = max(floor(log2 amax) - 2, -127); amax == 0 gives -127.
+ * floor(log2) is read exactly from the fp32 bit pattern. Returns e in [-127, 125]. */
+int oracle_e8m0_exponent(float amax);
+
+/* E2M1 round-to-nearest, ties to the even mantissa bit, saturating at +-6.
+ * Returns the 4-bit code (sign << 3 | index into {0,.5,1,1.5,2,3,4,6}); the sign of
+ * q is kept, so -0 and tiny negatives encode as 0x8. */
+uint8_t oracle_e2m1_encode(float q);
+
+/* Decode a 4-bit E2M1 code to its value. */
+double oracle_e2m1_decode(uint8_t code);
+
+/* Element-wise loops over the two scalar rules above, for sweeps from tests. */
+void oracle_e2m1_encode_array(const float* q, int64_t n, uint8_t* out);
+void oracle_e8m0_exponent_array(const float* amax, int64_t n, int32_t* out);
+
+/* Quantise rows of a bf16 matrix through the MACaQ transform.
+ *   x      : bf16 bits, rows x K, row stride ld (elements)
+ *   mult   : K fp32 multipliers (inv_s for activations, s for weights)
+ *   codes  : rows x K/2 bytes, element 2j in the low nibble of byte j
+ *   scales : rows x K/32 bytes, row-major E8M0 (value 2^(byte - 127))
+ * K must be a multiple of 32. */
+void oracle_quant_rows(const uint16_t* x, int64_t rows, int64_t K, int64_t ld,
+                       const float* mult, uint8_t* codes, uint8_t* scales);
+
+/* Offline weight preparation: W' = W D Hb quantised like the activations
+ * (multiplier s), and inv_s[k] = 1.0f / s[k] in IEEE fp32. */
+void oracle_prepare_weight(const uint16_t* W, int64_t N, int64_t K, int64_t ld,
+                           const float* s, uint8_t* codes, uint8_t* scales, float* inv_s);
+
+/* Padded geometry of the tensor-core scale layout: rows rounded up to 128, scale
+ * blocks per row rounded up to 8 (a whole number of 4-block atoms per 256-wide
+ * K tile). */
+int64_t oracle_scale_rows_padded(int64_t rows);
+int64_t oracle_scale_blocks_padded(int64_t K);
+
+/* Byte offset of scale (r, j) in the 128-row x 4-block atom layout consumed by the
+ * Blackwell block-scaled MMA. */
+int64_t oracle_scale_offset(int64_t r, int64_t j, int64_t K);
+
+/* Row-major [rows x K/32] scales -> atom layout (padding bytes set to 0), and back. */
+void oracle_swizzle_scales(const uint8_t* rowmajor, int64_t rows, int64_t K, uint8_t* atom);
+void oracle_unswizzle_scales(const uint8_t* atom, int64_t rows, int64_t K, uint8_t* rowmajor);
+
+/* y[m, n] = sum_k dec(a[m,k]) 2^ea[m,k/32] * dec(w[n,k]) 2^ew[n,k/32], summed in fp64.
+ * Codes as produced by oracle_quant_rows, scales row-major. Rows of A listed in
+ * `rows` (or all M rows if rows == NULL), output row i is y + i * N. */
+void oracle_gemm_fp64(const uint8_t* a_codes, const uint8_t* a_scales, int64_t M,
+                      const uint8_t* w_codes, const uint8_t* w_scales, int64_t N, int64_t K,
+                      const int64_t* rows, int64_t n_rows, double* y);
+
+/* Dequantise MXFP4 rows to fp64 (value = dec(code) * 2^e). */
+void oracle_dequant_rows(const uint8_t* codes, const uint8_t* scales, int64_t rows, int64_t K,
+                         double* out);
+
+/* Exact-algebra transform in fp64 with the dense block matrix (no butterfly, no
+ * quantisation): out[r, :] = (x[r, :] * mult) Hb_unnormalised / norm, where
+ * Hb_unnormalised has +-1 entries and norm is a caller-chosen divisor (sqrt(32) for
+ * the orthonormal transform, 1 for the raw +-1 product). */
+void oracle_transform_rows_f64(const double* x, int64_t rows, int64_t K, const double* mult,
+                               double norm, double* out);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif

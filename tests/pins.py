@@ -1,0 +1,328 @@
+"""Pins of the CPU oracle to things other than itself.
+
+Each pin checks one oracle function against a closed form, a library routine
+(scipy's Hadamard matrix, numpy's matmul and ldexp, IEEE division), brute force, or a
+value the pages print. The oracle tests run every pin; the mutation tests compile
+broken copies of the oracle and require that some pin fails for each.
+"""
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import scipy.linalg
+
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+H32 = scipy.linalg.hadamard(32).astype(np.int64)          # Sylvester order, library routine
+C32 = np.float32(1.0 / math.sqrt(32.0))                    # nearest fp32 to 2^-2.5
+
+
+def golden_e2m1():
+    vals = {}
+    with open(os.path.join(GOLDEN, "e2m1_values.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if line and not line.startswith("#"):
+                c, v = line.split()
+                vals[int(c)] = float(v)
+    return vals
+
+
+def golden_storage_bits():
+    with open(os.path.join(GOLDEN, "storage_bits.txt")) as f:
+        return float([ln for ln in f if ln.strip() and not ln.startswith("#")][0])
+
+
+# ----------------------------------------------------------- brute force -----
+
+def bf_e2m1_encode(q: np.float32) -> int:
+    """Nearest E2M1 magnitude by exhaustive search, ties to the even mantissa bit
+    (the code whose lowest bit is 0); the sign bit copies the sign of q."""
+    table = golden_e2m1()
+    mags = [Fraction(table[c]) for c in range(8)]
+    a = abs(Fraction(float(q)))                      # exact rational distances
+    best = None
+    for idx, m in enumerate(mags):
+        d = abs(m - a)
+        key = (d, idx & 1)           # distance first, then prefer even mantissa
+        if best is None or key < best[0]:
+            best = (key, idx)
+    sign = 8 if math.copysign(1.0, float(q)) < 0 else 0
+    return sign | best[1]
+
+
+def bf_e8m0(amax: float) -> int:
+    """e = clamp(floor(log2 amax) - 2, -127, 127) from math.frexp (exact)."""
+    if amax == 0.0:
+        return -127
+    _, ex = math.frexp(amax)      # amax = m * 2^ex, m in [0.5, 1)
+    return max(min(ex - 1 - 2, 127), -127)
+
+
+def blockdiag_H(K):
+    Hb = np.zeros((K, K), np.float64)
+    for b in range(K // 32):
+        Hb[32 * b:32 * b + 32, 32 * b:32 * b + 32] = H32
+    return Hb
+
+
+def pack_nibbles(codes_2d):
+    lo = codes_2d[:, 0::2].astype(np.uint8)
+    hi = codes_2d[:, 1::2].astype(np.uint8)
+    return lo | (hi << 4)
+
+
+# ------------------------------------------------------------------ pins -----
+
+def pin_hadamard_matches_scipy():
+    got = np.array([[oracle.hadamard_entry(i, j) for j in range(32)] for i in range(32)])
+    assert np.array_equal(got, H32), "H32 entries differ from scipy.linalg.hadamard(32)"
+
+
+def pin_hadamard_orthogonal():
+    H = np.array([[oracle.hadamard_entry(i, j) for j in range(32)] for i in range(32)], np.int64)
+    assert np.array_equal(H @ H.T, 32 * np.eye(32, dtype=np.int64))
+    assert np.array_equal(H, H.T)
+
+
+def pin_normalisation_constant():
+    assert C32.view(np.uint32) == 0x3E3504F3
+    exact = 2.0 ** -2.5
+    for nb in (np.nextafter(C32, np.float32(1)), np.nextafter(C32, np.float32(0))):
+        assert abs(float(C32) - exact) < abs(float(nb) - exact)
+
+
+def pin_fwht_integer_exact():
+    rng = np.random.default_rng(1)
+    for _ in range(200):
+        v = rng.integers(-1000, 1001, size=32)
+        expect = (np.float32(H32 @ v) * C32).astype(np.float32)
+        got = oracle.fwht32(v.astype(np.float32))
+        assert np.array_equal(got.view(np.uint32), expect.view(np.uint32)), (v, got, expect)
+
+
+def pin_fwht_float_bound():
+    rng = np.random.default_rng(2)
+    u = 2.0 ** -24
+    for _ in range(200):
+        v = (rng.standard_normal(32) * rng.choice([1e-3, 1.0, 1e3])).astype(np.float32)
+        exact = (H32 @ v.astype(np.float64)) / math.sqrt(32.0)
+        got = oracle.fwht32(v).astype(np.float64)
+        bound = 8 * u * np.abs(v.astype(np.float64)).sum() / math.sqrt(32.0)
+        assert np.all(np.abs(got - exact) <= bound), np.abs(got - exact).max() / bound
+
+
+def pin_identity_exact():
+    """x W^T == (x D^-1 H)(H D W^T) / 32 exactly, for small integers and s = 2^k."""
+    rng = np.random.default_rng(3)
+    M, N, K = 5, 7, 96
+    x = rng.integers(-8, 9, size=(M, K)).astype(np.float64)
+    W = rng.integers(-8, 9, size=(N, K)).astype(np.float64)
+    s = 2.0 ** rng.integers(-3, 4, size=K)
+    lhs = x @ W.T
+    xa = oracle.transform_rows_f64(x, 1.0 / s, 1.0)
+    wa = oracle.transform_rows_f64(W, s, 1.0)
+    rhs = (xa @ wa.T) / 32.0
+    assert np.array_equal(lhs, rhs)
+    # the same transform written with the dense block matrix from scipy
+    assert np.array_equal(xa, (x / s) @ blockdiag_H(K))
+
+
+def pin_identity_random():
+    rng = np.random.default_rng(4)
+    M, N, K = 6, 9, 128
+    x = rng.standard_normal((M, K))
+    W = rng.standard_normal((N, K))
+    s = np.exp(rng.normal(0, 0.5, K))
+    lhs = x @ W.T
+    rhs = oracle.transform_rows_f64(x, 1.0 / s, math.sqrt(32)) @ \
+        oracle.transform_rows_f64(W, s, math.sqrt(32)).T
+    assert np.linalg.norm(lhs - rhs) <= 1e-12 * np.linalg.norm(lhs)
+
+
+def pin_e2m1_decode():
+    table = golden_e2m1()
+    for c in range(16):
+        got = oracle.e2m1_decode(c)
+        assert got == table[c] and math.copysign(1, got) == math.copysign(1, table[c]), c
+
+
+def _encode_sweep_points():
+    table = golden_e2m1()
+    mags = sorted(set(abs(table[c]) for c in range(8)))
+    ties = [(a + b) / 2 for a, b in zip(mags[:-1], mags[1:])]
+    pts = [np.float32(t) for t in ties + mags + [7.0, 8.0, 100.0, 1e30]]
+    extra = []
+    for p in pts:
+        extra += [np.nextafter(p, np.float32(0)), np.nextafter(p, np.float32(np.inf))]
+    pts = np.array(pts + extra + [1e-30, 1.4e-45, 0.0], np.float32)
+    pts = np.concatenate([pts, -pts, np.linspace(-10, 10, 20001, dtype=np.float32)])
+    return pts
+
+
+def pin_e2m1_encode_bruteforce():
+    pts = _encode_sweep_points()
+    got = oracle.e2m1_encode(pts)
+    for q, g in zip(pts, got):
+        assert g == bf_e2m1_encode(q), (float(q), int(g), bf_e2m1_encode(q))
+
+
+def pin_e8m0_closed_form():
+    rng = np.random.default_rng(5)
+    vals = [0.0, 1.4e-45, 1e-40, 1.1754942e-38, 1.17549435e-38, 3.4e38]
+    for k in range(-149, 128):
+        p = np.float32(2.0 ** k)
+        vals += [p, np.nextafter(p, np.float32(0)), np.nextafter(p, np.float32(np.inf))]
+    vals += list(np.abs(rng.standard_normal(2000)).astype(np.float32) *
+                 np.float32(2.0) ** rng.integers(-140, 120, 2000).astype(np.float32))
+    a = np.array(vals, np.float32)
+    a = a[np.isfinite(a)]
+    got = oracle.e8m0_exponent(a)
+    for x, g in zip(a, got):
+        assert g == bf_e8m0(float(x)), (float(x), int(g), bf_e8m0(float(x)))
+        if g > -127:
+            r = float(x) * 2.0 ** (-int(g))
+            assert 4.0 <= r < 8.0
+
+
+def _exact_rows(rng, rows, K):
+    """Rows whose transform is exact in fp32: small-integer bf16 inputs and
+    power-of-two multipliers."""
+    xi = rng.integers(-64, 65, size=(rows, K)).astype(np.float32)
+    xi[rng.random((rows, K)) < 0.2] = 0.0
+    xi[0, :32] = 0.0                                   # an all-zero block
+    xi[1, 32:64] = 0.0
+    xi[1, 40] = 64.0                                   # a one-hot block
+    mult = (2.0 ** rng.integers(-3, 4, size=K)).astype(np.float32)
+    xb = (xi.view(np.uint32) >> 16).astype(np.uint16)  # small integers are exact in bf16
+    return xi, xb, mult
+
+
+def pin_quant_rows_exact_inputs():
+    rng = np.random.default_rng(6)
+    rows, K = 9, 192
+    xi, xb, mult = _exact_rows(rng, rows, K)
+    codes, scales = oracle.quant_rows(xb, mult)
+    u = xi.astype(np.float64) * mult                   # exact
+    for r in range(rows):
+        exp_codes = np.zeros(K, np.uint8)
+        for b in range(K // 32):
+            t = H32 @ u[r, 32 * b:32 * b + 32]          # exact integer-ish sums
+            v = (np.float32(t) * C32).astype(np.float32)
+            e = bf_e8m0(float(np.abs(v).max()))
+            assert scales[r, b] == e + 127, (r, b, scales[r, b], e)
+            q = (v.astype(np.float64) * 2.0 ** (-e)).astype(np.float32)
+            exp_codes[32 * b:32 * b + 32] = [bf_e2m1_encode(qq) for qq in q]
+        assert np.array_equal(codes[r], pack_nibbles(exp_codes[None, :])[0]), r
+
+
+def pin_quant_rows_error_bound():
+    rng = np.random.default_rng(7)
+    rows, K = 8, 256
+    x = rng.standard_t(3, size=(rows, K)).astype(np.float32)
+    x[:, 5] *= 40
+    xb = (x.view(np.uint32) >> 16).astype(np.uint16)   # truncation is fine for a bound test
+    mult = np.exp(rng.normal(0, 0.5, K)).astype(np.float32)
+    codes, scales = oracle.quant_rows(xb, mult)
+    deq = oracle.dequant_rows(codes, scales, K)
+    xf = (xb.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    v = (xf * mult.astype(np.float64)) @ blockdiag_H(K) / math.sqrt(32)
+    for r in range(rows):
+        for b in range(K // 32):
+            vb = v[r, 32 * b:32 * b + 32]
+            db = deq[r, 32 * b:32 * b + 32]
+            e = int(scales[r, b]) - 127
+            amax = np.abs(vb).max()
+            rel = 1e-5                                  # fp32 transform error vs fp64
+            if abs(math.log2(amax) - round(math.log2(amax))) > 1e-5:
+                assert e == math.floor(math.log2(amax)) - 2, (r, b)
+            step = 2.0 ** e
+            for vv, dd in zip(vb, db):
+                a = abs(vv) / step
+                half = 0.25 if a < 2 else (0.5 if a < 4 else 1.0)
+                lim = max(half, a - 6.0) * step + rel * amax
+                assert abs(dd - vv) <= lim, (r, b, vv, dd, lim)
+
+
+def pin_prepare_weight():
+    rng = np.random.default_rng(8)
+    N, K = 11, 128
+    _, Wb, _ = _exact_rows(rng, N, K)
+    s = np.exp(rng.normal(0, 0.5, K)).astype(np.float32)
+    codes, scales, inv_s = oracle.prepare_weight(Wb, s)
+    assert np.array_equal(inv_s.view(np.uint32), (np.float32(1.0) / s).view(np.uint32))
+    c2, s2 = oracle.quant_rows(Wb, s)
+    assert np.array_equal(codes, c2) and np.array_equal(scales, s2)
+
+
+def pin_scale_layout():
+    K = 32 * 13                                     # 13 blocks -> padded to 16
+    assert oracle.scale_blocks_padded(K) == 16 and oracle.scale_rows_padded(130) == 256
+    assert oracle.scale_rows_padded(128) == 128 and oracle.scale_blocks_padded(256) == 8
+    # hand-derived offsets of the 128 x 4 atom: row r%32 -> 16 B, (r/32)%4 -> 4 B, j%4 -> 1 B
+    cases = {(0, 0): 0, (1, 0): 16, (31, 0): 496, (32, 0): 4, (96, 0): 12, (0, 1): 1,
+             (0, 3): 3, (0, 4): 512, (33, 5): 512 + 16 + 4 + 1, (128, 0): 4 * 512,
+             (200, 9): (1 * 4 + 2) * 512 + (200 % 32) * 16 + 2 * 4 + 1}
+    for (r, j), off in cases.items():
+        assert oracle.scale_offset(r, j, K) == off, (r, j)
+    rows = 130
+    rng = np.random.default_rng(9)
+    rm = rng.integers(1, 255, size=(rows, K // 32)).astype(np.uint8)
+    atom = oracle.swizzle_scales(rm, K)
+    assert atom.size == 256 * 16
+    assert np.array_equal(oracle.unswizzle_scales(atom, rows, K), rm)
+    assert int((atom != 0).sum()) == rm.size         # every padding byte is zero
+
+
+def pin_dequant():
+    table = golden_e2m1()
+    rng = np.random.default_rng(10)
+    rows, K = 3, 64
+    codes = rng.integers(0, 256, size=(rows, K // 2)).astype(np.uint8)
+    scales = rng.integers(100, 150, size=(rows, K // 32)).astype(np.uint8)
+    got = oracle.dequant_rows(codes, scales, K)
+    nib = np.empty((rows, K), np.int64)
+    nib[:, 0::2] = codes & 0xF
+    nib[:, 1::2] = codes >> 4
+    dec = np.vectorize(lambda c: table[int(c)])(nib)
+    expect = np.ldexp(dec, np.repeat(scales.astype(np.int64) - 127, 32, axis=1))
+    assert np.array_equal(got, expect)
+
+
+def pin_gemm():
+    rng = np.random.default_rng(11)
+    M, N, K = 6, 10, 128
+    ac = rng.integers(0, 256, size=(M, K // 2)).astype(np.uint8)
+    as_ = rng.integers(117, 137, size=(M, K // 32)).astype(np.uint8)
+    wc = rng.integers(0, 256, size=(N, K // 2)).astype(np.uint8)
+    ws = rng.integers(117, 137, size=(N, K // 32)).astype(np.uint8)
+    y = oracle.gemm_fp64(ac, as_, wc, ws, K)
+    ref = oracle.dequant_rows(ac, as_, K) @ oracle.dequant_rows(wc, ws, K).T
+    assert np.allclose(y, ref, rtol=1e-12, atol=1e-300)
+    rows = np.array([4, 0, 5], np.int64)
+    assert np.array_equal(oracle.gemm_fp64(ac, as_, wc, ws, K, rows=rows), y[rows])
+    # one-hot: a single code 1.5 (0x3) at k=37 in row 2 against weight code 3.0 (0x5)
+    a1 = np.zeros_like(ac)
+    a1[2, 37 // 2] = 0x3 << 4                           # odd k -> high nibble
+    w1 = np.zeros_like(wc)
+    w1[7, 37 // 2] = 0x5 << 4
+    sa = np.full_like(as_, 127)
+    sa[2, 1] = 127 + 2
+    sw = np.full_like(ws, 127)
+    sw[7, 1] = 127 - 3
+    y1 = oracle.gemm_fp64(a1, sa, w1, sw, K)
+    expect = np.zeros((M, N))
+    expect[2, 7] = 1.5 * 4 * 3.0 * 0.125
+    assert np.array_equal(y1, expect)
+
+
+def pin_storage():
+    K = 4096
+    bits = (K // 2 + K // 32) * 8 / K
+    assert bits == golden_storage_bits()
+
+
+ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]
