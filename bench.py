@@ -1,0 +1,407 @@
+"""Benchmark of the MACaQ W4A4 linear layer on B200.
+
+One step = the whole path on one batch: offline weight preparation (W' = W diag(s) Hb
+-> MXFP4), online activation transform + MXFP4 quantisation, and the block-scaled FP4
+GEMM, on the Llama-3-8B gate/up prefill shape (x 4096x4096, W 14336x4096, bf16 out),
+seeded synthetic inputs resident in HBM. L2 is flushed (256 MiB write) before every
+timed step; each step is timed with CUDA events on the launching stream.
+
+  python bench.py [--gpus N --steps K --warmup W] [--impl reference] [--workload NAME]
+
+Under torchrun (N > 1) every rank runs its own replica of the workload (token rows
+are independent, no data-path collective): weak scaling, value = all ranks' FLOPs /
+max-over-ranks time. Rank 0 prints one JSON line.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+METRIC = "W4A4 linear TFLOPS & quant-kernel GB/s (fraction of B200 roofline)"
+UNIT = "TFLOP/s"
+QUANT_BYTES_PER_ELEM = 2.0 + 0.5 + 1.0 / 32.0      # bf16 in, E2M1 codes + E8M0 scales out
+L2_FLUSH_BYTES = 256 << 20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FP4_OVER_BF16 = 4.0                                   # dense FP4 : BF16 tensor rate on sm_100
+
+
+def workloads_by_name():
+    from mxfp4_w4a4_post_b200 import workloads as wl
+    ws = {L.name: L for L in wl.all_single_layers()}
+    ws.update({L.name: L for L in wl.qwen3_32b_layer_decode(256)})
+    return ws
+
+
+DEFAULT_WORKLOAD = "llama3_8b_gate_up_prefill_4096x14336x4096"
+
+
+def parse_args(argv=None):
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--sample-rows", type=int, default=16, help="oracle sample size (rows of x)")
+    return p.parse_args(argv)
+
+
+# ------------------------------------------------------------------ helpers ---
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def gemm_flops(L):
+    return 2.0 * L.M * L.N * L.K
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def reduce_max(x, device=None):
+    """Max over ranks of a float (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate(flops_per_rank, seconds_max, world):
+    """Whole-job throughput: every rank's work over the slowest rank's time."""
+    return flops_per_rank * world / seconds_max / 1e12
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu_index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100", "-f", self.path],
+                stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+        return False
+
+    def summary(self):
+        out = {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        if not self.path or not os.path.exists(self.path):
+            return out
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower().startswith("active"):
+                        reasons.add(n)
+        os.unlink(self.path)
+        if sm:
+            out = {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                   "samples": len(sm)}
+        return out
+
+
+# ------------------------------------------------------------- our (GPU) arm ---
+
+class DeviceStep:
+    """Preallocated device buffers and the three library calls of one step."""
+
+    def __init__(self, L, x, W, s, device):
+        import torch
+        import mxfp4_w4a4_post_b200 as mq
+        self.mq, self.L, self.dev = mq, L, device
+        to_bf16 = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16)
+        self.x_host = to_bf16(x).pin_memory()
+        self.W_host = to_bf16(W).pin_memory()
+        self.s_host = torch.from_numpy(s).pin_memory()
+        self.x = self.x_host.to(device)
+        self.W = self.W_host.to(device)
+        self.s = self.s_host.to(device)
+        M, N, K = L.M, L.N, L.K
+        self.pw = mq.PreparedWeight(torch.empty((N, K // 2), dtype=torch.uint8, device=device),
+                                    torch.empty(mq.scales_bytes(N, K), dtype=torch.uint8, device=device),
+                                    torch.empty(K, dtype=torch.float32, device=device), N, K)
+        self.a_codes = torch.empty((M, K // 2), dtype=torch.uint8, device=device)
+        self.a_scales = torch.empty(mq.scales_bytes(M, K), dtype=torch.uint8, device=device)
+        self.out_dtype = torch.bfloat16
+        self.y = torch.empty((M, N), dtype=self.out_dtype, device=device)
+        self.y_host = torch.empty((M, N), dtype=self.out_dtype).pin_memory()
+        nws = mq.gemm_workspace_bytes(M, N, K, self.out_dtype)
+        self.ws = torch.empty(max(nws, 256), dtype=torch.uint8, device=device)
+        self.flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+        self.launches_per_step = 3 + (2 if nws > 0 else 0)   # prep, quant, gemm (+ memset, finalize)
+
+    def step(self, ev=None):
+        mq = self.mq
+        if ev:
+            ev[0].record()
+        mq.prepare_weight(self.W, self.s, out=self.pw)
+        if ev:
+            ev[1].record()
+        mq.quant_act(self.x, self.pw.inv_s, self.a_codes, self.a_scales)
+        if ev:
+            ev[2].record()
+        mq.gemm_mxfp4(self.a_codes, self.a_scales, self.L.M, self.pw, y=self.y, workspace=self.ws)
+        if ev:
+            ev[3].record()
+
+    def step_e2e(self):
+        """The same step from pinned host buffers, host<->device copies included."""
+        self.x.copy_(self.x_host, non_blocking=True)
+        self.W.copy_(self.W_host, non_blocking=True)
+        self.s.copy_(self.s_host, non_blocking=True)
+        self.step()
+        self.y_host.copy_(self.y, non_blocking=True)
+
+    def h2d_bytes(self):
+        return self.x.numel() * 2 + self.W.numel() * 2 + self.s.numel() * 4
+
+    def d2h_bytes(self):
+        return self.y.numel() * self.y.element_size()
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    import mxfp4_w4a4_post_b200 as mq
+    from mxfp4_w4a4_post_b200 import workloads as wl
+
+    rank, world, local = dist_env()
+    if world > 1:
+        from datetime import timedelta
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+    device = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(device)
+    mq.lib()
+    L = workloads_by_name()[args.workload]
+    x, W, s = wl.draw_x(L), wl.draw_W(L), wl.draw_s(L)
+    st = DeviceStep(L, x, W, s, device)
+    stream = torch.cuda.current_stream(device)
+
+    for _ in range(max(args.warmup, 3)):
+        st.flush.fill_(1)
+        st.step()
+    torch.cuda.synchronize(device)
+    if mq.device_error() != 0:
+        raise RuntimeError("device error word set during warm-up")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(device)
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        for i in range(args.steps):
+            st.flush.fill_(i & 0xFF)              # evict L2 before the step (untimed)
+            st.step(evs[i])
+        torch.cuda.synchronize(device)
+    if world > 1:
+        dist.barrier()
+    assert mq.device_error() == 0
+
+    t_step = [evs[i][0].elapsed_time(evs[i][3]) * 1e-3 for i in range(args.steps)]
+    t_prep = [evs[i][0].elapsed_time(evs[i][1]) * 1e-3 for i in range(args.steps)]
+    t_quant = [evs[i][1].elapsed_time(evs[i][2]) * 1e-3 for i in range(args.steps)]
+    t_gemm = [evs[i][2].elapsed_time(evs[i][3]) * 1e-3 for i in range(args.steps)]
+    total = reduce_max(sum(t_step), device)
+    sec_per_step = total / args.steps
+    value = aggregate(gemm_flops(L), sec_per_step, world)
+
+    peaks, peak_src = load_peaks()
+    fp4_peak = peaks["bf16_tflops"] * FP4_OVER_BF16
+    g_avg = reduce_max(statistics.mean(t_gemm), device)
+    q_avg = reduce_max(statistics.mean(t_quant), device)
+    p_avg = reduce_max(statistics.mean(t_prep), device)
+    gemm_tflops = gemm_flops(L) / g_avg / 1e12
+    q_bytes = QUANT_BYTES_PER_ELEM * L.M * L.K + 4 * L.K
+    p_bytes = QUANT_BYTES_PER_ELEM * L.N * L.K + 8 * L.K
+    q_gbs = q_bytes / q_avg / 1e9
+    p_gbs = p_bytes / p_avg / 1e9
+
+    e2e = None
+    if not args.no_e2e:
+        for _ in range(2):
+            st.step_e2e()
+        torch.cuda.synchronize(device)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n_e2e = max(3, min(args.steps, 10))
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(device)
+        e0.record(stream)
+        for _ in range(n_e2e):
+            st.step_e2e()
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        t_e2e = reduce_max(e0.elapsed_time(e1) * 1e-3 / n_e2e, device)
+        e2e = {"value": aggregate(gemm_flops(L), t_e2e, world), "unit": UNIT,
+               "h2d_bytes_per_step": st.h2d_bytes(), "d2h_bytes_per_step": st.d2h_bytes(),
+               "ms_per_step": t_e2e * 1e3, "path": "pinned host x, W, s -> C ABI calls -> pinned host y"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(L, x, W, s, args.sample_rows)
+
+    result = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": max(args.warmup, 3), "ms_per_step": sec_per_step * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "mxfp4 (e2m1 x e2m1, e8m0 scales, f32 accumulate); transform in f32",
+        "data": "synthetic (seeded; Student-t(3) activations with 0.5% x20 outlier channels, N(0,0.02) weights)",
+        "config": {"workload": L.name, "M": L.M, "N": L.N, "K": L.K, "out_dtype": "bf16",
+                   "step": "prepare_weight + quant_act + gemm_mxfp4",
+                   "l2": f"flushed before every timed step ({L2_FLUSH_BYTES >> 20} MiB write)",
+                   "parallelism": f"replicas x{world}"},
+        "roofline": {"bound": "tensor", "achieved": gemm_tflops, "peak": fp4_peak, "unit": "TFLOP/s",
+                     "frac": gemm_tflops / fp4_peak, "traffic": None,
+                     "kernel": "gemm_mxf4_kernel",
+                     "peak_source": f"{peak_src} bf16 burst x {FP4_OVER_BF16:g} (dense FP4:BF16 rate)"},
+        "kernels": {
+            "gemm_mxfp4": {"us": g_avg * 1e6, "tflops": gemm_tflops, "frac_fp4_peak": gemm_tflops / fp4_peak},
+            "quant_act": {"us": q_avg * 1e6, "gbs": q_gbs, "frac_hbm": q_gbs / peaks["hbm_gbs"],
+                          "bytes": q_bytes},
+            "prepare_weight": {"us": p_avg * 1e6, "gbs": p_gbs, "frac_hbm": p_gbs / peaks["hbm_gbs"],
+                               "bytes": p_bytes},
+            "quant_over_gemm": q_avg / g_avg,
+            "hbm_peak_gbs": peaks["hbm_gbs"],
+        },
+        "e2e": e2e,
+        "cpu_baseline": cpu,
+        "gpu_launches": st.launches_per_step * args.steps,
+        "clocks": clk.summary(),
+    }
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    return result
+
+
+# ----------------------------------------------------------- oracle (CPU) ----
+
+def oracle_sample(L, x, W_codes_full, W_scales_full, W, s, rows, prep_rows):
+    """One bounded sample of the step on the host cores: weight preparation of
+    `prep_rows` rows of W (the sample's share), quantisation of `rows` rows of x and
+    their fp64 GEMM against the full prepared weight. Returns seconds."""
+    import oracle
+    t0 = time.perf_counter()
+    oracle.prepare_weight(W[:prep_rows], s)
+    inv_s = (np.float32(1.0) / s).astype(np.float32)
+    ac, as_ = oracle.quant_rows(x[:rows], inv_s)
+    oracle.gemm_fp64(ac, as_, W_codes_full, W_scales_full, L.K)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(L, x, W, s, rows):
+    import oracle
+    wc, ws, _ = oracle.prepare_weight(W, s)
+    prep_rows = max(1, int(round(L.N * rows / L.M)))
+    t = oracle_sample(L, x, wc, ws, W, s, rows, prep_rows)
+    flops = 2.0 * rows * L.N * L.K
+    return {"value": flops / t / 1e12, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"{rows} of {L.M} rows of x (quantise + fp64 GEMM against all {L.N} prepared "
+                      f"weight rows) plus the matching {prep_rows}-row share of the weight preparation; "
+                      f"single-threaded C, {t:.1f} s"}
+
+
+def run_reference(args):
+    import torch.distributed as dist  # noqa: F401
+    from mxfp4_w4a4_post_b200 import workloads as wl
+    import oracle
+
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return None
+    L = workloads_by_name()[args.workload]
+    x, W, s = wl.draw_x(L, rows=args.sample_rows), wl.draw_W(L), wl.draw_s(L)
+    wc, ws, _ = oracle.prepare_weight(W, s)
+    prep_rows = max(1, int(round(L.N * args.sample_rows / L.M)))
+    for _ in range(args.warmup):
+        oracle_sample(L, x, wc, ws, W, s, args.sample_rows, prep_rows)
+    times = [oracle_sample(L, x, wc, ws, W, s, args.sample_rows, prep_rows) for _ in range(args.steps)]
+    t = sum(times) / len(times)
+    flops = 2.0 * args.sample_rows * L.N * L.K
+    value = flops / t / 1e12
+    sample = (f"{args.sample_rows} of {L.M} rows of x per step (quantise + fp64 GEMM against all {L.N} "
+              f"prepared weight rows) plus the matching {prep_rows}-row share of the weight preparation")
+    result = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32 transform, f64 GEMM", "data": "synthetic (seeded)",
+        "config": {"workload": L.name, "M": L.M, "N": L.N, "K": L.K, "out_dtype": "f64",
+                   "step": "prepare_weight + quant_act + gemm (bounded row sample)"},
+        "impl": "reference",
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(result), flush=True)
+    return result
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

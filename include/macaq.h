@@ -1,0 +1,170 @@
+/*
+ * libmacaq: MACaQ W4A4 linear layer on NVIDIA B200 (sm_100a), C ABI.
+ *
+ * The layer (MACaQ pages: zicq.com "MACaQ Enables Streaming W4A4 Quantization",
+ * section "Quantization mechanism", equation y = xW^T and its transformed form;
+ * abstract on the Hugging Face papers mirror; openai-hub.com "华为开源MACaQ",
+ * paragraphs on MXFP4 and on the 32-element block Hadamard rotation):
+ *
+ *     y = x W^T = (x D^-1 Hb) (Hb D W^T),   D = diag(s),
+ *
+ * Hb block-diagonal with 32x32 Sylvester Hadamard blocks scaled by 1/sqrt(32), the
+ * blocks aligned with the 32-element MXFP4 groups. The weight factor Hb D W^T is
+ * computed once, ahead of inference; at inference the activation is scaled, rotated
+ * and quantised online, then both MXFP4 operands meet in a block-scaled FP4 GEMM.
+ *
+ * Conventions shared by every entry point:
+ *  - Pointers marked "device" are CUDA device pointers of the current device; the
+ *    caller allocates and owns every buffer. The library allocates no memory and keeps
+ *    no state apart from one device-side error word per device.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default stream).
+ *    A returned MACAQ_OK means the work was validated and enqueued.
+ *  - Arguments are validated on the host before any launch; a failed check returns an
+ *    error code and enqueues nothing. Nothing throws or aborts across the ABI.
+ *  - Only devices of compute capability 10.0 (B200, sm_100a) are supported.
+ *  - Inputs must be finite, and scaled/rotated values must stay finite in fp32;
+ *    anything else is out of contract.
+ *
+ * MXFP4 storage, 4.25 bits per element (the storage figure per weight in the
+ * openai-hub.com article's FLUX comparison paragraph):
+ *  - codes : rows x K/2 bytes, row stride K/2; element 2j of a row in the low nibble of
+ *            byte j; E2M1 code = sign<<3 | {0,.5,1,1.5,2,3,4,6} index.
+ *  - scales: E8M0 bytes (value 2^(byte-127)), one per 32 elements, in the tensor-core
+ *            atom layout: rows padded to a multiple of 128, scale blocks per row
+ *            padded to a multiple of 8; scale (r, j) at byte
+ *              ((r/128) * (Kb_pad/4) + j/4) * 512 + (r%32)*16 + ((r/32)%4)*4 + j%4
+ *            with Kb_pad = round_up(K/32, 8). Padding bytes are 0.
+ */
+#ifndef MACAQ_H
+#define MACAQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MACAQ_VERSION 1
+
+/* Same object as cudaStream_t, declared without the CUDA headers. */
+typedef struct CUstream_st* macaq_stream;
+
+typedef enum {
+    MACAQ_OK = 0,
+    MACAQ_ERR_INVALID_ARG = 1,        /* null pointer, non-positive size, bad enum */
+    MACAQ_ERR_MISALIGNED = 2,         /* pointer or leading dimension not aligned */
+    MACAQ_ERR_UNSUPPORTED_SHAPE = 3,  /* K % 32 != 0, sizes beyond the documented limits */
+    MACAQ_ERR_UNSUPPORTED_DEVICE = 4, /* current device is not compute capability 10.0 */
+    MACAQ_ERR_CUDA = 5,               /* a CUDA runtime/driver call or launch failed */
+    MACAQ_ERR_DEVICE_TIMEOUT = 6,     /* a kernel gave up a bounded wait (see below) */
+    MACAQ_ERR_WORKSPACE = 7,          /* workspace pointer null or smaller than required */
+    MACAQ_ERR_UNSUPPORTED = 8         /* a documented option that is not built */
+} macaq_status;
+
+typedef enum { MACAQ_OUT_F32 = 0, MACAQ_OUT_BF16 = 1 } macaq_out_dtype;
+
+/* Prepared weight (the offline artefact): codes/scales of W' = W D Hb, plus the
+ * activation multiplier inv_s = 1/s. All three device pointers, owned by the caller. */
+typedef struct {
+    const uint8_t* codes;  /* device, N x K/2 bytes, 16-byte aligned */
+    const uint8_t* scales; /* device, macaq_scales_bytes(N, K) bytes, 16-byte aligned */
+    const float* inv_s;    /* device, K floats, 16-byte aligned */
+    int64_t N;             /* output features */
+    int64_t K;             /* input features, multiple of 32 */
+} macaq_weight;
+
+/* ------------------------------------------------------------- sizes ---------- */
+
+/* Bytes of the packed E2M1 codes of a rows x K matrix: rows * K / 2. */
+size_t macaq_codes_bytes(int64_t rows, int64_t K);
+
+/* Bytes of the padded scale layout of a rows x K matrix:
+ * round_up(rows, 128) * round_up(K/32, 8). */
+size_t macaq_scales_bytes(int64_t rows, int64_t K);
+
+/* Device workspace macaq_gemm_mxfp4 needs for an M x N x K product with output
+ * `out` (an fp32 split-K accumulator when the library splits K; may be 0). */
+size_t macaq_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, macaq_out_dtype out);
+
+/* Device workspace macaq_linear_w4a4 needs: the activation codes and scales, plus
+ * the GEMM workspace, each 256-byte aligned inside the block. */
+size_t macaq_linear_workspace_bytes(int64_t M, int64_t N, int64_t K, macaq_out_dtype out);
+
+/* ------------------------------------------------------------ compute --------- */
+
+/* Offline weight preparation (pages: the weight factor is folded in before
+ * quantisation; round-to-nearest baseline of the ablation in the openai-hub.com
+ * article). For each row n of W: w = fp32(W[n,:]) * s (fp32, per channel), then per
+ * 32-block the normalised Hadamard butterfly, the E8M0 exponent
+ * e = max(floor(log2 amax) - 2, -127) and round-to-nearest-even E2M1 codes.
+ * Also writes inv_s[k] = 1.0f / s[k] (IEEE fp32 division).
+ *   W_bf16    device bf16 [N x K], row stride ldw elements (ldw >= K, ldw % 8 == 0),
+ *             16-byte aligned
+ *   s         device fp32 [K], 16-byte aligned, finite and non-zero
+ *   w_codes   device, macaq_codes_bytes(N, K), 16-byte aligned
+ *   w_scales  device, macaq_scales_bytes(N, K), 16-byte aligned (padding written 0)
+ *   inv_s_out device fp32 [K], 16-byte aligned
+ * K % 32 == 0, N >= 1. */
+macaq_status macaq_prepare_weight(const void* W_bf16, int64_t N, int64_t K, int64_t ldw,
+                                  const float* s, uint8_t* w_codes, uint8_t* w_scales,
+                                  float* inv_s_out, macaq_stream stream);
+
+/* Online activation transform (pages: per-channel scale and block Hadamard applied
+ * online to each layer's activation, then MXFP4): for each row m,
+ * u = fp32(x[m,:]) * inv_s, then the same block transform and encoding as above.
+ *   x_bf16   device bf16 [M x K], row stride ldx elements (ldx >= K, ldx % 8 == 0),
+ *            16-byte aligned
+ *   inv_s    device fp32 [K] (normally macaq_weight.inv_s), 16-byte aligned
+ *   a_codes  device, macaq_codes_bytes(M, K); a_scales device, macaq_scales_bytes(M, K)
+ * Results are bit-identical to the CPU definition for every finite input. */
+macaq_status macaq_quant_act(const void* x_bf16, int64_t M, int64_t K, int64_t ldx,
+                             const float* inv_s, uint8_t* a_codes, uint8_t* a_scales,
+                             macaq_stream stream);
+
+/* Block-scaled FP4 GEMM on pre-quantised operands (pages: the FP4 matrix product
+ * that follows the activation transform; W4A4 definition in the openai-hub.com
+ * article):
+ *   y[m, n] = sum_b 2^(ea[m,b] + ew[n,b]) * sum_{k in b} dec(a[m,k]) * dec(w[n,k]),
+ * fp32 accumulation on the tensor cores (tcgen05 kind::mxf4).
+ *   a_codes/a_scales device, as written by macaq_quant_act for M rows
+ *   w        prepared weight (inv_s unused here)
+ *   y        device [M x N] fp32 or bf16, row stride ldy elements (ldy >= N), aligned
+ *            to its element size (16-byte alignment of y and of ldy * element size
+ *            enables vector stores)
+ *   workspace device, >= macaq_gemm_workspace_bytes(M, N, K, out), 256-byte aligned
+ *            (may be NULL when that size is 0); contents are scratch
+ * M >= 1. Also the entry point for externally refined weight codes/scales. */
+macaq_status macaq_gemm_mxfp4(const uint8_t* a_codes, const uint8_t* a_scales, int64_t M,
+                              const macaq_weight* w, void* y, int64_t ldy, macaq_out_dtype out,
+                              void* workspace, size_t ws_bytes, macaq_stream stream);
+
+/* The whole online layer: macaq_quant_act into the workspace, then macaq_gemm_mxfp4.
+ *   fused     must be 0 (a variant quantising inside the GEMM producer is not built;
+ *             nonzero returns MACAQ_ERR_UNSUPPORTED)
+ *   workspace device, >= macaq_linear_workspace_bytes(M, N, K, out), 256-byte aligned
+ * Other arguments as for macaq_quant_act / macaq_gemm_mxfp4. */
+macaq_status macaq_linear_w4a4(const void* x_bf16, int64_t M, int64_t ldx, const macaq_weight* w,
+                               void* y, int64_t ldy, macaq_out_dtype out, int fused,
+                               void* workspace, size_t ws_bytes, macaq_stream stream);
+
+/* ------------------------------------------------------------ status ---------- */
+
+/* Every wait inside the GEMM kernel is bounded. A kernel that gives up a wait records
+ * a code in a device-side word and returns early (its output is then undefined).
+ * This call synchronises the current device, reads the word, clears it, and returns
+ * MACAQ_ERR_DEVICE_TIMEOUT if it was set (MACAQ_OK otherwise, MACAQ_ERR_CUDA if the
+ * read fails). */
+macaq_status macaq_get_device_error(void);
+
+/* Static, human-readable name of a status code. */
+const char* macaq_status_string(macaq_status status);
+
+/* MACAQ_VERSION of the built library. */
+int macaq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MACAQ_H */

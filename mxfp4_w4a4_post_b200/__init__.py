@@ -1,0 +1,221 @@
+"""MACaQ W4A4 linear layer (MXFP4) on NVIDIA B200: thin Python binding of libmacaq.
+
+Every step of the layer runs in the CUDA kernels behind the C ABI declared in
+include/macaq.h; this module only marshals torch tensors (device memory and the
+current stream) into those calls. There is no CPU fallback: if the library is missing
+or the device is not a B200, calls raise.
+
+    w = prepare_weight(W_bf16, s)          # offline: W' = W diag(s) Hb -> MXFP4
+    y = linear(x_bf16, w)                  # online: x diag(s)^-1 Hb -> MXFP4 -> FP4 GEMM
+"""
+import ctypes
+import os
+from dataclasses import dataclass
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmacaq.so")
+
+MACAQ_OK = 0
+OUT_F32 = 0
+OUT_BF16 = 1
+
+STATUS_NAMES = {
+    0: "MACAQ_OK", 1: "MACAQ_ERR_INVALID_ARG", 2: "MACAQ_ERR_MISALIGNED",
+    3: "MACAQ_ERR_UNSUPPORTED_SHAPE", 4: "MACAQ_ERR_UNSUPPORTED_DEVICE", 5: "MACAQ_ERR_CUDA",
+    6: "MACAQ_ERR_DEVICE_TIMEOUT", 7: "MACAQ_ERR_WORKSPACE", 8: "MACAQ_ERR_UNSUPPORTED",
+}
+
+
+class MacaqError(RuntimeError):
+    def __init__(self, status, what=""):
+        self.status = status
+        super().__init__(f"{what}: {STATUS_NAMES.get(status, status)}")
+
+
+class MacaqWeight(ctypes.Structure):
+    _fields_ = [("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("inv_s", ctypes.c_void_p),
+                ("N", ctypes.c_int64), ("K", ctypes.c_int64)]
+
+
+_lib = None
+
+
+def lib():
+    """The loaded libmacaq.so (ctypes), with argument types declared."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libmacaq.so not built ({LIB_PATH}); run __graft_entry__.build()")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I64, SZ, I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t, ctypes.c_int
+        sig = {
+            "macaq_codes_bytes": (SZ, [I64, I64]),
+            "macaq_scales_bytes": (SZ, [I64, I64]),
+            "macaq_gemm_workspace_bytes": (SZ, [I64, I64, I64, I]),
+            "macaq_linear_workspace_bytes": (SZ, [I64, I64, I64, I]),
+            "macaq_prepare_weight": (I, [P, I64, I64, I64, P, P, P, P, P]),
+            "macaq_quant_act": (I, [P, I64, I64, I64, P, P, P, P]),
+            "macaq_gemm_mxfp4": (I, [P, P, I64, ctypes.POINTER(MacaqWeight), P, I64, I, P, SZ, P]),
+            "macaq_linear_w4a4": (I, [P, I64, I64, ctypes.POINTER(MacaqWeight), P, I64, I, I, P, SZ, P]),
+            "macaq_get_device_error": (I, []),
+            "macaq_status_string": (ctypes.c_char_p, [I]),
+            "macaq_version": (I, []),
+        }
+        for name, (res, args) in sig.items():
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _check(status, what):
+    if status != MACAQ_OK:
+        raise MacaqError(status, what)
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def _stream_ptr(device):
+    torch = _torch()
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _out_code(dtype):
+    torch = _torch()
+    if dtype == torch.float32:
+        return OUT_F32
+    if dtype == torch.bfloat16:
+        return OUT_BF16
+    raise ValueError(f"unsupported output dtype {dtype}")
+
+
+def codes_bytes(rows, K):
+    return lib().macaq_codes_bytes(rows, K)
+
+
+def scales_bytes(rows, K):
+    return lib().macaq_scales_bytes(rows, K)
+
+
+def linear_workspace_bytes(M, N, K, out_dtype=None):
+    torch = _torch()
+    return lib().macaq_linear_workspace_bytes(M, N, K, _out_code(out_dtype or torch.bfloat16))
+
+
+def gemm_workspace_bytes(M, N, K, out_dtype=None):
+    torch = _torch()
+    return lib().macaq_gemm_workspace_bytes(M, N, K, _out_code(out_dtype or torch.bfloat16))
+
+
+@dataclass
+class PreparedWeight:
+    """Offline artefact: MXFP4 codes/scales of W' = W diag(s) Hb, and inv_s = 1/s."""
+    codes: "object"    # uint8 [N, K/2]
+    scales: "object"   # uint8 [scales_bytes(N, K)] (tensor-core atom layout)
+    inv_s: "object"    # float32 [K]
+    N: int
+    K: int
+
+    def c_struct(self):
+        return MacaqWeight(self.codes.data_ptr(), self.scales.data_ptr(), self.inv_s.data_ptr(),
+                           self.N, self.K)
+
+
+def _require(t, dtype, name):
+    torch = _torch()
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.dim() == 2 and t.stride(1) != 1:
+        raise ValueError(f"{name} must have unit stride along its last dimension")
+
+
+def prepare_weight(W, s, out=None):
+    """W: bf16 [N, K] CUDA tensor (row stride W.stride(0)); s: fp32 [K]."""
+    torch = _torch()
+    _require(W, torch.bfloat16, "W")
+    _require(s, torch.float32, "s")
+    N, K = W.shape
+    dev = W.device
+    if out is None:
+        out = PreparedWeight(torch.empty((N, K // 2), dtype=torch.uint8, device=dev),
+                             torch.empty(scales_bytes(N, K), dtype=torch.uint8, device=dev),
+                             torch.empty(K, dtype=torch.float32, device=dev), N, K)
+    st = lib().macaq_prepare_weight(W.data_ptr(), N, K, W.stride(0), s.data_ptr(), out.codes.data_ptr(),
+                                    out.scales.data_ptr(), out.inv_s.data_ptr(), _stream_ptr(dev))
+    _check(st, "macaq_prepare_weight")
+    return out
+
+
+def quant_act(x, inv_s, codes=None, scales=None):
+    """x: bf16 [M, K]; inv_s: fp32 [K]. Returns (codes uint8 [M, K/2], scales uint8)."""
+    torch = _torch()
+    _require(x, torch.bfloat16, "x")
+    _require(inv_s, torch.float32, "inv_s")
+    M, K = x.shape
+    dev = x.device
+    if codes is None:
+        codes = torch.empty((M, K // 2), dtype=torch.uint8, device=dev)
+    if scales is None:
+        scales = torch.empty(scales_bytes(M, K), dtype=torch.uint8, device=dev)
+    st = lib().macaq_quant_act(x.data_ptr(), M, K, x.stride(0), inv_s.data_ptr(), codes.data_ptr(),
+                               scales.data_ptr(), _stream_ptr(dev))
+    _check(st, "macaq_quant_act")
+    return codes, scales
+
+
+def _workspace(nbytes, device, workspace):
+    torch = _torch()
+    if nbytes == 0:
+        return None, 0
+    if workspace is not None and workspace.numel() >= nbytes:
+        return workspace, workspace.numel()
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=device)
+    return ws, nbytes
+
+
+def gemm_mxfp4(a_codes, a_scales, M, w, out_dtype=None, y=None, workspace=None):
+    """Block-scaled FP4 GEMM on pre-quantised activations: y = A W'^T."""
+    torch = _torch()
+    out_dtype = out_dtype or torch.bfloat16
+    dev = a_codes.device
+    if y is None:
+        y = torch.empty((M, w.N), dtype=out_dtype, device=dev)
+    need = gemm_workspace_bytes(M, w.N, w.K, out_dtype)
+    ws, ws_bytes = _workspace(need, dev, workspace)
+    cw = w.c_struct()
+    st = lib().macaq_gemm_mxfp4(a_codes.data_ptr(), a_scales.data_ptr(), M, ctypes.byref(cw), y.data_ptr(),
+                                y.stride(0), _out_code(y.dtype), ws.data_ptr() if ws is not None else None,
+                                ws_bytes, _stream_ptr(dev))
+    _check(st, "macaq_gemm_mxfp4")
+    return y
+
+
+def linear(x, w, out_dtype=None, y=None, workspace=None):
+    """The MACaQ W4A4 layer: y = x W^T computed as (x diag(s)^-1 Hb)(Hb diag(s) W^T) in MXFP4."""
+    torch = _torch()
+    _require(x, torch.bfloat16, "x")
+    out_dtype = out_dtype or torch.bfloat16
+    M, K = x.shape
+    if K != w.K:
+        raise ValueError(f"x has K={K}, weight has K={w.K}")
+    dev = x.device
+    if y is None:
+        y = torch.empty((M, w.N), dtype=out_dtype, device=dev)
+    need = linear_workspace_bytes(M, w.N, K, y.dtype)
+    ws, ws_bytes = _workspace(need, dev, workspace)
+    cw = w.c_struct()
+    st = lib().macaq_linear_w4a4(x.data_ptr(), M, x.stride(0), ctypes.byref(cw), y.data_ptr(), y.stride(0),
+                                 _out_code(y.dtype), 0, ws.data_ptr(), ws_bytes, _stream_ptr(dev))
+    _check(st, "macaq_linear_w4a4")
+    return y
+
+
+def device_error():
+    """Synchronise, read and clear the device error word (MACAQ_OK or a timeout)."""
+    return lib().macaq_get_device_error()

@@ -1,0 +1,435 @@
+// Block-scaled FP4 GEMM for the MACaQ W4A4 layer on Blackwell tensor cores (sm_100a).
+//
+//   D[p, q] = sum_b 2^(e_P[p,b] + e_Q[q,b]) * sum_{k in block b} dec(P[p,k]) dec(Q[q,k])
+//
+// P (the "M-slot" operand, 128-row tiles) and Q (the "N-slot" operand, BN-row tiles)
+// are MXFP4: packed E2M1 codes, K-major, plus E8M0 scales in the 128x4 atom layout.
+// For prefill P = activations and Q = weights, D = y. For decode the roles swap
+// (P = weights, so the 128-wide MMA M dimension covers output features and the few
+// tokens become the MMA N dimension), and the epilogue writes D transposed.
+//
+// One persistent CTA per SM, warp-specialised:
+//   warp 0      TMA producer: codes via 2D tensor maps with the 128-byte swizzle (one
+//               256-element K tile = 128 bytes per row), scale atoms via bulk copies
+//   warp 1      TMEM owner and single-thread MMA issuer: tcgen05.cp moves the scale
+//               atoms SMEM -> TMEM, then four tcgen05.mma kind::mxf4.block_scale
+//               (K = 64 each) per K tile into an fp32 TMEM accumulator
+//   warps 2-5   epilogue: tcgen05.ld the accumulator (each warp owns one 32-lane TMEM
+//               subpartition), convert, store (or fp32 reduce for split K)
+// Accumulators are double-buffered in TMEM when they fit, so the epilogue of one tile
+// overlaps the MMAs of the next. Every mbarrier wait is bounded by a wall-clock limit;
+// a kernel that gives up records an error code, drains what it issued, frees its TMEM
+// and returns.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "ptx_sm100.cuh"
+
+namespace macaq {
+
+struct GemmParams {
+    const uint8_t* sf_p;     // scale atoms of P
+    const uint8_t* sf_q;     // scale atoms of Q
+    void* out;               // output, or the fp32 accumulator when atomic
+    int64_t ldo;             // leading dimension of out, elements
+    int32_t p_rows, q_rows;  // logical rows of P and Q
+    int32_t k_tiles;         // ceil(K / 256)
+    int32_t kb4_pad;         // scale atoms per 128-row slab along K
+    int32_t tiles_p, tiles_q;
+    int32_t splits, k_tiles_per_split;
+    int32_t total_units;     // tiles_p * tiles_q * splits
+    int32_t group_p;         // raster group height (in P tiles)
+    int32_t out_bf16;        // 1: bf16 output, 0: fp32 (ignored when atomic)
+    int32_t atomic;          // 1: fp32 reduction into out (split K)
+    int32_t transpose_out;   // 1: out[q * ldo + p], 0: out[p * ldo + q]
+    int32_t vec_ok;          // 1: out and ldo allow 16-byte vector stores
+    int* err;                // device error word
+};
+
+enum : int { kErrTimeoutProducer = 1, kErrTimeoutMma = 2, kErrTimeoutEpilogue = 3, kErrSfOffset = 4 };
+
+template <int BN>
+struct GemmShape {
+    // Q tiles start on a 64-row boundary of the 128-row scale slabs (offset 0 or 2 TMEM
+    // columns), the only scale-factor column offsets the MMA is given.
+    static_assert(BN == 16 || BN == 32 || BN == 64 || BN == 128 || BN == 192 || BN == 256,
+                  "unsupported tile width");
+    static constexpr int kBM = 128;
+    static constexpr int kBKBytes = 128;                    // 256 FP4 elements per row
+    static constexpr int kPTileBytes = kBM * kBKBytes;      // 16 KB
+    static constexpr int kQTileBytes = BN * kBKBytes;
+    static constexpr int kSfChunkBytes = 1024;              // 128 rows x 8 scale blocks
+    // 128-row scale slabs a Q tile can touch (a 192-row tile may start 64 rows into one)
+    static constexpr int kQChunks = (BN <= 128) ? 1 : 2;
+    static constexpr int kSfCols = 8 + 8 * kQChunks;        // 4 columns per atom, 2 atoms per tile
+    static constexpr int kAccStride = (BN == 192) ? 256 : BN;
+    static constexpr int kNumAcc = (BN + kAccStride + kSfCols <= 512) ? 2 : 1;
+    static constexpr int kSfBase = (kNumAcc - 1) * kAccStride + BN;
+    static constexpr int kTmemNeed = kSfBase + kSfCols;
+    static constexpr int kTmemCols = kTmemNeed <= 32 ? 32 : kTmemNeed <= 64 ? 64
+                                   : kTmemNeed <= 128 ? 128 : kTmemNeed <= 256 ? 256 : 512;
+    static constexpr int kChunkCols = BN < 32 ? BN : 32;    // epilogue TMEM load width
+};
+
+template <int BN, int STAGES>
+struct GemmSmem {
+    using S = GemmShape<BN>;
+    static constexpr int kOffP = 0;
+    static constexpr int kOffQ = kOffP + STAGES * S::kPTileBytes;
+    static constexpr int kOffSfP = kOffQ + STAGES * S::kQTileBytes;
+    static constexpr int kOffSfQ = kOffSfP + STAGES * S::kSfChunkBytes;
+    static constexpr int kOffBar = kOffSfQ + STAGES * S::kQChunks * S::kSfChunkBytes;
+    static constexpr int kNumBars = 2 * STAGES + 4 + 1;
+    static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+    static constexpr int kBytes = kOffMisc + 16;
+    static constexpr int kAlloc = kBytes + 1024;            // slack to align the base to 1 KB
+};
+
+__device__ __forceinline__ uint64_t global_timer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Wait for `parity` on `bar`, giving up after ~2 s (or as soon as another role of the
+// CTA has given up). On give-up record `code`, raise the CTA abort flag, return false.
+__device__ __noinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                           int* err, int code) {
+    if (ptx::mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t it = 0;; ++it) {
+        if (ptx::mbar_try_wait(bar, parity)) return true;
+        if ((it & 63) == 63) {
+            if (*abort) return false;
+            if (global_timer_ns() - t0 > 2000000000ull) {
+                atomicExch(err, code);
+                *abort = 1;
+                return false;
+            }
+        }
+        __nanosleep(32);
+    }
+}
+
+struct Unit {
+    int tp, tq, kt_begin, kt_end;
+};
+
+__device__ __forceinline__ Unit decode_unit(const GemmParams& p, int u) {
+    const int tile = u / p.splits;
+    const int split = u - tile * p.splits;
+    const int per_group = p.group_p * p.tiles_q;
+    const int g = tile / per_group;
+    const int r = tile - g * per_group;
+    const int gp = min(p.group_p, p.tiles_p - g * p.group_p);
+    Unit x;
+    x.tp = g * p.group_p + r % gp;
+    x.tq = r / gp;
+    x.kt_begin = split * p.k_tiles_per_split;
+    x.kt_end = min(p.k_tiles, x.kt_begin + p.k_tiles_per_split);
+    return x;
+}
+
+template <int BN>
+__device__ __forceinline__ void store_chunk(const GemmParams& p, int prow, int q_base,
+                                            const uint32_t (&r)[GemmShape<BN>::kChunkCols]) {
+    constexpr int CW = GemmShape<BN>::kChunkCols;
+    if (prow >= p.p_rows) return;
+    if (p.transpose_out) {
+        // out[q, prow]: for each column the 32 lanes of the warp write consecutive prow
+        if (p.atomic) {
+            float* o = reinterpret_cast<float*>(p.out);
+#pragma unroll
+            for (int j = 0; j < CW; ++j) {
+                const int q = q_base + j;
+                if (q < p.q_rows) atomicAdd(o + (int64_t)q * p.ldo + prow, __uint_as_float(r[j]));
+            }
+        } else if (p.out_bf16) {
+            __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(p.out);
+#pragma unroll
+            for (int j = 0; j < CW; ++j) {
+                const int q = q_base + j;
+                if (q < p.q_rows) o[(int64_t)q * p.ldo + prow] = __float2bfloat16_rn(__uint_as_float(r[j]));
+            }
+        } else {
+            float* o = reinterpret_cast<float*>(p.out);
+#pragma unroll
+            for (int j = 0; j < CW; ++j) {
+                const int q = q_base + j;
+                if (q < p.q_rows) o[(int64_t)q * p.ldo + prow] = __uint_as_float(r[j]);
+            }
+        }
+        return;
+    }
+    const bool full = q_base + CW <= p.q_rows && p.vec_ok;
+    if (p.atomic) {
+        float* o = reinterpret_cast<float*>(p.out) + (int64_t)prow * p.ldo + q_base;
+        if (full) {
+#pragma unroll
+            for (int j = 0; j < CW; j += 4)
+                atomicAdd(reinterpret_cast<float4*>(o + j),
+                          make_float4(__uint_as_float(r[j]), __uint_as_float(r[j + 1]),
+                                      __uint_as_float(r[j + 2]), __uint_as_float(r[j + 3])));
+        } else {
+#pragma unroll
+            for (int j = 0; j < CW; ++j)
+                if (q_base + j < p.q_rows) atomicAdd(o + j, __uint_as_float(r[j]));
+        }
+    } else if (p.out_bf16) {
+        __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(p.out) + (int64_t)prow * p.ldo + q_base;
+        if (full) {
+#pragma unroll
+            for (int j = 0; j < CW; j += 8) {
+                uint4 v;
+                __nv_bfloat162 h0 = __floats2bfloat162_rn(__uint_as_float(r[j + 0]), __uint_as_float(r[j + 1]));
+                __nv_bfloat162 h1 = __floats2bfloat162_rn(__uint_as_float(r[j + 2]), __uint_as_float(r[j + 3]));
+                __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(r[j + 4]), __uint_as_float(r[j + 5]));
+                __nv_bfloat162 h3 = __floats2bfloat162_rn(__uint_as_float(r[j + 6]), __uint_as_float(r[j + 7]));
+                v.x = *reinterpret_cast<uint32_t*>(&h0);
+                v.y = *reinterpret_cast<uint32_t*>(&h1);
+                v.z = *reinterpret_cast<uint32_t*>(&h2);
+                v.w = *reinterpret_cast<uint32_t*>(&h3);
+                *reinterpret_cast<uint4*>(o + j) = v;
+            }
+        } else {
+#pragma unroll
+            for (int j = 0; j < CW; ++j)
+                if (q_base + j < p.q_rows) o[j] = __float2bfloat16_rn(__uint_as_float(r[j]));
+        }
+    } else {
+        float* o = reinterpret_cast<float*>(p.out) + (int64_t)prow * p.ldo + q_base;
+        if (full) {
+#pragma unroll
+            for (int j = 0; j < CW; j += 4)
+                *reinterpret_cast<float4*>(o + j) =
+                    make_float4(__uint_as_float(r[j]), __uint_as_float(r[j + 1]),
+                                __uint_as_float(r[j + 2]), __uint_as_float(r[j + 3]));
+        } else {
+#pragma unroll
+            for (int j = 0; j < CW; ++j)
+                if (q_base + j < p.q_rows) o[j] = __uint_as_float(r[j]);
+        }
+    }
+}
+
+template <int CW>
+__device__ __forceinline__ void tmem_load_chunk(uint32_t taddr, uint32_t (&r)[CW]);
+
+template <>
+__device__ __forceinline__ void tmem_load_chunk<32>(uint32_t taddr, uint32_t (&r)[32]) {
+    ptx::tmem_ld_32x32b_x32(taddr, r);
+}
+
+template <>
+__device__ __forceinline__ void tmem_load_chunk<16>(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32"
+        " {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+}
+
+template <int BN, int STAGES>
+__global__ void __launch_bounds__(192, 1)
+    gemm_mxf4_kernel(const __grid_constant__ CUtensorMap tmap_p,
+                     const __grid_constant__ CUtensorMap tmap_q, const GemmParams p) {
+    using S = GemmShape<BN>;
+    using L = GemmSmem<BN, STAGES>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kOffBar);
+    uint64_t* full = bars;
+    uint64_t* empty = bars + STAGES;
+    uint64_t* acc_full = bars + 2 * STAGES;
+    uint64_t* acc_empty = bars + 2 * STAGES + 2;
+    uint64_t* drain = bars + 2 * STAGES + 4;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kOffMisc);
+    volatile int* abort = reinterpret_cast<volatile int*>(smem + L::kOffMisc + 4);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            ptx::mbar_init(&full[s], 1);
+            ptx::mbar_init(&empty[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            ptx::mbar_init(&acc_full[a], 1);
+            ptx::mbar_init(&acc_empty[a], 4);
+        }
+        ptx::mbar_init(drain, 1);
+        *abort = 0;
+        ptx::fence_mbar_init();
+        ptx::fence_proxy_async_smem();
+        ptx::prefetch_tensormap(&tmap_p);
+        ptx::prefetch_tensormap(&tmap_q);
+    }
+    if (warp == 1) {
+        ptx::tmem_alloc(tmem_slot, S::kTmemCols);
+        ptx::tmem_relinquish();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer ---
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t issued_mask = 0, issued_phase = 0;
+            const int q_slabs = (p.q_rows + 127) / 128;
+            for (int u = blockIdx.x; u < p.total_units && !*abort; u += gridDim.x) {
+                const Unit t = decode_unit(p, u);
+                const int q0 = t.tq * BN;
+                const int slab0 = q0 / 128;
+                const int nchunks = min(S::kQChunks, q_slabs - slab0);
+                const uint32_t bytes = S::kPTileBytes + S::kQTileBytes + S::kSfChunkBytes * (1 + nchunks);
+                for (int kt = t.kt_begin; kt < t.kt_end; ++kt) {
+                    if (!wait_or_abort(&empty[stage], phase ^ 1, abort, p.err, kErrTimeoutProducer)) break;
+                    ptx::mbar_arrive_expect_tx(&full[stage], bytes);
+                    ptx::tma_load_2d(smem + L::kOffP + stage * S::kPTileBytes, &tmap_p, &full[stage],
+                                     kt * S::kBKBytes, t.tp * S::kBM);
+                    ptx::tma_load_2d(smem + L::kOffQ + stage * S::kQTileBytes, &tmap_q, &full[stage],
+                                     kt * S::kBKBytes, q0);
+                    ptx::bulk_load(smem + L::kOffSfP + stage * S::kSfChunkBytes,
+                                   p.sf_p + ((int64_t)t.tp * p.kb4_pad + 2 * kt) * 512,
+                                   S::kSfChunkBytes, &full[stage]);
+                    for (int c = 0; c < nchunks; ++c)
+                        ptx::bulk_load(smem + L::kOffSfQ + (stage * S::kQChunks + c) * S::kSfChunkBytes,
+                                       p.sf_q + ((int64_t)(slab0 + c) * p.kb4_pad + 2 * kt) * 512,
+                                       S::kSfChunkBytes, &full[stage]);
+                    issued_mask |= 1u << stage;
+                    issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
+                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
+                }
+            }
+            if (*abort) {
+                // let copies already in flight land before the CTA can exit: wait
+                // (bounded) for the phase of the latest fill of every stage
+                for (int s = 0; s < STAGES; ++s) {
+                    if (!((issued_mask >> s) & 1)) continue;
+                    const uint32_t ph = (issued_phase >> s) & 1;
+                    const uint64_t t0 = global_timer_ns();
+                    while (!ptx::mbar_try_wait(&full[s], ph) && global_timer_ns() - t0 < 100000000ull) {
+                    }
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // -------------------------------------------------------------- MMA -----
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int acc = 0;
+            uint32_t acc_phase = 0;
+            const uint32_t sf_base = tmem + S::kSfBase;
+            bool issued = false;
+            for (int u = blockIdx.x; u < p.total_units && !*abort; u += gridDim.x) {
+                const Unit t = decode_unit(p, u);
+                const uint32_t q_off = (uint32_t)((t.tq * BN) % 128) / 32;
+                if ((q_off & 1) != 0 || q_off * 32 + (BN < 32 ? 32 : BN) > 128 * S::kQChunks) {
+                    // never planned: a scale-factor column offset the MMA is not given
+                    atomicExch(p.err, kErrSfOffset);
+                    *abort = 1;
+                    break;
+                }
+                if (!wait_or_abort(&acc_empty[acc], acc_phase ^ 1, abort, p.err, kErrTimeoutMma)) break;
+                ptx::tc_fence_after();
+                const uint32_t d_tmem = tmem + acc * S::kAccStride;
+                bool ok = true;
+                for (int kt = t.kt_begin; kt < t.kt_end; ++kt) {
+                    if (!wait_or_abort(&full[stage], phase, abort, p.err, kErrTimeoutMma)) { ok = false; break; }
+                    ptx::tc_fence_after();
+                    const uint32_t sfp_s = ptx::smem_u32(smem + L::kOffSfP + stage * S::kSfChunkBytes);
+                    const uint32_t sfq_s = ptx::smem_u32(smem + L::kOffSfQ + stage * S::kQChunks * S::kSfChunkBytes);
+#pragma unroll
+                    for (int a = 0; a < 2; ++a) {
+                        ptx::tmem_cp_32x128b_x4(sf_base + 4 * a, ptx::smem_desc_sf(sfp_s + 512 * a));
+#pragma unroll
+                        for (int c = 0; c < S::kQChunks; ++c)
+                            ptx::tmem_cp_32x128b_x4(sf_base + 8 + a * 4 * S::kQChunks + 4 * c,
+                                                    ptx::smem_desc_sf(sfq_s + 1024 * c + 512 * a));
+                    }
+                    const uint64_t adesc = ptx::smem_desc_sw128(ptx::smem_u32(smem + L::kOffP + stage * S::kPTileBytes));
+                    const uint64_t bdesc = ptx::smem_desc_sw128(ptx::smem_u32(smem + L::kOffQ + stage * S::kQTileBytes));
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk) {
+                        const uint32_t a = kk >> 1;
+                        const uint32_t sfid = (kk & 1) * 2;
+                        const uint32_t sfa = (sf_base + 4 * a) | (sfid << 30);
+                        const uint32_t sfb = (sf_base + 8 + a * 4 * S::kQChunks + q_off) | (sfid << 30);
+                        ptx::mma_mxf4(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, ptx::idesc_mxf4(BN, sfid, sfid),
+                                      sfa, sfb, (kt > t.kt_begin || kk > 0) ? 1u : 0u);
+                    }
+                    issued = true;
+                    ptx::tc_commit(&empty[stage]);
+                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
+                }
+                if (!ok) break;
+                ptx::tc_commit(&acc_full[acc]);
+                if (S::kNumAcc == 2) {
+                    acc ^= 1;
+                    if (acc == 0) acc_phase ^= 1;
+                } else {
+                    acc_phase ^= 1;
+                }
+            }
+            if (*abort && issued) {
+                // wait (bounded) for every MMA this thread issued before TMEM is freed
+                ptx::tc_commit(drain);
+                const uint64_t t0 = global_timer_ns();
+                while (!ptx::mbar_try_wait(drain, 0) && global_timer_ns() - t0 < 100000000ull) {
+                }
+            }
+        }
+        __syncwarp();
+    } else {
+        // ----------------------------------------------------------- epilogue ---
+        const int quad = warp & 3;                 // TMEM subpartition this warp may read
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        constexpr int CW = S::kChunkCols;
+        for (int u = blockIdx.x; u < p.total_units && !*abort; u += gridDim.x) {
+            const Unit t = decode_unit(p, u);
+            if (!wait_or_abort(&acc_full[acc], acc_phase, abort, p.err, kErrTimeoutEpilogue)) break;
+            ptx::tc_fence_after();
+            const int prow = t.tp * S::kBM + quad * 32 + lane;
+            const uint32_t taddr = tmem + acc * S::kAccStride + ((uint32_t)(quad * 32) << 16);
+#pragma unroll 1
+            for (int c = 0; c < BN / CW; ++c) {
+                uint32_t r[CW];
+                tmem_load_chunk<CW>(taddr + c * CW, r);
+                ptx::tmem_ld_wait();
+                store_chunk<BN>(p, prow, t.tq * BN + c * CW, r);
+            }
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&acc_empty[acc]);
+            if (S::kNumAcc == 2) {
+                acc ^= 1;
+                if (acc == 0) acc_phase ^= 1;
+            } else {
+                acc_phase ^= 1;
+            }
+        }
+    }
+
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem, S::kTmemCols);
+    }
+}
+
+}  // namespace macaq

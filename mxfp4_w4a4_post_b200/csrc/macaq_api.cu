@@ -1,0 +1,443 @@
+// C ABI of libmacaq (declared in include/macaq.h): argument validation, launch
+// planning and kernel launches for the MACaQ W4A4 linear layer on sm_100a.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/macaq.h"
+#include "gemm_kernel.cuh"
+#include "quant_kernel.cuh"
+
+namespace macaq {
+
+__device__ int g_device_error;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+    bool ready = false;
+    bool supported = false;
+    int num_sms = 0;
+    int* err_ptr = nullptr;
+};
+
+std::mutex g_mutex;
+DeviceInfo g_devices[kMaxDevices];
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+
+macaq_status device_info(DeviceInfo** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MACAQ_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_mutex);
+    DeviceInfo& d = g_devices[dev];
+    if (!d.ready) {
+        int major = 0, minor = 0, sms = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return MACAQ_ERR_CUDA;
+        d.supported = (major == 10 && minor == 0);
+        d.num_sms = sms;
+        if (d.supported) {
+            void* p = nullptr;
+            if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return MACAQ_ERR_CUDA;
+            d.err_ptr = static_cast<int*>(p);
+            if (g_encode == nullptr) {
+                void* fn = nullptr;
+                cudaDriverEntryPointQueryResult q;
+                if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+                        cudaSuccess || q != cudaDriverEntryPointSuccess || fn == nullptr)
+                    return MACAQ_ERR_CUDA;
+                g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+            }
+        }
+        d.ready = true;
+    }
+    if (!d.supported) return MACAQ_ERR_UNSUPPORTED_DEVICE;
+    *out = &d;
+    return MACAQ_OK;
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+inline int64_t round_up(int64_t a, int64_t b) { return (a + b - 1) / b * b; }
+inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// Limits that keep every index inside 32 bits where the kernels use int.
+constexpr int64_t kMaxRows = (int64_t)1 << 30;
+constexpr int64_t kMaxK = (int64_t)1 << 24;
+
+// --------------------------------------------------------------------- quant ---
+
+macaq_status launch_quant(const void* x, int64_t rows, int64_t K, int64_t ld, const float* mult,
+                          uint8_t* codes, uint8_t* scales, const float* s_for_inv, float* inv_out,
+                          cudaStream_t stream) {
+    DeviceInfo* dev = nullptr;
+    macaq_status st = device_info(&dev);
+    if (st != MACAQ_OK) return st;
+    QuantParams p{};
+    p.x = static_cast<const uint16_t*>(x);
+    p.mult = mult;
+    p.codes = codes;
+    p.scales = scales;
+    p.s_for_inv = s_for_inv;
+    p.inv_out = inv_out;
+    p.rows = rows;
+    p.K = K;
+    p.ld = ld;
+    p.rows_pad = round_up(rows, 128);
+    p.kb_pad = round_up(K / 32, 8);
+    p.chunks_per_row = p.kb_pad / 8;
+    p.items = p.rows_pad * p.chunks_per_row;
+    constexpr int kThreads = 256, kUnroll = 4;
+    const int64_t warps_needed = cdiv(p.items, kUnroll);
+    const int64_t blocks_needed = cdiv(warps_needed * 32, kThreads);
+    const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>(blocks_needed, (int64_t)dev->num_sms * 8));
+    quant_rows_kernel<kUnroll><<<blocks, kThreads, 0, stream>>>(p);
+    return cudaGetLastError() == cudaSuccess ? MACAQ_OK : MACAQ_ERR_CUDA;
+}
+
+macaq_status check_quant_args(const void* x, int64_t rows, int64_t K, int64_t ld, const void* mult,
+                              const void* codes, const void* scales) {
+    if (!x || !mult || !codes || !scales) return MACAQ_ERR_INVALID_ARG;
+    if (rows < 1 || K < 32 || ld < K) return MACAQ_ERR_INVALID_ARG;
+    if (K % 32 != 0 || rows > kMaxRows || K > kMaxK) return MACAQ_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(x) || !aligned16(mult) || !aligned16(codes) || !aligned16(scales) || ld % 8 != 0)
+        return MACAQ_ERR_MISALIGNED;
+    return MACAQ_OK;
+}
+
+// ---------------------------------------------------------------------- GEMM ---
+
+struct GemmPlan {
+    bool swap;        // P = weight, Q = activations, output written transposed
+    int bn;
+    int tiles_p, tiles_q, k_tiles;
+    int splits, kps;
+    int group_p;
+    int grid;
+    bool atomic;
+};
+
+GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, int num_sms) {
+    GemmPlan g{};
+    g.k_tiles = (int)cdiv(K, 256);
+    int64_t p_rows, q_rows;
+    if (M <= 128) {
+        g.swap = true;
+        g.bn = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : 128;
+        p_rows = N;
+        q_rows = M;
+    } else {
+        g.swap = false;
+        g.bn = N <= 128 ? 128 : 192;
+        p_rows = M;
+        q_rows = N;
+    }
+    g.tiles_p = (int)cdiv(p_rows, 128);
+    g.tiles_q = (int)cdiv(q_rows, g.bn);
+    const int64_t tiles = (int64_t)g.tiles_p * g.tiles_q;
+    // Split K when the tiles alone fill the SMs poorly. Score each split count by its
+    // wave efficiency times kps / (kps + 1) (one K tile of pipeline fill per unit), and
+    // take a larger split count only when it scores 2% better.
+    auto score = [&](int s) {
+        const int kps = (int)cdiv(g.k_tiles, s);
+        const int64_t units = tiles * cdiv(g.k_tiles, kps);
+        const double eff = (double)units / (double)(cdiv(units, num_sms) * num_sms);
+        return eff * (double)kps / (double)(kps + 1);
+    };
+    g.splits = 1;
+    if (tiles < 2 * (int64_t)num_sms && g.k_tiles > 1) {
+        double best = score(1);
+        const int max_splits = std::max(1, g.k_tiles / 2);
+        for (int s = 2; s <= max_splits; ++s) {
+            const double sc = score(s);
+            if (sc > best * 1.02) {
+                best = sc;
+                g.splits = s;
+            }
+        }
+    }
+    g.kps = (int)cdiv(g.k_tiles, g.splits);
+    g.splits = (int)cdiv(g.k_tiles, g.kps);
+    g.atomic = g.splits > 1;
+    g.group_p = std::min(g.tiles_p, 16);
+    const int64_t units = tiles * g.splits;
+    g.grid = (int)std::min<int64_t>(units, num_sms);
+    return g;
+}
+
+// Row stride (elements) of the fp32 split-K accumulator: a multiple of 4 so that the
+// epilogue's 16-byte vector reductions stay aligned.
+inline int64_t acc_ld(int64_t N) { return round_up(N, 4); }
+
+size_t gemm_workspace(int64_t M, int64_t N, int64_t K, int num_sms) {
+    const GemmPlan g = plan_gemm(M, N, K, num_sms);
+    return g.atomic ? (size_t)round_up(M * acc_ld(N) * 4, 256) : 0;
+}
+
+bool encode_codes_map(CUtensorMap* map, const uint8_t* codes, int64_t rows, int64_t K, int box_rows) {
+    cuuint64_t dims[2] = {(cuuint64_t)(K / 2), (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)(K / 2)};
+    cuuint32_t box[2] = {128, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(codes), dims,
+                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <int BN, int STAGES>
+macaq_status launch_gemm_bn(const CUtensorMap& mp, const CUtensorMap& mq, const GemmParams& gp,
+                            int grid, cudaStream_t stream) {
+    using L = GemmSmem<BN, STAGES>;
+    static_assert(L::kAlloc <= 232448, "shared memory budget");
+    static std::atomic<uint64_t> configured_mask{0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const uint64_t bit = 1ull << (dev & 63);
+    if (!(configured_mask.load() & bit)) {
+        if (cudaFuncSetAttribute(gemm_mxf4_kernel<BN, STAGES>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc) != cudaSuccess)
+            return MACAQ_ERR_CUDA;
+        configured_mask.fetch_or(bit);
+    }
+    gemm_mxf4_kernel<BN, STAGES><<<grid, 192, L::kAlloc, stream>>>(mp, mq, gp);
+    return cudaGetLastError() == cudaSuccess ? MACAQ_OK : MACAQ_ERR_CUDA;
+}
+
+__global__ void finalize_kernel(const float* __restrict__ acc, int64_t lda, int64_t M, int64_t N, void* y,
+                                int64_t ldy, int bf16) {
+    const int64_t total = M * N;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t m = i / N, n = i - m * N;
+        const float v = acc[m * lda + n];
+        if (bf16)
+            static_cast<__nv_bfloat16*>(y)[m * ldy + n] = __float2bfloat16_rn(v);
+        else
+            static_cast<float*>(y)[m * ldy + n] = v;
+    }
+}
+
+macaq_status check_weight(const macaq_weight* w) {
+    if (!w || !w->codes || !w->scales) return MACAQ_ERR_INVALID_ARG;
+    if (w->N < 1 || w->K < 32) return MACAQ_ERR_INVALID_ARG;
+    if (w->K % 32 != 0 || w->N > kMaxRows || w->K > kMaxK) return MACAQ_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(w->codes) || !aligned16(w->scales)) return MACAQ_ERR_MISALIGNED;
+    return MACAQ_OK;
+}
+
+macaq_status run_gemm(const uint8_t* a_codes, const uint8_t* a_scales, int64_t M,
+                      const macaq_weight* w, void* y, int64_t ldy, macaq_out_dtype out,
+                      void* workspace, size_t ws_bytes, cudaStream_t stream) {
+    DeviceInfo* dev = nullptr;
+    macaq_status st = device_info(&dev);
+    if (st != MACAQ_OK) return st;
+    const int64_t N = w->N, K = w->K;
+    const GemmPlan g = plan_gemm(M, N, K, dev->num_sms);
+    const size_t need = gemm_workspace(M, N, K, dev->num_sms);
+    if (need > 0 && (workspace == nullptr || ws_bytes < need)) return MACAQ_ERR_WORKSPACE;
+    if (need > 0 && (reinterpret_cast<uintptr_t>(workspace) & 255) != 0) return MACAQ_ERR_MISALIGNED;
+
+    const uint8_t* p_codes = g.swap ? w->codes : a_codes;
+    const uint8_t* q_codes = g.swap ? a_codes : w->codes;
+    const int64_t p_rows = g.swap ? N : M;
+    const int64_t q_rows = g.swap ? M : N;
+    CUtensorMap mp, mq;
+    if (!encode_codes_map(&mp, p_codes, p_rows, K, 128) || !encode_codes_map(&mq, q_codes, q_rows, K, g.bn))
+        return MACAQ_ERR_CUDA;
+
+    GemmParams gp{};
+    gp.sf_p = g.swap ? w->scales : a_scales;
+    gp.sf_q = g.swap ? a_scales : w->scales;
+    gp.p_rows = (int32_t)p_rows;
+    gp.q_rows = (int32_t)q_rows;
+    gp.k_tiles = g.k_tiles;
+    gp.kb4_pad = (int32_t)(round_up(K / 32, 8) / 4);
+    gp.tiles_p = g.tiles_p;
+    gp.tiles_q = g.tiles_q;
+    gp.splits = g.splits;
+    gp.k_tiles_per_split = g.kps;
+    gp.total_units = g.tiles_p * g.tiles_q * g.splits;
+    gp.group_p = g.group_p;
+    gp.transpose_out = g.swap ? 1 : 0;
+    gp.err = dev->err_ptr;
+    if (g.atomic) {
+        if (cudaMemsetAsync(workspace, 0, (size_t)(M * acc_ld(N) * 4), stream) != cudaSuccess)
+            return MACAQ_ERR_CUDA;
+        gp.out = workspace;
+        gp.ldo = acc_ld(N);
+        gp.atomic = 1;
+        gp.out_bf16 = 0;
+        gp.vec_ok = 1;
+    } else {
+        const int64_t esz = out == MACAQ_OUT_BF16 ? 2 : 4;
+        gp.out = y;
+        gp.ldo = ldy;
+        gp.atomic = 0;
+        gp.out_bf16 = out == MACAQ_OUT_BF16 ? 1 : 0;
+        gp.vec_ok = (aligned16(y) && (ldy * esz) % 16 == 0) ? 1 : 0;
+    }
+
+    switch (g.bn) {
+        case 16: st = launch_gemm_bn<16, 8>(mp, mq, gp, g.grid, stream); break;
+        case 32: st = launch_gemm_bn<32, 8>(mp, mq, gp, g.grid, stream); break;
+        case 64: st = launch_gemm_bn<64, 8>(mp, mq, gp, g.grid, stream); break;
+        case 128: st = launch_gemm_bn<128, 6>(mp, mq, gp, g.grid, stream); break;
+        default: st = launch_gemm_bn<192, 5>(mp, mq, gp, g.grid, stream); break;
+    }
+    if (st != MACAQ_OK) return st;
+    if (g.atomic) {
+        const int64_t total = M * N;
+        const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>(cdiv(total, 256), (int64_t)dev->num_sms * 8));
+        finalize_kernel<<<blocks, 256, 0, stream>>>(static_cast<const float*>(workspace), acc_ld(N), M, N, y, ldy,
+                                                    out == MACAQ_OUT_BF16 ? 1 : 0);
+        if (cudaGetLastError() != cudaSuccess) return MACAQ_ERR_CUDA;
+    }
+    return MACAQ_OK;
+}
+
+macaq_status check_gemm_args(int64_t M, const macaq_weight* w, const void* y, int64_t ldy,
+                             macaq_out_dtype out) {
+    macaq_status st = check_weight(w);
+    if (st != MACAQ_OK) return st;
+    if (!y || M < 1 || ldy < w->N) return MACAQ_ERR_INVALID_ARG;
+    if (out != MACAQ_OUT_F32 && out != MACAQ_OUT_BF16) return MACAQ_ERR_INVALID_ARG;
+    if (M > kMaxRows || M * w->N > ((int64_t)1 << 40)) return MACAQ_ERR_UNSUPPORTED_SHAPE;
+    const uintptr_t esz = out == MACAQ_OUT_BF16 ? 2 : 4;
+    if ((reinterpret_cast<uintptr_t>(y) & (esz - 1)) != 0) return MACAQ_ERR_MISALIGNED;
+    return MACAQ_OK;
+}
+
+}  // namespace
+}  // namespace macaq
+
+using namespace macaq;
+
+extern "C" {
+
+size_t macaq_codes_bytes(int64_t rows, int64_t K) {
+    if (rows < 0 || K < 0) return 0;
+    return (size_t)(rows * (K / 2));
+}
+
+size_t macaq_scales_bytes(int64_t rows, int64_t K) {
+    if (rows < 0 || K < 0) return 0;
+    return (size_t)(round_up(rows, 128) * round_up(K / 32, 8));
+}
+
+size_t macaq_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, macaq_out_dtype out) {
+    (void)out;
+    if (M < 1 || N < 1 || K < 32) return 0;
+    DeviceInfo* dev = nullptr;
+    int sms = 148;
+    if (device_info(&dev) == MACAQ_OK) sms = dev->num_sms;
+    return gemm_workspace(M, N, K, sms);
+}
+
+static size_t linear_ws_parts(int64_t M, int64_t N, int64_t K, macaq_out_dtype out, size_t* off_scales,
+                              size_t* off_gemm) {
+    const size_t codes = (size_t)round_up((int64_t)macaq_codes_bytes(M, K), 256);
+    const size_t scales = (size_t)round_up((int64_t)macaq_scales_bytes(M, K), 256);
+    *off_scales = codes;
+    *off_gemm = codes + scales;
+    return codes + scales + macaq_gemm_workspace_bytes(M, N, K, out);
+}
+
+size_t macaq_linear_workspace_bytes(int64_t M, int64_t N, int64_t K, macaq_out_dtype out) {
+    if (M < 1 || N < 1 || K < 32) return 0;
+    size_t a, b;
+    return linear_ws_parts(M, N, K, out, &a, &b);
+}
+
+macaq_status macaq_prepare_weight(const void* W_bf16, int64_t N, int64_t K, int64_t ldw, const float* s,
+                                  uint8_t* w_codes, uint8_t* w_scales, float* inv_s_out,
+                                  macaq_stream stream) {
+    macaq_status st = check_quant_args(W_bf16, N, K, ldw, s, w_codes, w_scales);
+    if (st != MACAQ_OK) return st;
+    if (!inv_s_out) return MACAQ_ERR_INVALID_ARG;
+    if (!aligned16(inv_s_out)) return MACAQ_ERR_MISALIGNED;
+    return launch_quant(W_bf16, N, K, ldw, s, w_codes, w_scales, s, inv_s_out, (cudaStream_t)stream);
+}
+
+macaq_status macaq_quant_act(const void* x_bf16, int64_t M, int64_t K, int64_t ldx, const float* inv_s,
+                             uint8_t* a_codes, uint8_t* a_scales, macaq_stream stream) {
+    macaq_status st = check_quant_args(x_bf16, M, K, ldx, inv_s, a_codes, a_scales);
+    if (st != MACAQ_OK) return st;
+    return launch_quant(x_bf16, M, K, ldx, inv_s, a_codes, a_scales, nullptr, nullptr, (cudaStream_t)stream);
+}
+
+macaq_status macaq_gemm_mxfp4(const uint8_t* a_codes, const uint8_t* a_scales, int64_t M,
+                              const macaq_weight* w, void* y, int64_t ldy, macaq_out_dtype out,
+                              void* workspace, size_t ws_bytes, macaq_stream stream) {
+    macaq_status st = check_gemm_args(M, w, y, ldy, out);
+    if (st != MACAQ_OK) return st;
+    if (!a_codes || !a_scales) return MACAQ_ERR_INVALID_ARG;
+    if (!aligned16(a_codes) || !aligned16(a_scales)) return MACAQ_ERR_MISALIGNED;
+    return run_gemm(a_codes, a_scales, M, w, y, ldy, out, workspace, ws_bytes, (cudaStream_t)stream);
+}
+
+macaq_status macaq_linear_w4a4(const void* x_bf16, int64_t M, int64_t ldx, const macaq_weight* w, void* y,
+                               int64_t ldy, macaq_out_dtype out, int fused, void* workspace, size_t ws_bytes,
+                               macaq_stream stream) {
+    macaq_status st = check_gemm_args(M, w, y, ldy, out);
+    if (st != MACAQ_OK) return st;
+    if (fused != 0) return MACAQ_ERR_UNSUPPORTED;
+    if (!w->inv_s) return MACAQ_ERR_INVALID_ARG;
+    st = check_quant_args(x_bf16, M, w->K, ldx, w->inv_s, w->codes, w->scales);
+    if (st != MACAQ_OK) return st;
+    size_t off_scales, off_gemm;
+    const size_t need = linear_ws_parts(M, w->N, w->K, out, &off_scales, &off_gemm);
+    if (!workspace || ws_bytes < need) return MACAQ_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255) != 0) return MACAQ_ERR_MISALIGNED;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    uint8_t* a_codes = ws;
+    uint8_t* a_scales = ws + off_scales;
+    st = launch_quant(x_bf16, M, w->K, ldx, w->inv_s, a_codes, a_scales, nullptr, nullptr, (cudaStream_t)stream);
+    if (st != MACAQ_OK) return st;
+    return run_gemm(a_codes, a_scales, M, w, y, ldy, out, ws + off_gemm, ws_bytes - off_gemm, (cudaStream_t)stream);
+}
+
+macaq_status macaq_get_device_error(void) {
+    DeviceInfo* dev = nullptr;
+    macaq_status st = device_info(&dev);
+    if (st != MACAQ_OK) return st;
+    if (cudaDeviceSynchronize() != cudaSuccess) return MACAQ_ERR_CUDA;
+    int v = 0, zero = 0;
+    if (cudaMemcpy(&v, dev->err_ptr, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return MACAQ_ERR_CUDA;
+    if (v != 0 && cudaMemcpy(dev->err_ptr, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
+        return MACAQ_ERR_CUDA;
+    return v != 0 ? MACAQ_ERR_DEVICE_TIMEOUT : MACAQ_OK;
+}
+
+const char* macaq_status_string(macaq_status s) {
+    switch (s) {
+        case MACAQ_OK: return "MACAQ_OK";
+        case MACAQ_ERR_INVALID_ARG: return "MACAQ_ERR_INVALID_ARG";
+        case MACAQ_ERR_MISALIGNED: return "MACAQ_ERR_MISALIGNED";
+        case MACAQ_ERR_UNSUPPORTED_SHAPE: return "MACAQ_ERR_UNSUPPORTED_SHAPE";
+        case MACAQ_ERR_UNSUPPORTED_DEVICE: return "MACAQ_ERR_UNSUPPORTED_DEVICE";
+        case MACAQ_ERR_CUDA: return "MACAQ_ERR_CUDA";
+        case MACAQ_ERR_DEVICE_TIMEOUT: return "MACAQ_ERR_DEVICE_TIMEOUT";
+        case MACAQ_ERR_WORKSPACE: return "MACAQ_ERR_WORKSPACE";
+        case MACAQ_ERR_UNSUPPORTED: return "MACAQ_ERR_UNSUPPORTED";
+    }
+    return "MACAQ_ERR_UNKNOWN";
+}
+
+int macaq_version(void) { return MACAQ_VERSION; }
+
+}  // extern "C"

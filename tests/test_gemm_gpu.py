@@ -1,0 +1,113 @@
+"""Parity of the block-scaled FP4 GEMM (tcgen05 kind::mxf4) with the oracle's fp64 sum
+of decoded products. One-hot operands pin the nibble order and the scale layout;
+random codes and scales cover every tile path (swapped decode tiles of width 16..128,
+prefill tiles of width 128/224, split K, ragged M/N/K)."""
+import numpy as np
+import pytest
+
+import oracle
+from helpers import (assert_bf16_matches_f32, assert_gemm_close, host, random_mxfp4, u8_dev)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def mq():
+    import mxfp4_w4a4_post_b200 as m
+    from mxfp4_w4a4_post_b200 import build
+    build.build()
+    return m
+
+
+def gpu_gemm(mq, a_codes, a_scales_rm, w_codes, w_scales_rm, K, out="f32"):
+    """Run the CUDA GEMM on row-major oracle-format operands (scales swizzled into the
+    tensor-core layout by the oracle's own layout function)."""
+    import torch
+    M, N = a_codes.shape[0], w_codes.shape[0]
+    a_c = u8_dev(a_codes)
+    a_s = u8_dev(oracle.swizzle_scales(a_scales_rm, K))
+    w = mq.PreparedWeight(u8_dev(w_codes), u8_dev(oracle.swizzle_scales(w_scales_rm, K)),
+                          torch.ones(K, dtype=torch.float32, device="cuda"), N, K)
+    dt = torch.float32 if out == "f32" else torch.bfloat16
+    y = mq.gemm_mxfp4(a_c, a_s, M, w, out_dtype=dt)
+    torch.cuda.synchronize()
+    return y
+
+
+def one_hot_operands(M, N, K, picks):
+    """picks: list of (m, n, k, code_a, code_w, ea, ew). Each pick puts one code in row m
+    of A and row n of W at column k, with the given block exponents."""
+    a = np.zeros((M, K), np.uint8)
+    w = np.zeros((N, K), np.uint8)
+    sa = np.full((M, K // 32), 127, np.uint8)
+    sw = np.full((N, K // 32), 127, np.uint8)
+    for m, n, k, ca, cw, ea, ew in picks:
+        a[m, k] = ca
+        w[n, k] = cw
+        sa[m, k // 32] = 127 + ea
+        sw[n, k // 32] = 127 + ew
+    pack = lambda c: (c[:, 0::2] | (c[:, 1::2] << 4)).astype(np.uint8)
+    return pack(a), sa, pack(w), sw
+
+
+@pytest.mark.parametrize("M,N,K", [(16, 128, 256), (300, 448, 512), (200, 130, 768)])
+def test_one_hot_layout(mq, M, N, K):
+    rng = np.random.default_rng(M + N + K)
+    picks, used_k, used_m, used_n = [], set(), set(), set()
+    cand_k = [k for k in range(K) if k % 2 == 0 or k % 7 == 1]
+    while len(picks) < min(M, N, 24):
+        m, n, k = int(rng.integers(M)), int(rng.integers(N)), int(rng.choice(cand_k))
+        if m in used_m or n in used_n or k // 32 in used_k:
+            continue
+        used_m.add(m), used_n.add(n), used_k.add(k // 32)
+        picks.append((m, n, k, int(rng.integers(1, 16)), int(rng.integers(1, 16)),
+                      int(rng.integers(-6, 7)), int(rng.integers(-6, 7))))
+        if len(used_k) == K // 32:
+            break
+    a, sa, w, sw = one_hot_operands(M, N, K, picks)
+    y = host(gpu_gemm(mq, a, sa, w, sw, K)).astype(np.float64)
+    expect = oracle.gemm_fp64(a, sa, w, sw, K)
+    for m, n, k, ca, cw, ea, ew in picks:
+        v = oracle.e2m1_decode(ca) * oracle.e2m1_decode(cw) * 2.0 ** (ea + ew)
+        assert expect[m, n] == v
+    assert np.array_equal(y, expect), np.argwhere(y != expect)[:5]
+
+
+# (M, N, K): swapped decode tiles (M <= 128), prefill tiles (M > 128), ragged tails
+SHAPES = [
+    (1, 128, 256), (3, 300, 512), (16, 1000, 1024), (17, 256, 5120), (32, 2000, 2048),
+    (64, 640, 4096), (100, 384, 1280), (128, 512, 768),
+    (129, 224, 256), (256, 1024, 5120), (300, 700, 800), (512, 2240, 2048), (1000, 130, 1536),
+]
+
+
+@pytest.mark.parametrize("M,N,K", SHAPES)
+def test_random_operands(mq, M, N, K):
+    rng = np.random.default_rng(M * 7 + N * 3 + K)
+    a, sa = random_mxfp4(rng, M, K)
+    w, sw = random_mxfp4(rng, N, K)
+    y = host(gpu_gemm(mq, a, sa, w, sw, K))
+    rows = np.arange(M) if M <= 256 else np.unique(np.concatenate([rng.choice(M, 48, replace=False), [0, M - 1]]))
+    ref = oracle.gemm_fp64(a, sa, w, sw, K, rows=rows)
+    assert_gemm_close(y[rows], ref, f"gemm {M}x{N}x{K}")
+
+
+@pytest.mark.parametrize("M,N,K", [(8, 384, 1024), (300, 700, 800)])
+def test_bf16_output(mq, M, N, K):
+    rng = np.random.default_rng(5)
+    a, sa = random_mxfp4(rng, M, K)
+    w, sw = random_mxfp4(rng, N, K)
+    y32 = gpu_gemm(mq, a, sa, w, sw, K, out="f32")
+    y16 = gpu_gemm(mq, a, sa, w, sw, K, out="bf16")
+    assert_bf16_matches_f32(y16, y32, f"bf16 {M}x{N}x{K}")
+
+
+def test_extreme_scales(mq):
+    """Scale bytes near both ends of the range the quantiser emits (0 and 252), and
+    block sums that cancel exactly."""
+    rng = np.random.default_rng(6)
+    M, N, K = 64, 256, 512
+    a, sa = random_mxfp4(rng, M, K, 0, 5)
+    w, sw = random_mxfp4(rng, N, K, 240, 252)
+    y = host(gpu_gemm(mq, a, sa, w, sw, K))
+    assert_gemm_close(y, oracle.gemm_fp64(a, sa, w, sw, K), "extreme scales")
