@@ -148,6 +148,36 @@ macaq_status macaq_linear_w4a4(const void* x_bf16, int64_t M, int64_t ldx, const
                                void* y, int64_t ldy, macaq_out_dtype out, int fused,
                                void* workspace, size_t ws_bytes, macaq_stream stream);
 
+/* Largest scratch the no-allocation variant below can use: 16 MiB, held in a static
+ * device array on every GPU that loads this library, for as long as it stays loaded. */
+#define MACAQ_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+
+/* macaq_linear_w4a4 for callers that cannot allocate device memory. (The paper has no
+ * counterpart: this is a deployment convenience of this library.)
+ *
+ * Some callers cannot call cudaMalloc or hand the library a workspace: code embedded in
+ * a serving runtime or plugin host that owns the whole device memory pool and gives
+ * libraries none of it, and latency-critical loops where allocating or freeing would
+ * stall the device (cudaFree synchronises it) or could fail under memory pressure in the
+ * middle of serving. This entry point takes no workspace: the activation codes, scales
+ * and split-K accumulator live in one file-scope static device array of
+ * MACAQ_NOALLOC_SCRATCH_BYTES. The caller still passes x, the prepared weight and y,
+ * with the same meaning, layout and alignment rules as macaq_linear_w4a4 (fused = 0).
+ *
+ * - Sizes whose workspace (macaq_linear_workspace_bytes(M, N, K, out)) exceeds
+ *   MACAQ_NOALLOC_SCRATCH_BYTES are rejected with MACAQ_ERR_WORKSPACE; nothing is
+ *   enqueued.
+ * - The first call on each device looks up the array's device address (once per device,
+ *   with that device current); make that first call before any stream capture.
+ * - Every call on a device shares the one array, and the array keeps the last call's
+ *   contents. Whatever must start at zero is cleared by each call on its stream. Calls
+ *   whose executions overlap on the GPU (other streams, or no ordering between them)
+ *   race on the array and give undefined results: order them on one stream.
+ * - Allocates nothing: no cudaMalloc, cudaFree or allocating library routine. */
+macaq_status macaq_linear_w4a4_noalloc(const void* x_bf16, int64_t M, int64_t ldx,
+                                       const macaq_weight* w, void* y, int64_t ldy,
+                                       macaq_out_dtype out, macaq_stream stream);
+
 /* ------------------------------------------------------------ status ---------- */
 
 /* Every wait inside the GEMM kernel is bounded. A kernel that gives up a wait records

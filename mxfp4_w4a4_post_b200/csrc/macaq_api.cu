@@ -411,6 +411,45 @@ macaq_status macaq_linear_w4a4(const void* x_bf16, int64_t M, int64_t ldx, const
     return run_gemm(a_codes, a_scales, M, w, y, ldy, out, ws + off_gemm, ws_bytes - off_gemm, (cudaStream_t)stream);
 }
 
+}  // extern "C"
+
+// Scratch of macaq_linear_w4a4_noalloc: one static array per device that loads the
+// library. Host code must not pass the symbol itself to a kernel (on the host it names
+// a stand-in, not device memory); its device address is looked up once per device.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[MACAQ_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+std::mutex g_noalloc_mutex;
+void* g_noalloc_ptr[macaq::kMaxDevices];
+}  // namespace
+
+extern "C" {
+
+macaq_status macaq_linear_w4a4_noalloc(const void* x_bf16, int64_t M, int64_t ldx, const macaq_weight* w,
+                                       void* y, int64_t ldy, macaq_out_dtype out, macaq_stream stream) {
+    macaq_status st = check_gemm_args(M, w, y, ldy, out);
+    if (st != MACAQ_OK) return st;
+    if (macaq_linear_workspace_bytes(M, w->N, w->K, out) > MACAQ_NOALLOC_SCRATCH_BYTES)
+        return MACAQ_ERR_WORKSPACE;
+    DeviceInfo* info = nullptr;
+    st = device_info(&info);
+    if (st != MACAQ_OK) return st;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MACAQ_ERR_CUDA;
+    void* scratch = nullptr;
+    {
+        std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+        if (g_noalloc_ptr[dev] == nullptr) {
+            void* p = nullptr;
+            if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+                return MACAQ_ERR_CUDA;
+            g_noalloc_ptr[dev] = p;
+        }
+        scratch = g_noalloc_ptr[dev];
+    }
+    return macaq_linear_w4a4(x_bf16, M, ldx, w, y, ldy, out, 0, scratch, MACAQ_NOALLOC_SCRATCH_BYTES, stream);
+}
+
 macaq_status macaq_get_device_error(void) {
     DeviceInfo* dev = nullptr;
     macaq_status st = device_info(&dev);
