@@ -11,11 +11,14 @@
 // One persistent CTA per SM, warp-specialised:
 //   warp 0      TMA producer: codes via 2D tensor maps with the 128-byte swizzle (one
 //               256-element K tile = 128 bytes per row), scale atoms via bulk copies
-//   warp 1      TMEM owner and single-thread MMA issuer: tcgen05.cp moves the scale
-//               atoms SMEM -> TMEM, then four tcgen05.mma kind::mxf4.block_scale
-//               (K = 64 each) per K tile into an fp32 TMEM accumulator
+//   warp 1      TMEM owner and single-thread MMA issuer: four tcgen05.mma
+//               kind::mxf4.block_scale (K = 64 each) per K tile into an fp32 TMEM
+//               accumulator
 //   warps 2-5   epilogue: tcgen05.ld the accumulator (each warp owns one 32-lane TMEM
 //               subpartition), convert, store (or fp32 reduce for split K)
+//   warps 6-9   scale-factor writers: each reads the scale atoms of a K tile from
+//               shared memory and writes them into its TMEM subpartition with
+//               tcgen05.st, so the tensor pipe executes nothing but MMAs
 // Accumulators are double-buffered in TMEM when they fit, so the epilogue of one tile
 // overlaps the MMAs of the next. Every mbarrier wait is bounded by a wall-clock limit;
 // a kernel that gives up records an error code, drains what it issued, frees its TMEM
@@ -65,10 +68,12 @@ struct GemmShape {
     // 128-row scale slabs a Q tile can touch (a 192-row tile may start 64 rows into one)
     static constexpr int kQChunks = (BN <= 128) ? 1 : 2;
     static constexpr int kSfCols = 8 + 8 * kQChunks;        // 4 columns per atom, 2 atoms per tile
+    // Two scale-factor slots, used by alternate K tiles.
+    static constexpr int kSfSlots = 2;
     static constexpr int kAccStride = (BN == 192) ? 256 : BN;
-    static constexpr int kNumAcc = (BN + kAccStride + kSfCols <= 512) ? 2 : 1;
+    static constexpr int kNumAcc = (BN + kAccStride + kSfSlots * kSfCols <= 512) ? 2 : 1;
     static constexpr int kSfBase = (kNumAcc - 1) * kAccStride + BN;
-    static constexpr int kTmemNeed = kSfBase + kSfCols;
+    static constexpr int kTmemNeed = kSfBase + kSfSlots * kSfCols;
     static constexpr int kTmemCols = kTmemNeed <= 32 ? 32 : kTmemNeed <= 64 ? 64
                                    : kTmemNeed <= 128 ? 128 : kTmemNeed <= 256 ? 256 : 512;
     static constexpr int kChunkCols = BN < 32 ? BN : 32;    // epilogue TMEM load width
@@ -82,7 +87,7 @@ struct GemmSmem {
     static constexpr int kOffSfP = kOffQ + STAGES * S::kQTileBytes;
     static constexpr int kOffSfQ = kOffSfP + STAGES * S::kSfChunkBytes;
     static constexpr int kOffBar = kOffSfQ + STAGES * S::kQChunks * S::kSfChunkBytes;
-    static constexpr int kNumBars = 2 * STAGES + 4 + 1;
+    static constexpr int kNumBars = 2 * STAGES + 4 + 1 + 2;
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;
     static constexpr int kBytes = kOffMisc + 16;
     static constexpr int kAlloc = kBytes + 1024;            // slack to align the base to 1 KB
@@ -94,15 +99,26 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
     return t;
 }
 
+__device__ __noinline__ bool wait_or_abort_slow(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                                int* err, int code);
+
 // Wait for `parity` on `bar`, giving up after ~2 s (or as soon as another role of the
 // CTA has given up). On give-up record `code`, raise the CTA abort flag, return false.
-__device__ __noinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                           int* err, int code) {
+// mbarrier.try_wait suspends the thread in hardware until the phase completes or a
+// short hardware time limit passes, so the loop just polls again; the wall clock and
+// the abort flag are read every 16 polls.
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                              int* err, int code) {
     if (ptx::mbar_try_wait(bar, parity)) return true;
+    return wait_or_abort_slow(bar, parity, abort, err, code);
+}
+
+__device__ __noinline__ bool wait_or_abort_slow(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                                int* err, int code) {
     const uint64_t t0 = global_timer_ns();
-    for (uint32_t it = 0;; ++it) {
+    for (uint32_t it = 1;; ++it) {
         if (ptx::mbar_try_wait(bar, parity)) return true;
-        if ((it & 63) == 63) {
+        if ((it & 15) == 0) {
             if (*abort) return false;
             if (global_timer_ns() - t0 > 2000000000ull) {
                 atomicExch(err, code);
@@ -110,7 +126,6 @@ __device__ __noinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volat
                 return false;
             }
         }
-        __nanosleep(32);
     }
 }
 
@@ -234,8 +249,10 @@ __device__ __forceinline__ void tmem_load_chunk<16>(uint32_t taddr, uint32_t (&r
         : "r"(taddr));
 }
 
+constexpr int kGemmThreads = 320;
+
 template <int BN, int STAGES>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_mxf4_kernel(const __grid_constant__ CUtensorMap tmap_p,
                      const __grid_constant__ CUtensorMap tmap_q, const GemmParams p) {
     using S = GemmShape<BN>;
@@ -249,6 +266,7 @@ __global__ void __launch_bounds__(192, 1)
     uint64_t* acc_full = bars + 2 * STAGES;
     uint64_t* acc_empty = bars + 2 * STAGES + 2;
     uint64_t* drain = bars + 2 * STAGES + 4;
+    uint64_t* sf_full = bars + 2 * STAGES + 5;    // [2]: scale-factor slot written
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kOffMisc);
     volatile int* abort = reinterpret_cast<volatile int*>(smem + L::kOffMisc + 4);
 
@@ -265,6 +283,8 @@ __global__ void __launch_bounds__(192, 1)
             ptx::mbar_init(&acc_empty[a], 4);
         }
         ptx::mbar_init(drain, 1);
+        ptx::mbar_init(&sf_full[0], 4);
+        ptx::mbar_init(&sf_full[1], 4);
         *abort = 0;
         ptx::fence_mbar_init();
         ptx::fence_proxy_async_smem();
@@ -332,8 +352,10 @@ __global__ void __launch_bounds__(192, 1)
             uint32_t phase = 0;
             int acc = 0;
             uint32_t acc_phase = 0;
-            const uint32_t sf_base = tmem + S::kSfBase;
             bool issued = false;
+            // K tiles issued so far; K tile i reads its scale factors from TMEM slot
+            // i % 2, written by the scale-factor warps.
+            uint32_t kt_count = 0;
             for (int u = blockIdx.x; u < p.total_units && !*abort; u += gridDim.x) {
                 const Unit t = decode_unit(p, u);
                 const uint32_t q_off = (uint32_t)((t.tq * BN) % 128) / 32;
@@ -349,17 +371,13 @@ __global__ void __launch_bounds__(192, 1)
                 bool ok = true;
                 for (int kt = t.kt_begin; kt < t.kt_end; ++kt) {
                     if (!wait_or_abort(&full[stage], phase, abort, p.err, kErrTimeoutMma)) { ok = false; break; }
-                    ptx::tc_fence_after();
-                    const uint32_t sfp_s = ptx::smem_u32(smem + L::kOffSfP + stage * S::kSfChunkBytes);
-                    const uint32_t sfq_s = ptx::smem_u32(smem + L::kOffSfQ + stage * S::kQChunks * S::kSfChunkBytes);
-#pragma unroll
-                    for (int a = 0; a < 2; ++a) {
-                        ptx::tmem_cp_32x128b_x4(sf_base + 4 * a, ptx::smem_desc_sf(sfp_s + 512 * a));
-#pragma unroll
-                        for (int c = 0; c < S::kQChunks; ++c)
-                            ptx::tmem_cp_32x128b_x4(sf_base + 8 + a * 4 * S::kQChunks + 4 * c,
-                                                    ptx::smem_desc_sf(sfq_s + 1024 * c + 512 * a));
+                    const uint32_t slot = kt_count & 1;
+                    if (!wait_or_abort(&sf_full[slot], (kt_count >> 1) & 1, abort, p.err, kErrTimeoutMma)) {
+                        ok = false;
+                        break;
                     }
+                    ptx::tc_fence_after();
+                    const uint32_t sf_base = tmem + S::kSfBase + slot * S::kSfCols;
                     const uint64_t adesc = ptx::smem_desc_sw128(ptx::smem_u32(smem + L::kOffP + stage * S::kPTileBytes));
                     const uint64_t bdesc = ptx::smem_desc_sw128(ptx::smem_u32(smem + L::kOffQ + stage * S::kQTileBytes));
 #pragma unroll
@@ -373,6 +391,7 @@ __global__ void __launch_bounds__(192, 1)
                     }
                     issued = true;
                     ptx::tc_commit(&empty[stage]);
+                    ++kt_count;
                     if (++stage == STAGES) { stage = 0; phase ^= 1; }
                 }
                 if (!ok) break;
@@ -393,6 +412,63 @@ __global__ void __launch_bounds__(192, 1)
             }
         }
         __syncwarp();
+    } else if (warp >= 6) {
+        // ------------------------------------------------- scale-factor writers ---
+        // Warp q' (= warp % 4) owns TMEM lanes 32q'..32q'+31. In the 128x4 scale atom,
+        // the 16 bytes of shared-memory row l hold, as word w, the four block scales of
+        // matrix row l + 32w. The MMA's subpartition q reads the P scales of its rows
+        // 32q + l from column (atom base + q) and the Q scales of Q row l + 32w from
+        // column (atom base + w) of every subpartition.
+        const int quad = warp & 3;
+        const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
+        int stage = 0;
+        uint32_t phase = 0;
+        uint32_t kt_count = 0;
+        int hist_stage0 = 0, hist_stage1 = 0;
+        uint32_t hist_phase0 = 0, hist_phase1 = 0;
+        for (int u = blockIdx.x; u < p.total_units && !*abort; u += gridDim.x) {
+            const Unit t = decode_unit(p, u);
+            bool ok = true;
+            for (int kt = t.kt_begin; kt < t.kt_end; ++kt) {
+                if (!wait_or_abort(&full[stage], phase, abort, p.err, kErrTimeoutMma)) { ok = false; break; }
+                const uint32_t slot = kt_count & 1;
+                // the slot's previous readers (the MMAs of K tile kt_count - 2) must be done
+                if (kt_count >= 2 &&
+                    !wait_or_abort(&empty[slot ? hist_stage1 : hist_stage0], slot ? hist_phase1 : hist_phase0,
+                                   abort, p.err, kErrTimeoutMma)) {
+                    ok = false;
+                    break;
+                }
+                ptx::tc_fence_after();
+                const uint32_t col = lane_base + S::kSfBase + slot * S::kSfCols;
+                const uint32_t sfp_s = ptx::smem_u32(smem + L::kOffSfP + stage * S::kSfChunkBytes) + lane * 16;
+                const uint32_t sfq_s =
+                    ptx::smem_u32(smem + L::kOffSfQ + stage * S::kQChunks * S::kSfChunkBytes) + lane * 16;
+#pragma unroll
+                for (int a = 0; a < 2; ++a) {
+                    ptx::tmem_st_32x32b_x1(col + 4 * a + quad, ptx::lds32(sfp_s + 512 * a + 4 * quad));
+#pragma unroll
+                    for (int c = 0; c < S::kQChunks; ++c) {
+                        const uint4 v = ptx::lds128(sfq_s + 1024 * c + 512 * a);
+                        ptx::tmem_st_32x32b_x4(col + 8 + a * 4 * S::kQChunks + 4 * c, v.x, v.y, v.z, v.w);
+                    }
+                }
+                ptx::tmem_st_wait();
+                ptx::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(&sf_full[slot]);
+                if (slot) {
+                    hist_stage1 = stage;
+                    hist_phase1 = phase;
+                } else {
+                    hist_stage0 = stage;
+                    hist_phase0 = phase;
+                }
+                ++kt_count;
+                if (++stage == STAGES) { stage = 0; phase ^= 1; }
+            }
+            if (!ok) break;
+        }
     } else {
         // ----------------------------------------------------------- epilogue ---
         const int quad = warp & 3;                 // TMEM subpartition this warp may read

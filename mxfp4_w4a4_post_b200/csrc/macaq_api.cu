@@ -8,8 +8,9 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <numeric>
 
-#include "../../include/macaq.h"
+#include "macaq.h"
 #include "gemm_kernel.cuh"
 #include "quant_kernel.cuh"
 
@@ -98,13 +99,24 @@ macaq_status launch_quant(const void* x, int64_t rows, int64_t K, int64_t ld, co
     p.ld = ld;
     p.rows_pad = round_up(rows, 128);
     p.kb_pad = round_up(K / 32, 8);
-    p.chunks_per_row = p.kb_pad / 8;
-    p.items = p.rows_pad * p.chunks_per_row;
-    constexpr int kThreads = 256, kUnroll = 4;
-    const int64_t warps_needed = cdiv(p.items, kUnroll);
-    const int64_t blocks_needed = cdiv(warps_needed * 32, kThreads);
-    const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>(blocks_needed, (int64_t)dev->num_sms * 8));
-    quant_rows_kernel<kUnroll><<<blocks, kThreads, 0, stream>>>(p);
+    p.chunks_per_row = cdiv(p.kb_pad, 32);
+    // Every warp keeps one column chunk, so the grid's warp count is a multiple of the
+    // chunks per row; no more warps than (chunk, row) pairs, and two CTAs per SM.
+    const int64_t warps_per_cta = kQuantThreads / 32;
+    const int64_t unit = std::max<int64_t>(1, std::lcm<int64_t>(warps_per_cta, p.chunks_per_row));
+    const int64_t want = std::min<int64_t>((int64_t)dev->num_sms * 2 * warps_per_cta, p.rows_pad * p.chunks_per_row);
+    const int64_t nwarps = std::max<int64_t>(unit, want / unit * unit);
+    const int blocks = (int)(nwarps / warps_per_cta);
+    static std::atomic<uint64_t> smem_set{0};
+    int devid = 0;
+    cudaGetDevice(&devid);
+    if (!(smem_set.load() & (1ull << (devid & 63)))) {
+        if (cudaFuncSetAttribute(quant_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kQuantSmemBytes) != cudaSuccess)
+            return MACAQ_ERR_CUDA;
+        smem_set.fetch_or(1ull << (devid & 63));
+    }
+    quant_rows_kernel<<<blocks, kQuantThreads, kQuantSmemBytes, stream>>>(p);
     return cudaGetLastError() == cudaSuccess ? MACAQ_OK : MACAQ_ERR_CUDA;
 }
 
@@ -214,7 +226,7 @@ macaq_status launch_gemm_bn(const CUtensorMap& mp, const CUtensorMap& mq, const 
             return MACAQ_ERR_CUDA;
         configured_mask.fetch_or(bit);
     }
-    gemm_mxf4_kernel<BN, STAGES><<<grid, 192, L::kAlloc, stream>>>(mp, mq, gp);
+    gemm_mxf4_kernel<BN, STAGES><<<grid, kGemmThreads, L::kAlloc, stream>>>(mp, mq, gp);
     return cudaGetLastError() == cudaSuccess ? MACAQ_OK : MACAQ_ERR_CUDA;
 }
 

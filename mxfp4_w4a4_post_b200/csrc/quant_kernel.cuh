@@ -1,23 +1,36 @@
 // MACaQ online activation transform / offline weight preparation kernel (sm_100a).
 //
 // Per row r and 32-element block b (MACaQ pages: per-channel scale then block
-// Hadamard "micro-rotation" aligned to the MXFP4 group, openai-hub.com article;
-// MXFP4 = E2M1 elements + one E8M0 scale per 32):
+// Hadamard rotation aligned to the MXFP4 group, openai-hub.com article; MXFP4 = E2M1
+// elements + one E8M0 scale per 32):
 //   u   = fp32(x[r, k]) * mult[k]                      (mult = 1/s or s)
-//   v   = c * FWHT32(u)   stages h = 1,2,4,8,16, (a+b, a-b), c = fp32(1/sqrt(32))
+//   t   = FWHT32(u)    stages h = 1,2,4,8,16, pair (a+b, a-b), a the lower index
+//   v   = c * t        c = fp32(1/sqrt(32))
 //   e   = max(floor(log2 max|v|) - 2, -127)             (0 for an all-zero block)
 //   q   = v * 2^-e  ->  E2M1 round-to-nearest-even, saturating, sign kept
 //
-// Mapping: one warp handles a 256-element chunk of one row (8 blocks); lane l holds
-// elements 8*(l%4) .. 8*(l%4)+7 of block l/4, loaded with one 16-byte load. Butterfly
-// stages h = 1, 2, 4 stay inside a lane, h = 8 and 16 use xor-shuffles over lane bits
-// 0 and 1. Every arithmetic step uses the explicit round-to-nearest intrinsics, so the
-// compiler cannot contract a multiply into an add.
+// One thread owns one block; a warp covers 32 consecutive blocks (1024 elements) of a
+// row and keeps that column chunk for all its rows, so its 32 multipliers stay in
+// registers. Activation bytes move global -> shared with per-thread cp.async (16 bytes
+// each, 4 per block), STAGES - 1 blocks ahead of the one being computed; each thread
+// reads back only what it copied, so a wait_group is the only synchronisation. The
+// four 16-byte pieces of a block sit XOR-swizzled in the thread's 64-byte slot
+// (piece j at (j ^ ((lane >> 1) & 3))), which keeps both the copies and the reads free
+// of bank conflicts. The butterfly runs in registers, no shuffles. Every fp32 step uses
+// the explicit round-to-nearest intrinsics, so nothing is contracted.
 //
-// Output: the lane's 8 codes as one 32-bit word (nibble t = element t), and one 32-bit
-// word of four consecutive block scales per 4 blocks, placed in the 128-row x 4-block
-// atom layout of the tensor-core scale factors. Padding rows (up to a multiple of 128)
-// and padding blocks (up to a multiple of 8) get scale byte 0.
+// Two exact shortcuts, each giving the same bits as the steps above:
+//  - max|v| = fl(c * max|t|): rounding is monotone and c > 0.
+//  - for -123 <= e <= 123, q = fl(t * (c * 2^-e)) with c * 2^-e an exact normal fp32:
+//    whenever fl(c t) is normal, fl(c t) * 2^-e is exact, so both round c t 2^-e once;
+//    whenever it is not, |q| < 2^-3 and both give a zero code of the same sign. Outside
+//    that range the two multiplies are done one after the other.
+// E2M1 encoding uses cvt.rn.satfinite.e2m1x2.f32 (round to nearest even, saturating to
+// +-6, sign of zero kept), two elements per instruction, element 2j in the low nibble.
+//
+// Scales: one byte per thread; the four threads of blocks 4g..4g+3 combine them into
+// one 32-bit word of the 128-row x 4-block atom layout. Padding rows (up to a multiple
+// of 128) and padding blocks (up to a multiple of 8) get scale byte 0.
 #pragma once
 
 #include <cstdint>
@@ -26,149 +39,219 @@
 namespace macaq {
 
 struct QuantParams {
-    const uint16_t* x;     // bf16 bits [rows x K], row stride ld
-    const float* mult;     // [K]
-    uint8_t* codes;        // [rows x K/2]
-    uint8_t* scales;       // atom layout, rows_pad x kb_pad bytes
+    const uint16_t* x;       // bf16 bits [rows x K], row stride ld
+    const float* mult;       // [K]
+    uint8_t* codes;          // [rows x K/2]
+    uint8_t* scales;         // atom layout, rows_pad x kb_pad bytes
     const float* s_for_inv;  // non-null: also write inv_out[k] = 1/s[k]
     float* inv_out;
     int64_t rows, K, ld;
-    int64_t rows_pad;      // round_up(rows, 128)
-    int64_t kb_pad;        // round_up(K/32, 8)
-    int64_t chunks_per_row;  // kb_pad / 8
-    int64_t items;         // rows_pad * chunks_per_row
+    int64_t rows_pad;        // round_up(rows, 128)
+    int64_t kb_pad;          // round_up(K/32, 8)
+    int64_t chunks_per_row;  // ceil(kb_pad / 32): warp-sized groups of blocks per row
 };
 
-__device__ __forceinline__ uint32_t e2m1_code(float q) {
-    // Count of rounding thresholds exceeded: 0.25 and 1.25, 2.5 and 5 are ties that go
-    // down (to the even mantissa), 0.75, 1.75 and 3.5 ties that go up.
-    const float a = fabsf(q);
-    uint32_t idx = (a > 0.25f) + (a >= 0.75f) + (a > 1.25f) + (a >= 1.75f) + (a > 2.5f) +
-                   (a >= 3.5f) + (a > 5.0f);
-    return ((__float_as_uint(q) >> 31) << 3) | idx;
+// Eight fp32 values -> eight E2M1 codes in one 32-bit word, value i in nibble i.
+__device__ __forceinline__ uint32_t cvt_e2m1x8(const float (&a)[8]) {
+    uint32_t out;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+        : "=r"(out)
+        : "f"(a[0]), "f"(a[1]), "f"(a[2]), "f"(a[3]), "f"(a[4]), "f"(a[5]), "f"(a[6]), "f"(a[7]));
+    return out;
 }
 
-// Quantise the lane's 8 values; returns the packed codes and, through `sbyte`, the
-// block's scale byte (identical in the 4 lanes of the block).
-__device__ __forceinline__ uint32_t transform_and_encode(float (&v)[8], uint32_t lane,
-                                                         uint32_t& sbyte) {
-    // in-lane butterfly stages h = 1, 2, 4
-#pragma unroll
-    for (int h = 1; h < 8; h <<= 1) {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            if (i & h) continue;
-            const float a = v[i], b = v[i + h];
-            v[i] = __fadd_rn(a, b);
-            v[i + h] = __fsub_rn(a, b);
-        }
-    }
-    // cross-lane stages h = 8 (lane bit 0) and h = 16 (lane bit 1)
-#pragma unroll
-    for (int bit = 1; bit <= 2; bit <<= 1) {
-        const bool upper = (lane & bit) != 0;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const float p = __shfl_xor_sync(0xffffffffu, v[i], bit);
-            // lower position keeps a + b, upper keeps a - b, a being the lower one
-            v[i] = upper ? __fsub_rn(p, v[i]) : __fadd_rn(v[i], p);
-        }
-    }
-    const float c = __uint_as_float(0x3E3504F3u);  // nearest fp32 to 1/sqrt(32)
-    float amax = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        v[i] = __fmul_rn(v[i], c);
-        amax = fmaxf(amax, fabsf(v[i]));
-    }
-    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-
-    // floor(log2 amax) from the exponent field; any amax below 2^-124 (subnormals
-    // included) lands on the clamp e = -127.
-    const int biased = (int)(__float_as_uint(amax) >> 23);
-    int e = biased - 127 - 2;
-    if (biased == 0) e = -127;
-    e = max(e, -127);
-    sbyte = (uint32_t)(e + 127);
-    const float inv = __uint_as_float((uint32_t)(127 - e) << 23);  // 2^-e, exact
-
-    uint32_t word = 0;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) word |= e2m1_code(__fmul_rn(v[i], inv)) << (4 * i);
-    return word;
+// Packed fp32 pairs (sm_100 f32x2 instructions): each half is an independent IEEE
+// round-to-nearest operation, bit-identical to the scalar one.
+__device__ __forceinline__ uint64_t pk(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void upk(uint64_t v, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ float max3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+// Eight fp32 values held as four pairs -> eight E2M1 codes, value i in nibble i.
+__device__ __forceinline__ uint32_t cvt_e2m1x8(uint64_t p0, uint64_t p1, uint64_t p2, uint64_t p3) {
+    float a[8];
+    upk(p0, a[0], a[1]);
+    upk(p1, a[2], a[3]);
+    upk(p2, a[4], a[5]);
+    upk(p3, a[6], a[7]);
+    return cvt_e2m1x8(a);
 }
 
-template <int UNROLL>
-__global__ void __launch_bounds__(256) quant_rows_kernel(QuantParams p) {
+constexpr int kQuantThreads = 256;
+constexpr int kQuantStages = 4;
+constexpr int kQuantSmemBytes = kQuantStages * kQuantThreads * 64;
+
+__device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+__global__ void __launch_bounds__(kQuantThreads, 2) quant_rows_kernel(QuantParams p) {
+    extern __shared__ __align__(16) uint8_t qsmem[];
     const uint32_t lane = threadIdx.x & 31;
-    const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int64_t gw = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    // the host makes nwarps a multiple of chunks_per_row: every warp keeps one chunk
+    const int64_t chunk = gw % p.chunks_per_row;
+    const int64_t row_step = nwarps / p.chunks_per_row;
+    const int64_t b = chunk * 32 + lane;                 // block index in the row
     const int64_t kb = p.K >> 5;
-    const uint32_t blk_in_chunk = lane >> 2;   // 0..7
-    const uint32_t quarter = lane & 3;         // which 8 elements of the block
+    const bool col_live = b < kb;
+    const float c = __uint_as_float(0x3E3504F3u);        // nearest fp32 to 1/sqrt(32)
+    const uint32_t swz = (lane >> 1) & 3;
+    const uint32_t slot0 = (uint32_t)__cvta_generic_to_shared(qsmem) + threadIdx.x * 64;
 
-    for (int64_t base = warp; base < p.items; base += nwarps * UNROLL) {
-        uint4 raw[UNROLL];
-        float4 m0[UNROLL], m1[UNROLL];
-        bool valid[UNROLL];
-        int64_t row[UNROLL], k0[UNROLL];
-        // issue every load of the unrolled items first
+    uint64_t mult[16];                                   // multiplier pairs (2j, 2j+1)
+    if (col_live) {
+        const float4* mp = reinterpret_cast<const float4*>(p.mult + b * 32);
 #pragma unroll
-        for (int u = 0; u < UNROLL; ++u) {
-            const int64_t item = base + (int64_t)u * nwarps;
-            row[u] = item / p.chunks_per_row;
-            const int64_t chunk = item - row[u] * p.chunks_per_row;
-            const int64_t blk = chunk * 8 + blk_in_chunk;
-            k0[u] = blk * 32 + quarter * 8;
-            valid[u] = item < p.items && row[u] < p.rows && blk < kb;
-            raw[u] = make_uint4(0, 0, 0, 0);
-            m0[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-            m1[u] = m0[u];
-            if (valid[u]) {
-                raw[u] = __ldg(reinterpret_cast<const uint4*>(p.x + row[u] * p.ld + k0[u]));
-                m0[u] = __ldg(reinterpret_cast<const float4*>(p.mult + k0[u]));
-                m1[u] = __ldg(reinterpret_cast<const float4*>(p.mult + k0[u] + 4));
+        for (int i = 0; i < 8; ++i) {
+            const float4 m = __ldg(mp + i);
+            mult[2 * i] = pk(m.x, m.y);
+            mult[2 * i + 1] = pk(m.z, m.w);
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) mult[i] = 0;
+    }
+
+    const int64_t row0 = gw / p.chunks_per_row;
+    auto issue = [&](int64_t row, int stage) {
+        if (row < p.rows && col_live) {
+            const uint8_t* src = reinterpret_cast<const uint8_t*>(p.x + row * p.ld + b * 32);
+            const uint32_t dst = slot0 + (uint32_t)stage * (kQuantThreads * 64);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) cp_async_16(dst + 16 * (j ^ swz), src + 16 * j);
+        }
+        cp_async_commit();
+    };
+#pragma unroll
+    for (int s = 0; s < kQuantStages - 1; ++s) issue(row0 + s * row_step, s);
+
+    int stage = 0;
+    for (int64_t row = row0; row < p.rows_pad; row += row_step) {
+        issue(row + (kQuantStages - 1) * row_step, (stage + kQuantStages - 1) % kQuantStages);
+        cp_async_wait<kQuantStages - 1>();
+        const bool live = row < p.rows && col_live;
+
+        // T[j] holds elements (2j, 2j+1) of the block
+        uint64_t T[16];
+        if (live) {
+            const uint32_t src = slot0 + (uint32_t)stage * (kQuantThreads * 64);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                uint32_t w[4];
+                asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                             : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
+                             : "r"(src + 16 * (j ^ swz)));
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    T[4 * j + q] = mul2(pk(__uint_as_float(w[q] << 16), __uint_as_float(w[q] & 0xFFFF0000u)),
+                                        mult[4 * j + q]);
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) T[i] = 0;
+        }
+        stage = (stage + 1) % kQuantStages;
+
+        // butterfly stage h = 1 combines the two halves of each pair
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            float a, d;
+            upk(T[j], a, d);
+            T[j] = pk(__fadd_rn(a, d), __fsub_rn(a, d));
+        }
+        // stages h = 2, 4, 8, 16 pair T[j] with T[j + h/2], two elements per instruction
+#pragma unroll
+        for (int hp = 1; hp < 16; hp <<= 1) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                if (j & hp) continue;
+                const uint64_t A = T[j], B = T[j + hp];
+                T[j] = add2(A, B);
+                T[j + hp] = sub2(A, B);
             }
         }
+
+        float tmax = 0.0f;
 #pragma unroll
-        for (int u = 0; u < UNROLL; ++u) {
-            const int64_t item = base + (int64_t)u * nwarps;
-            if (item >= p.items) break;   // warp-uniform
-            const float mm[8] = {m0[u].x, m0[u].y, m0[u].z, m0[u].w,
-                                 m1[u].x, m1[u].y, m1[u].z, m1[u].w};
-            const uint32_t w[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
-            float v[8];
+        for (int j = 0; j < 16; ++j) {
+            float a, d;
+            upk(T[j], a, d);
+            tmax = max3(tmax, fabsf(a), fabsf(d));
+        }
+        const float amax = __fmul_rn(tmax, c);
+        const int biased = (int)(__float_as_uint(amax) >> 23);
+        const int e = max(biased - 129, -127);        // biased == 0 (zero / subnormal) -> -127
+        const uint32_t sbyte = (uint32_t)(e + 127);
+
+        uint32_t packed[4];
+        if (e >= -123 && e <= 123) {
+            const float k = __uint_as_float(0x3E3504F3u - ((uint32_t)e << 23));   // c * 2^-e
+            const uint64_t kk = pk(k, k);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                v[2 * i] = __fmul_rn(__uint_as_float(w[i] << 16), mm[2 * i]);
-                v[2 * i + 1] = __fmul_rn(__uint_as_float(w[i] & 0xFFFF0000u), mm[2 * i + 1]);
-            }
-            uint32_t sbyte;
-            const uint32_t word = transform_and_encode(v, lane, sbyte);
-            if (valid[u]) {
-                *reinterpret_cast<uint32_t*>(p.codes + row[u] * (p.K >> 1) + (k0[u] >> 1)) = word;
-                if (p.s_for_inv != nullptr && row[u] == 0) {
+            for (int i = 0; i < 4; ++i)
+                packed[i] = cvt_e2m1x8(mul2(T[4 * i], kk), mul2(T[4 * i + 1], kk), mul2(T[4 * i + 2], kk),
+                                       mul2(T[4 * i + 3], kk));
+        } else {
+            const float inv = __uint_as_float((uint32_t)(127 - e) << 23);      // 2^-e
+            const uint64_t cc = pk(c, c), ii = pk(inv, inv);
 #pragma unroll
-                    for (int i = 0; i < 8; ++i)
-                        p.inv_out[k0[u] + i] = __fdiv_rn(1.0f, p.s_for_inv[k0[u] + i]);
-                }
+            for (int i = 0; i < 4; ++i)
+                packed[i] = cvt_e2m1x8(mul2(mul2(T[4 * i], cc), ii), mul2(mul2(T[4 * i + 1], cc), ii),
+                                       mul2(mul2(T[4 * i + 2], cc), ii), mul2(mul2(T[4 * i + 3], cc), ii));
+        }
+
+        if (live) {
+            *reinterpret_cast<uint4*>(p.codes + row * (p.K >> 1) + b * 16) =
+                make_uint4(packed[0], packed[1], packed[2], packed[3]);
+            if (p.s_for_inv != nullptr && row == 0) {
+#pragma unroll 4
+                for (int i = 0; i < 32; ++i) p.inv_out[b * 32 + i] = __fdiv_rn(1.0f, p.s_for_inv[b * 32 + i]);
             }
-            // gather the scale bytes of blocks 4g .. 4g+3 (lanes 16g, 16g+4, ...)
-            const uint32_t b0 = __shfl_sync(0xffffffffu, sbyte, (lane & 16) + 0);
-            const uint32_t b1 = __shfl_sync(0xffffffffu, sbyte, (lane & 16) + 4);
-            const uint32_t b2 = __shfl_sync(0xffffffffu, sbyte, (lane & 16) + 8);
-            const uint32_t b3 = __shfl_sync(0xffffffffu, sbyte, (lane & 16) + 12);
-            if ((lane & 15) == 0) {
-                const int64_t r = row[u];
-                const int64_t chunk = item - r * p.chunks_per_row;
-                const int64_t j = chunk * 8 + (lane >> 2);   // multiple of 4
-                const int64_t off = ((r >> 7) * (p.kb_pad >> 2) + (j >> 2)) * 512 +
-                                    (r & 31) * 16 + ((r >> 5) & 3) * 4;
-                *reinterpret_cast<uint32_t*>(p.scales + off) = b0 | (b1 << 8) | (b2 << 16) | (b3 << 24);
-            }
+        }
+        // four consecutive blocks -> one scale word (lanes 4g .. 4g+3 of the warp)
+        const uint32_t s1 = __shfl_down_sync(0xffffffffu, sbyte, 1);
+        const uint32_t s2 = __shfl_down_sync(0xffffffffu, sbyte, 2);
+        const uint32_t s3 = __shfl_down_sync(0xffffffffu, sbyte, 3);
+        if ((lane & 3) == 0 && b < p.kb_pad) {
+            const int64_t off = ((row >> 7) * (p.kb_pad >> 2) + (b >> 2)) * 512 + (row & 31) * 16 +
+                                ((row >> 5) & 3) * 4;
+            *reinterpret_cast<uint32_t*>(p.scales + off) = sbyte | (s1 << 8) | (s2 << 16) | (s3 << 24);
         }
     }
+    cp_async_wait<0>();
 }
 
 }  // namespace macaq
