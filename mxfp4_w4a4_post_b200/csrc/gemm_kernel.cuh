@@ -16,9 +16,10 @@
 //               accumulator
 //   warps 2-5   epilogue: tcgen05.ld the accumulator (each warp owns one 32-lane TMEM
 //               subpartition), convert, store (or fp32 reduce for split K)
-//   warps 6-9   scale-factor writers: each reads the scale atoms of a K tile from
-//               shared memory and writes them into its TMEM subpartition with
-//               tcgen05.st, so the tensor pipe executes nothing but MMAs
+//   warps 6-13  scale-factor writers, two sets of four taking alternate K tiles: each
+//               warp reads the scale atoms of a K tile from shared memory and writes
+//               them into its TMEM subpartition with tcgen05.st, so the tensor pipe
+//               executes nothing but MMAs
 // Accumulators are double-buffered in TMEM when they fit, so the epilogue of one tile
 // overlaps the MMAs of the next. Every mbarrier wait is bounded by a wall-clock limit;
 // a kernel that gives up records an error code, drains what it issued, frees its TMEM
@@ -54,11 +55,11 @@ struct GemmParams {
 
 enum : int { kErrTimeoutProducer = 1, kErrTimeoutMma = 2, kErrTimeoutEpilogue = 3, kErrSfOffset = 4 };
 
-template <int BN>
+template <int BN, int STAGES>
 struct GemmShape {
     // Q tiles start on a 64-row boundary of the 128-row scale slabs (offset 0 or 2 TMEM
     // columns), the only scale-factor column offsets the MMA is given.
-    static_assert(BN == 16 || BN == 32 || BN == 64 || BN == 128 || BN == 192 || BN == 256,
+    static_assert(BN == 16 || BN == 32 || BN == 64 || BN == 128 || BN == 192,
                   "unsupported tile width");
     static constexpr int kBM = 128;
     static constexpr int kBKBytes = 128;                    // 256 FP4 elements per row
@@ -68,12 +69,13 @@ struct GemmShape {
     // 128-row scale slabs a Q tile can touch (a 192-row tile may start 64 rows into one)
     static constexpr int kQChunks = (BN <= 128) ? 1 : 2;
     static constexpr int kSfCols = 8 + 8 * kQChunks;        // 4 columns per atom, 2 atoms per tile
-    // Two scale-factor slots, used by alternate K tiles.
-    static constexpr int kSfSlots = 2;
-    static constexpr int kAccStride = (BN == 192) ? 256 : BN;
-    static constexpr int kNumAcc = (BN + kAccStride + kSfSlots * kSfCols <= 512) ? 2 : 1;
-    static constexpr int kSfBase = (kNumAcc - 1) * kAccStride + BN;
-    static constexpr int kTmemNeed = kSfBase + kSfSlots * kSfCols;
+    // TMEM: two fp32 accumulators of BN columns side by side, then one scale-factor
+    // slot per pipeline stage (the K tile in stage s uses slot s).
+    static constexpr int kNumAcc = 2;
+    static constexpr int kAccStride = BN;
+    static constexpr int kSfBase = kNumAcc * BN;
+    static constexpr int kTmemNeed = kSfBase + STAGES * kSfCols;
+    static_assert(kTmemNeed <= 512, "tensor memory budget");
     static constexpr int kTmemCols = kTmemNeed <= 32 ? 32 : kTmemNeed <= 64 ? 64
                                    : kTmemNeed <= 128 ? 128 : kTmemNeed <= 256 ? 256 : 512;
     static constexpr int kChunkCols = BN < 32 ? BN : 32;    // epilogue TMEM load width
@@ -81,13 +83,13 @@ struct GemmShape {
 
 template <int BN, int STAGES>
 struct GemmSmem {
-    using S = GemmShape<BN>;
+    using S = GemmShape<BN, STAGES>;
     static constexpr int kOffP = 0;
     static constexpr int kOffQ = kOffP + STAGES * S::kPTileBytes;
     static constexpr int kOffSfP = kOffQ + STAGES * S::kQTileBytes;
     static constexpr int kOffSfQ = kOffSfP + STAGES * S::kSfChunkBytes;
     static constexpr int kOffBar = kOffSfQ + STAGES * S::kQChunks * S::kSfChunkBytes;
-    static constexpr int kNumBars = 2 * STAGES + 4 + 1 + 2;
+    static constexpr int kNumBars = 3 * STAGES + 4 + 1;
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;
     static constexpr int kBytes = kOffMisc + 16;
     static constexpr int kAlloc = kBytes + 1024;            // slack to align the base to 1 KB
@@ -148,10 +150,8 @@ __device__ __forceinline__ Unit decode_unit(const GemmParams& p, int u) {
     return x;
 }
 
-template <int BN>
-__device__ __forceinline__ void store_chunk(const GemmParams& p, int prow, int q_base,
-                                            const uint32_t (&r)[GemmShape<BN>::kChunkCols]) {
-    constexpr int CW = GemmShape<BN>::kChunkCols;
+template <int CW>
+__device__ __forceinline__ void store_chunk(const GemmParams& p, int prow, int q_base, const uint32_t (&r)[CW]) {
     if (prow >= p.p_rows) return;
     if (p.transpose_out) {
         // out[q, prow]: for each column the 32 lanes of the warp write consecutive prow
@@ -249,13 +249,14 @@ __device__ __forceinline__ void tmem_load_chunk<16>(uint32_t taddr, uint32_t (&r
         : "r"(taddr));
 }
 
-constexpr int kGemmThreads = 320;
+constexpr int kSfWarpSets = 2;                                // scale-writer sets
+constexpr int kGemmThreads = 32 * (6 + 4 * kSfWarpSets);
 
 template <int BN, int STAGES>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_mxf4_kernel(const __grid_constant__ CUtensorMap tmap_p,
                      const __grid_constant__ CUtensorMap tmap_q, const GemmParams p) {
-    using S = GemmShape<BN>;
+    using S = GemmShape<BN, STAGES>;
     using L = GemmSmem<BN, STAGES>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -266,7 +267,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint64_t* acc_full = bars + 2 * STAGES;
     uint64_t* acc_empty = bars + 2 * STAGES + 2;
     uint64_t* drain = bars + 2 * STAGES + 4;
-    uint64_t* sf_full = bars + 2 * STAGES + 5;    // [2]: scale-factor slot written
+    uint64_t* sf_full = bars + 2 * STAGES + 5;    // [STAGES]: scale-factor slot written
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kOffMisc);
     volatile int* abort = reinterpret_cast<volatile int*>(smem + L::kOffMisc + 4);
 
@@ -283,8 +284,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             ptx::mbar_init(&acc_empty[a], 4);
         }
         ptx::mbar_init(drain, 1);
-        ptx::mbar_init(&sf_full[0], 4);
-        ptx::mbar_init(&sf_full[1], 4);
+        for (int s = 0; s < STAGES; ++s) ptx::mbar_init(&sf_full[s], 4);
         *abort = 0;
         ptx::fence_mbar_init();
         ptx::fence_proxy_async_smem();
@@ -353,9 +353,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             int acc = 0;
             uint32_t acc_phase = 0;
             bool issued = false;
-            // K tiles issued so far; K tile i reads its scale factors from TMEM slot
-            // i % 2, written by the scale-factor warps.
-            uint32_t kt_count = 0;
             for (int u = blockIdx.x; u < p.total_units && !*abort; u += gridDim.x) {
                 const Unit t = decode_unit(p, u);
                 const uint32_t q_off = (uint32_t)((t.tq * BN) % 128) / 32;
@@ -371,13 +368,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 bool ok = true;
                 for (int kt = t.kt_begin; kt < t.kt_end; ++kt) {
                     if (!wait_or_abort(&full[stage], phase, abort, p.err, kErrTimeoutMma)) { ok = false; break; }
-                    const uint32_t slot = kt_count & 1;
-                    if (!wait_or_abort(&sf_full[slot], (kt_count >> 1) & 1, abort, p.err, kErrTimeoutMma)) {
+                    // scale factors of this K tile, written into slot `stage` by the
+                    // scale-factor warps
+                    if (!wait_or_abort(&sf_full[stage], phase, abort, p.err, kErrTimeoutMma)) {
                         ok = false;
                         break;
                     }
                     ptx::tc_fence_after();
-                    const uint32_t sf_base = tmem + S::kSfBase + slot * S::kSfCols;
+                    const uint32_t sf_base = tmem + S::kSfBase + stage * S::kSfCols;
                     const uint64_t adesc = ptx::smem_desc_sw128(ptx::smem_u32(smem + L::kOffP + stage * S::kPTileBytes));
                     const uint64_t bdesc = ptx::smem_desc_sw128(ptx::smem_u32(smem + L::kOffQ + stage * S::kQTileBytes));
 #pragma unroll
@@ -391,7 +389,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     }
                     issued = true;
                     ptx::tc_commit(&empty[stage]);
-                    ++kt_count;
                     if (++stage == STAGES) { stage = 0; phase ^= 1; }
                 }
                 if (!ok) break;
@@ -420,27 +417,28 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         // 32q + l from column (atom base + q) and the Q scales of Q row l + 32w from
         // column (atom base + w) of every subpartition.
         const int quad = warp & 3;
+        const int set = (warp - 6) >> 2;          // this set writes K tiles with count % sets == set
         const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
         int stage = 0;
         uint32_t phase = 0;
         uint32_t kt_count = 0;
-        int hist_stage0 = 0, hist_stage1 = 0;
-        uint32_t hist_phase0 = 0, hist_phase1 = 0;
         for (int u = blockIdx.x; u < p.total_units && !*abort; u += gridDim.x) {
             const Unit t = decode_unit(p, u);
             bool ok = true;
-            for (int kt = t.kt_begin; kt < t.kt_end; ++kt) {
+            for (int kt = t.kt_begin; kt < t.kt_end; ++kt, ++kt_count) {
+                // Every set waits for every fill, in order, even those it does not
+                // write: a fill's barrier can then never be more than one phase ahead
+                // of the parity waited for, so a wait cannot match an older phase.
+                // Slot `stage` was last read by the MMAs of the previous fill of this
+                // stage; the producer waited for their completion before refilling the
+                // stage, so once the new fill has landed the slot is free.
                 if (!wait_or_abort(&full[stage], phase, abort, p.err, kErrTimeoutMma)) { ok = false; break; }
-                const uint32_t slot = kt_count & 1;
-                // the slot's previous readers (the MMAs of K tile kt_count - 2) must be done
-                if (kt_count >= 2 &&
-                    !wait_or_abort(&empty[slot ? hist_stage1 : hist_stage0], slot ? hist_phase1 : hist_phase0,
-                                   abort, p.err, kErrTimeoutMma)) {
-                    ok = false;
-                    break;
+                if ((int)(kt_count % kSfWarpSets) != set) {
+                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
+                    continue;
                 }
                 ptx::tc_fence_after();
-                const uint32_t col = lane_base + S::kSfBase + slot * S::kSfCols;
+                const uint32_t col = lane_base + S::kSfBase + stage * S::kSfCols;
                 const uint32_t sfp_s = ptx::smem_u32(smem + L::kOffSfP + stage * S::kSfChunkBytes) + lane * 16;
                 const uint32_t sfq_s =
                     ptx::smem_u32(smem + L::kOffSfQ + stage * S::kQChunks * S::kSfChunkBytes) + lane * 16;
@@ -456,15 +454,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 ptx::tmem_st_wait();
                 ptx::tc_fence_before();
                 __syncwarp();
-                if (lane == 0) ptx::mbar_arrive(&sf_full[slot]);
-                if (slot) {
-                    hist_stage1 = stage;
-                    hist_phase1 = phase;
-                } else {
-                    hist_stage0 = stage;
-                    hist_phase0 = phase;
-                }
-                ++kt_count;
+                if (lane == 0) ptx::mbar_arrive(&sf_full[stage]);
                 if (++stage == STAGES) { stage = 0; phase ^= 1; }
             }
             if (!ok) break;
@@ -486,7 +476,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 uint32_t r[CW];
                 tmem_load_chunk<CW>(taddr + c * CW, r);
                 ptx::tmem_ld_wait();
-                store_chunk<BN>(p, prow, t.tq * BN + c * CW, r);
+                store_chunk<CW>(p, prow, t.tq * BN + c * CW, r);
             }
             ptx::tc_fence_before();
             __syncwarp();
