@@ -299,6 +299,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    // Set-up above overlaps the previous kernel's tail; operands are read only after it.
+    ptx::griddep_wait();
+    ptx::griddep_launch_dependents();
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer ---

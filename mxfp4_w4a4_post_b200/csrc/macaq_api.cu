@@ -81,6 +81,26 @@ constexpr int64_t kMaxK = (int64_t)1 << 24;
 
 // --------------------------------------------------------------------- quant ---
 
+// Every kernel is launched with programmatic stream serialization: its launch and
+// set-up may overlap the tail of the previous kernel on the stream, and each kernel
+// executes griddepcontrol.wait before its first global memory access, so the order of
+// memory effects is the same as with plain stream order.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       Args&&... args) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 macaq_status launch_quant(const void* x, int64_t rows, int64_t K, int64_t ld, const float* mult,
                           uint8_t* codes, uint8_t* scales, const float* s_for_inv, float* inv_out,
                           cudaStream_t stream) {
@@ -116,8 +136,9 @@ macaq_status launch_quant(const void* x, int64_t rows, int64_t K, int64_t ld, co
             return MACAQ_ERR_CUDA;
         smem_set.fetch_or(1ull << (devid & 63));
     }
-    quant_rows_kernel<<<blocks, kQuantThreads, kQuantSmemBytes, stream>>>(p);
-    return cudaGetLastError() == cudaSuccess ? MACAQ_OK : MACAQ_ERR_CUDA;
+    return launch_pdl(quant_rows_kernel, dim3(blocks), dim3(kQuantThreads), kQuantSmemBytes, stream, p) == cudaSuccess
+               ? MACAQ_OK
+               : MACAQ_ERR_CUDA;
 }
 
 macaq_status check_quant_args(const void* x, int64_t rows, int64_t K, int64_t ld, const void* mult,
@@ -226,12 +247,16 @@ macaq_status launch_gemm_bn(const CUtensorMap& mp, const CUtensorMap& mq, const 
             return MACAQ_ERR_CUDA;
         configured_mask.fetch_or(bit);
     }
-    gemm_mxf4_kernel<BN, STAGES><<<grid, kGemmThreads, L::kAlloc, stream>>>(mp, mq, gp);
-    return cudaGetLastError() == cudaSuccess ? MACAQ_OK : MACAQ_ERR_CUDA;
+    return launch_pdl(gemm_mxf4_kernel<BN, STAGES>, dim3(grid), dim3(kGemmThreads), L::kAlloc, stream, mp, mq, gp) ==
+                   cudaSuccess
+               ? MACAQ_OK
+               : MACAQ_ERR_CUDA;
 }
 
 __global__ void finalize_kernel(const float* __restrict__ acc, int64_t lda, int64_t M, int64_t N, void* y,
                                 int64_t ldy, int bf16) {
+    ptx::griddep_wait();
+    ptx::griddep_launch_dependents();
     const int64_t total = M * N;
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
          i += (int64_t)gridDim.x * blockDim.x) {
@@ -315,9 +340,9 @@ macaq_status run_gemm(const uint8_t* a_codes, const uint8_t* a_scales, int64_t M
     if (g.atomic) {
         const int64_t total = M * N;
         const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>(cdiv(total, 256), (int64_t)dev->num_sms * 8));
-        finalize_kernel<<<blocks, 256, 0, stream>>>(static_cast<const float*>(workspace), acc_ld(N), M, N, y, ldy,
-                                                    out == MACAQ_OUT_BF16 ? 1 : 0);
-        if (cudaGetLastError() != cudaSuccess) return MACAQ_ERR_CUDA;
+        if (launch_pdl(finalize_kernel, dim3(blocks), dim3(256), 0, stream, static_cast<const float*>(workspace),
+                       acc_ld(N), M, N, y, ldy, out == MACAQ_OUT_BF16 ? 1 : 0) != cudaSuccess)
+            return MACAQ_ERR_CUDA;
     }
     return MACAQ_OK;
 }

@@ -23,6 +23,19 @@ __device__ __forceinline__ bool elect_one() {
     return pred != 0;
 }
 
+// --------------------------------------------------- programmatic dependent launch ----
+
+// Wait until the grids this one depends on (the previous kernel on the stream, when this
+// one was launched with programmatic stream serialization) have completed and their
+// memory is visible. Without that launch attribute it returns at once.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Allow the next kernel on the stream to start launching; it still waits for this grid
+// to complete before it touches memory (griddep_wait above).
+__device__ __forceinline__ void griddep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ------------------------------------------------------------------ mbarrier ----
 
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {

@@ -12,11 +12,13 @@
 // One thread owns one block; a warp covers 32 consecutive blocks (1024 elements) of a
 // row and keeps that column chunk for all its rows, so its 32 multipliers stay in
 // registers. Activation bytes move global -> shared with per-thread cp.async (16 bytes
-// each, 4 per block), STAGES - 1 blocks ahead of the one being computed; each thread
+// each, 4 per block), STAGES - 1 rows ahead of the one being computed; each thread
 // reads back only what it copied, so a wait_group is the only synchronisation. The
-// four 16-byte pieces of a block sit XOR-swizzled in the thread's 64-byte slot
-// (piece j at (j ^ ((lane >> 1) & 3))), which keeps both the copies and the reads free
-// of bank conflicts. The butterfly runs in registers, no shuffles. Every fp32 step uses
+// first copies are issued before the multipliers are fetched, so the two latencies
+// overlap. The four 16-byte pieces of a block sit XOR-swizzled in the thread's 64-byte
+// slot (piece j at (j ^ ((lane >> 1) & 3))), which keeps both the copies and the reads
+// free of bank conflicts. The butterfly runs in registers, no shuffles; max |t| is a
+// three-level tree of 3-input maxima rather than a 32-long chain. Every fp32 step uses
 // the explicit round-to-nearest intrinsics, so nothing is contracted.
 //
 // Two exact shortcuts, each giving the same bits as the steps above:
@@ -35,6 +37,8 @@
 
 #include <cstdint>
 #include <cuda_bf16.h>
+
+#include "ptx_sm100.cuh"
 
 namespace macaq {
 
@@ -107,29 +111,79 @@ __device__ __forceinline__ uint32_t cvt_e2m1x8(uint64_t p0, uint64_t p1, uint64_
 
 constexpr int kQuantThreads = 256;
 constexpr int kQuantStages = 4;
-constexpr int kQuantSmemBytes = kQuantStages * kQuantThreads * 64;
+constexpr uint32_t kQuantStageBytes = kQuantThreads * 64;
+constexpr int kQuantSmemBytes = kQuantStages * kQuantStageBytes;
 
-__device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+// 16-byte global -> shared copy; src_bytes = 0 reads nothing and writes 16 zero bytes.
+__device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
+                 : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
+__device__ __forceinline__ float absmax3(float a, float b, float c) { return max3(fabsf(a), fabsf(b), fabsf(c)); }
+
 __global__ void __launch_bounds__(kQuantThreads, 2) quant_rows_kernel(QuantParams p) {
     extern __shared__ __align__(16) uint8_t qsmem[];
     const uint32_t lane = threadIdx.x & 31;
-    const int64_t gw = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    // grid sizes are small (a few thousand warps): 32-bit warp and row indices
+    const int gw = (int)((blockIdx.x * kQuantThreads + threadIdx.x) >> 5);
+    const int nwarps = (int)((gridDim.x * kQuantThreads) >> 5);
+    const int cpr = (int)p.chunks_per_row;
     // the host makes nwarps a multiple of chunks_per_row: every warp keeps one chunk
-    const int64_t chunk = gw % p.chunks_per_row;
-    const int64_t row_step = nwarps / p.chunks_per_row;
-    const int64_t b = chunk * 32 + lane;                 // block index in the row
-    const int64_t kb = p.K >> 5;
-    const bool col_live = b < kb;
+    const int chunk = gw % cpr;
+    const int row_step = nwarps / cpr;
+    const int row0 = gw / cpr;
+    const int rows = (int)p.rows, rows_pad = (int)p.rows_pad;
+    const int b = chunk * 32 + lane;                     // block index in the row
+    const bool col_live = b < (int)(p.K >> 5);
     const float c = __uint_as_float(0x3E3504F3u);        // nearest fp32 to 1/sqrt(32)
-    const uint32_t swz = (lane >> 1) & 3;
+
+    // Copy pipeline. Rows past the end and blocks past K are zero-filled instead of
+    // branched around: they give zero blocks, whose scale byte 0 is exactly what the
+    // padding of the scale layout needs, and their codes are never stored.
+    const uint32_t swz16 = ((lane >> 1) & 3) << 4;
+    uint32_t off[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) off[j] = (uint32_t)(16 * j) ^ swz16;
     const uint32_t slot0 = (uint32_t)__cvta_generic_to_shared(qsmem) + threadIdx.x * 64;
+    const uint32_t slot_end = slot0 + kQuantStages * kQuantStageBytes;
+    const uint8_t* xbase = reinterpret_cast<const uint8_t*>(p.x);
+    const int64_t ld_bytes = p.ld * 2;
+    const uint8_t* isrc = xbase + (int64_t)row0 * ld_bytes + (int64_t)b * 64;
+    const int64_t istep = (int64_t)row_step * ld_bytes;
+    int irow = row0;
+    uint32_t islot = slot0;
+    auto issue = [&]() {
+        const bool v = col_live && irow < rows;
+        const uint8_t* src = v ? isrc : xbase;
+        const uint32_t n = v ? 16u : 0u;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) cp_async_16(islot + off[j], src + 16 * j, n);
+        cp_async_commit();
+        irow += row_step;
+        isrc += istep;
+        islot += kQuantStageBytes;
+        if (islot == slot_end) islot = slot0;
+    };
+    // Nothing global is touched before the previous kernel on the stream has finished.
+    ptx::griddep_wait();
+    ptx::griddep_launch_dependents();
+#pragma unroll
+    for (int s = 0; s < kQuantStages - 1; ++s) issue();
+
+    if (p.s_for_inv != nullptr && row0 == 0 && col_live) {
+        const float4* sp = reinterpret_cast<const float4*>(p.s_for_inv + b * 32);
+        float4* ip = reinterpret_cast<float4*>(p.inv_out + b * 32);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const float4 v = __ldg(sp + i);
+            ip[i] = make_float4(__fdiv_rn(1.0f, v.x), __fdiv_rn(1.0f, v.y), __fdiv_rn(1.0f, v.z),
+                                __fdiv_rn(1.0f, v.w));
+        }
+    }
 
     uint64_t mult[16];                                   // multiplier pairs (2j, 2j+1)
     if (col_live) {
@@ -145,45 +199,31 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_rows_kernel(QuantParam
         for (int i = 0; i < 16; ++i) mult[i] = 0;
     }
 
-    const int64_t row0 = gw / p.chunks_per_row;
-    auto issue = [&](int64_t row, int stage) {
-        if (row < p.rows && col_live) {
-            const uint8_t* src = reinterpret_cast<const uint8_t*>(p.x + row * p.ld + b * 32);
-            const uint32_t dst = slot0 + (uint32_t)stage * (kQuantThreads * 64);
-#pragma unroll
-            for (int j = 0; j < 4; ++j) cp_async_16(dst + 16 * (j ^ swz), src + 16 * j);
-        }
-        cp_async_commit();
-    };
-#pragma unroll
-    for (int s = 0; s < kQuantStages - 1; ++s) issue(row0 + s * row_step, s);
 
-    int stage = 0;
-    for (int64_t row = row0; row < p.rows_pad; row += row_step) {
-        issue(row + (kQuantStages - 1) * row_step, (stage + kQuantStages - 1) % kQuantStages);
+    uint32_t rslot = slot0;
+    uint8_t* cdst = p.codes + (int64_t)row0 * (p.K >> 1) + (int64_t)b * 16;
+    const int64_t cstep = (int64_t)row_step * (p.K >> 1);
+    const int kb_pad = (int)p.kb_pad;
+    const int64_t kb4 = p.kb_pad >> 2;
+    for (int row = row0; row < rows_pad; row += row_step) {
+        issue();
         cp_async_wait<kQuantStages - 1>();
-        const bool live = row < p.rows && col_live;
 
         // T[j] holds elements (2j, 2j+1) of the block
         uint64_t T[16];
-        if (live) {
-            const uint32_t src = slot0 + (uint32_t)stage * (kQuantThreads * 64);
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                uint32_t w[4];
-                asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                             : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
-                             : "r"(src + 16 * (j ^ swz)));
+        for (int j = 0; j < 4; ++j) {
+            uint32_t w[4];
+            asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
+                         : "r"(rslot + off[j]));
 #pragma unroll
-                for (int q = 0; q < 4; ++q)
-                    T[4 * j + q] = mul2(pk(__uint_as_float(w[q] << 16), __uint_as_float(w[q] & 0xFFFF0000u)),
-                                        mult[4 * j + q]);
-            }
-        } else {
-#pragma unroll
-            for (int i = 0; i < 16; ++i) T[i] = 0;
+            for (int q = 0; q < 4; ++q)
+                T[4 * j + q] = mul2(pk(__uint_as_float(w[q] << 16), __uint_as_float(w[q] & 0xFFFF0000u)),
+                                    mult[4 * j + q]);
         }
-        stage = (stage + 1) % kQuantStages;
+        rslot += kQuantStageBytes;
+        if (rslot == slot_end) rslot = slot0;
 
         // butterfly stage h = 1 combines the two halves of each pair
 #pragma unroll
@@ -204,13 +244,16 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_rows_kernel(QuantParam
             }
         }
 
-        float tmax = 0.0f;
+        // max |t| as a three-level tree (the order of a max does not change its value)
+        float a[32];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-            float a, d;
-            upk(T[j], a, d);
-            tmax = max3(tmax, fabsf(a), fabsf(d));
-        }
+        for (int j = 0; j < 16; ++j) upk(T[j], a[2 * j], a[2 * j + 1]);
+        float m[11];
+#pragma unroll
+        for (int i = 0; i < 10; ++i) m[i] = absmax3(a[3 * i], a[3 * i + 1], a[3 * i + 2]);
+        m[10] = fmaxf(fabsf(a[30]), fabsf(a[31]));
+        const float tmax = max3(max3(m[0], m[1], m[2]), max3(m[3], m[4], m[5]),
+                                max3(max3(m[6], m[7], m[8]), m[9], m[10]));
         const float amax = __fmul_rn(tmax, c);
         const int biased = (int)(__float_as_uint(amax) >> 23);
         const int e = max(biased - 129, -127);        // biased == 0 (zero / subnormal) -> -127
@@ -233,22 +276,16 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_rows_kernel(QuantParam
                                        mul2(mul2(T[4 * i + 2], cc), ii), mul2(mul2(T[4 * i + 3], cc), ii));
         }
 
-        if (live) {
-            *reinterpret_cast<uint4*>(p.codes + row * (p.K >> 1) + b * 16) =
-                make_uint4(packed[0], packed[1], packed[2], packed[3]);
-            if (p.s_for_inv != nullptr && row == 0) {
-#pragma unroll 4
-                for (int i = 0; i < 32; ++i) p.inv_out[b * 32 + i] = __fdiv_rn(1.0f, p.s_for_inv[b * 32 + i]);
-            }
-        }
+        if (col_live && row < rows)
+            *reinterpret_cast<uint4*>(cdst) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+        cdst += cstep;
         // four consecutive blocks -> one scale word (lanes 4g .. 4g+3 of the warp)
         const uint32_t s1 = __shfl_down_sync(0xffffffffu, sbyte, 1);
         const uint32_t s2 = __shfl_down_sync(0xffffffffu, sbyte, 2);
         const uint32_t s3 = __shfl_down_sync(0xffffffffu, sbyte, 3);
-        if ((lane & 3) == 0 && b < p.kb_pad) {
-            const int64_t off = ((row >> 7) * (p.kb_pad >> 2) + (b >> 2)) * 512 + (row & 31) * 16 +
-                                ((row >> 5) & 3) * 4;
-            *reinterpret_cast<uint32_t*>(p.scales + off) = sbyte | (s1 << 8) | (s2 << 16) | (s3 << 24);
+        if ((lane & 3) == 0 && b < kb_pad) {
+            const int64_t o = ((int64_t)(row >> 7) * kb4 + (b >> 2)) * 512 + (row & 31) * 16 + ((row >> 5) & 3) * 4;
+            *reinterpret_cast<uint32_t*>(p.scales + o) = sbyte | (s1 << 8) | (s2 << 16) | (s3 << 24);
         }
     }
     cp_async_wait<0>();
