@@ -10,10 +10,14 @@
 //
 // One persistent CTA per SM, warp-specialised:
 //   warp 0      TMA producer: codes via 2D tensor maps with the 128-byte swizzle (one
-//               256-element K tile = 128 bytes per row), scale atoms via bulk copies
+//               256-element K tile = 128 bytes per row), scale atoms via bulk copies.
+//               The producer and the MMA issuer run their loops on the whole warp, so
+//               every address and descriptor is a warp-uniform value, and one elected
+//               lane issues.
 //   warp 1      TMEM owner and single-thread MMA issuer: four tcgen05.mma
 //               kind::mxf4.block_scale (K = 64 each) per K tile into an fp32 TMEM
-//               accumulator
+//               accumulator (for narrow tiles, into 2 or 4 partial accumulators in
+//               turn, summed by the epilogue)
 //   warps 2-5   epilogue: tcgen05.ld the accumulator (each warp owns one 32-lane TMEM
 //               subpartition), convert, store (or fp32 reduce for split K)
 //   warps 6-13  scale-factor writers, two sets of four taking alternate K tiles: each
@@ -69,11 +73,16 @@ struct GemmShape {
     // 128-row scale slabs a Q tile can touch (a 192-row tile may start 64 rows into one)
     static constexpr int kQChunks = (BN <= 128) ? 1 : 2;
     static constexpr int kSfCols = 8 + 8 * kQChunks;        // 4 columns per atom, 2 atoms per tile
-    // TMEM: two fp32 accumulators of BN columns side by side, then one scale-factor
-    // slot per pipeline stage (the K tile in stage s uses slot s).
+    // Narrow tiles split each accumulator into kSub independent partial sums: the four
+    // MMAs of a K tile rotate over them, so consecutive MMAs do not wait on one another's
+    // result (a 128 x BN x 64 MMA is short next to its latency when BN is small), and the
+    // epilogue adds the partial sums.
+    static constexpr int kSub = BN <= 32 ? 4 : BN == 64 ? 2 : 1;
+    // TMEM: two fp32 accumulators of kSub x BN columns side by side, then one
+    // scale-factor slot per pipeline stage (the K tile in stage s uses slot s).
     static constexpr int kNumAcc = 2;
-    static constexpr int kAccStride = BN;
-    static constexpr int kSfBase = kNumAcc * BN;
+    static constexpr int kAccStride = kSub * BN;
+    static constexpr int kSfBase = kNumAcc * kAccStride;
     static constexpr int kTmemNeed = kSfBase + STAGES * kSfCols;
     static_assert(kTmemNeed <= 512, "tensor memory budget");
     static constexpr int kTmemCols = kTmemNeed <= 32 ? 32 : kTmemNeed <= 64 ? 64
@@ -129,6 +138,16 @@ __device__ __noinline__ bool wait_or_abort_slow(uint64_t* bar, uint32_t parity, 
             }
         }
     }
+}
+
+// The CTA abort flag as a warp-uniform value.
+__device__ __forceinline__ bool cta_aborted(volatile int* abort) { return __any_sync(0xffffffffu, *abort != 0); }
+
+// wait_or_abort by every lane of a warp, with a warp-uniform result: false if any lane
+// gave up.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort, int* err,
+                                          int code) {
+    return __all_sync(0xffffffffu, wait_or_abort(bar, parity, abort, err, code));
 }
 
 struct Unit {
@@ -305,19 +324,24 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer ---
-        if (lane == 0) {
-            int stage = 0;
-            uint32_t phase = 0;
-            uint32_t issued_mask = 0, issued_phase = 0;
-            const int q_slabs = (p.q_rows + 127) / 128;
-            for (int u = blockIdx.x; u < p.total_units && !*abort; u += gridDim.x) {
-                const Unit t = decode_unit(p, u);
-                const int q0 = t.tq * BN;
-                const int slab0 = q0 / 128;
-                const int nchunks = min(S::kQChunks, q_slabs - slab0);
-                const uint32_t bytes = S::kPTileBytes + S::kQTileBytes + S::kSfChunkBytes * (1 + nchunks);
-                for (int kt = t.kt_begin; kt < t.kt_end; ++kt) {
-                    if (!wait_or_abort(&empty[stage], phase ^ 1, abort, p.err, kErrTimeoutProducer)) break;
+        // The whole warp runs the loop, so addresses and coordinates are warp-uniform
+        // values; one elected lane issues the copies.
+        const bool leader = ptx::elect_one();
+        int stage = 0;
+        uint32_t phase = 0;
+        uint32_t issued_mask = 0, issued_phase = 0;
+        const int q_slabs = (p.q_rows + 127) / 128;
+        for (int u = blockIdx.x; u < p.total_units; u += gridDim.x) {
+            if (cta_aborted(abort)) break;
+            const Unit t = decode_unit(p, u);
+            const int q0 = t.tq * BN;
+            const int slab0 = q0 / 128;
+            const int nchunks = min(S::kQChunks, q_slabs - slab0);
+            const uint32_t bytes = S::kPTileBytes + S::kQTileBytes + S::kSfChunkBytes * (1 + nchunks);
+            bool ok = true;
+            for (int kt = t.kt_begin; kt < t.kt_end; ++kt) {
+                if (!warp_wait(&empty[stage], phase ^ 1, abort, p.err, kErrTimeoutProducer)) { ok = false; break; }
+                if (leader) {
                     ptx::mbar_arrive_expect_tx(&full[stage], bytes);
                     ptx::tma_load_2d(smem + L::kOffP + stage * S::kPTileBytes, &tmap_p, &full[stage],
                                      kt * S::kBKBytes, t.tp * S::kBM);
@@ -330,85 +354,93 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         ptx::bulk_load(smem + L::kOffSfQ + (stage * S::kQChunks + c) * S::kSfChunkBytes,
                                        p.sf_q + ((int64_t)(slab0 + c) * p.kb4_pad + 2 * kt) * 512,
                                        S::kSfChunkBytes, &full[stage]);
-                    issued_mask |= 1u << stage;
-                    issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
-                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
                 }
+                __syncwarp();
+                issued_mask |= 1u << stage;
+                issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
+                if (++stage == STAGES) { stage = 0; phase ^= 1; }
             }
-            if (*abort) {
-                // let copies already in flight land before the CTA can exit: wait
-                // (bounded) for the phase of the latest fill of every stage
-                for (int s = 0; s < STAGES; ++s) {
-                    if (!((issued_mask >> s) & 1)) continue;
-                    const uint32_t ph = (issued_phase >> s) & 1;
-                    const uint64_t t0 = global_timer_ns();
-                    while (!ptx::mbar_try_wait(&full[s], ph) && global_timer_ns() - t0 < 100000000ull) {
-                    }
+            if (!ok) break;
+        }
+        if (cta_aborted(abort) && leader) {
+            // let copies already in flight land before the CTA can exit: wait
+            // (bounded) for the phase of the latest fill of every stage
+            for (int s = 0; s < STAGES; ++s) {
+                if (!((issued_mask >> s) & 1)) continue;
+                const uint32_t ph = (issued_phase >> s) & 1;
+                const uint64_t t0 = global_timer_ns();
+                while (!ptx::mbar_try_wait(&full[s], ph) && global_timer_ns() - t0 < 100000000ull) {
                 }
             }
         }
         __syncwarp();
     } else if (warp == 1) {
         // -------------------------------------------------------------- MMA -----
-        if (lane == 0) {
-            int stage = 0;
-            uint32_t phase = 0;
-            int acc = 0;
-            uint32_t acc_phase = 0;
-            bool issued = false;
-            for (int u = blockIdx.x; u < p.total_units && !*abort; u += gridDim.x) {
-                const Unit t = decode_unit(p, u);
-                const uint32_t q_off = (uint32_t)((t.tq * BN) % 128) / 32;
-                if ((q_off & 1) != 0 || q_off * 32 + (BN < 32 ? 32 : BN) > 128 * S::kQChunks) {
-                    // never planned: a scale-factor column offset the MMA is not given
+        // Whole-warp loop with warp-uniform descriptors; the elected lane issues the
+        // MMAs and the commits (a commit tracks the MMAs of the thread that issues it).
+        // A K tile is ready once its scale-factor slot is: the scale-factor warps arrive
+        // on sf_full only after they have waited for the same fill's full barrier.
+        const bool leader = ptx::elect_one();
+        int stage = 0;
+        uint32_t phase = 0;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        bool issued = false;
+        for (int u = blockIdx.x; u < p.total_units; u += gridDim.x) {
+            if (cta_aborted(abort)) break;
+            const Unit t = decode_unit(p, u);
+            const uint32_t q_off = (uint32_t)((t.tq * BN) % 128) / 32;
+            if ((q_off & 1) != 0 || q_off * 32 + (BN < 32 ? 32 : BN) > 128 * S::kQChunks) {
+                // never planned: a scale-factor column offset the MMA is not given
+                if (leader) {
                     atomicExch(p.err, kErrSfOffset);
                     *abort = 1;
-                    break;
                 }
-                if (!wait_or_abort(&acc_empty[acc], acc_phase ^ 1, abort, p.err, kErrTimeoutMma)) break;
+                __syncwarp();
+                break;
+            }
+            if (!warp_wait(&acc_empty[acc], acc_phase ^ 1, abort, p.err, kErrTimeoutMma)) break;
+            ptx::tc_fence_after();
+            const uint32_t d_tmem = tmem + acc * S::kAccStride;
+            bool ok = true;
+            for (int kt = t.kt_begin; kt < t.kt_end; ++kt) {
+                if (!warp_wait(&sf_full[stage], phase, abort, p.err, kErrTimeoutMma)) { ok = false; break; }
                 ptx::tc_fence_after();
-                const uint32_t d_tmem = tmem + acc * S::kAccStride;
-                bool ok = true;
-                for (int kt = t.kt_begin; kt < t.kt_end; ++kt) {
-                    if (!wait_or_abort(&full[stage], phase, abort, p.err, kErrTimeoutMma)) { ok = false; break; }
-                    // scale factors of this K tile, written into slot `stage` by the
-                    // scale-factor warps
-                    if (!wait_or_abort(&sf_full[stage], phase, abort, p.err, kErrTimeoutMma)) {
-                        ok = false;
-                        break;
-                    }
-                    ptx::tc_fence_after();
-                    const uint32_t sf_base = tmem + S::kSfBase + stage * S::kSfCols;
-                    const uint64_t adesc = ptx::smem_desc_sw128(ptx::smem_u32(smem + L::kOffP + stage * S::kPTileBytes));
-                    const uint64_t bdesc = ptx::smem_desc_sw128(ptx::smem_u32(smem + L::kOffQ + stage * S::kQTileBytes));
+                const uint32_t sf_base = tmem + S::kSfBase + stage * S::kSfCols;
+                const uint64_t adesc = ptx::smem_desc_sw128(ptx::smem_u32(smem + L::kOffP + stage * S::kPTileBytes));
+                const uint64_t bdesc = ptx::smem_desc_sw128(ptx::smem_u32(smem + L::kOffQ + stage * S::kQTileBytes));
+                if (leader) {
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk) {
                         const uint32_t a = kk >> 1;
                         const uint32_t sfid = (kk & 1) * 2;
                         const uint32_t sfa = (sf_base + 4 * a) | (sfid << 30);
                         const uint32_t sfb = (sf_base + 8 + a * 4 * S::kQChunks + q_off) | (sfid << 30);
-                        ptx::mma_mxf4(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, ptx::idesc_mxf4(BN, sfid, sfid),
-                                      sfa, sfb, (kt > t.kt_begin || kk > 0) ? 1u : 0u);
+                        ptx::mma_mxf4(d_tmem + (kk % S::kSub) * BN, adesc + 2 * kk, bdesc + 2 * kk,
+                                      ptx::idesc_mxf4(BN, sfid, sfid), sfa, sfb,
+                                      (kt > t.kt_begin || kk >= S::kSub) ? 1u : 0u);
                     }
-                    issued = true;
                     ptx::tc_commit(&empty[stage]);
-                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
                 }
-                if (!ok) break;
-                ptx::tc_commit(&acc_full[acc]);
-                if (S::kNumAcc == 2) {
-                    acc ^= 1;
-                    if (acc == 0) acc_phase ^= 1;
-                } else {
-                    acc_phase ^= 1;
-                }
+                __syncwarp();
+                issued = true;
+                if (++stage == STAGES) { stage = 0; phase ^= 1; }
             }
-            if (*abort && issued) {
-                // wait (bounded) for every MMA this thread issued before TMEM is freed
-                ptx::tc_commit(drain);
-                const uint64_t t0 = global_timer_ns();
-                while (!ptx::mbar_try_wait(drain, 0) && global_timer_ns() - t0 < 100000000ull) {
-                }
+            if (!ok) break;
+            if (leader) ptx::tc_commit(&acc_full[acc]);
+            __syncwarp();
+            if (S::kNumAcc == 2) {
+                acc ^= 1;
+                if (acc == 0) acc_phase ^= 1;
+            } else {
+                acc_phase ^= 1;
+            }
+        }
+        if (cta_aborted(abort) && issued && leader) {
+            // wait (bounded) for every MMA this thread issued before TMEM is freed
+            ptx::tc_commit(drain);
+            const uint64_t t0 = global_timer_ns();
+            while (!ptx::mbar_try_wait(drain, 0) && global_timer_ns() - t0 < 100000000ull) {
             }
         }
         __syncwarp();
@@ -478,6 +510,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             for (int c = 0; c < BN / CW; ++c) {
                 uint32_t r[CW];
                 tmem_load_chunk<CW>(taddr + c * CW, r);
+                if (S::kSub > 1) {
+                    uint32_t r2[CW];
+#pragma unroll
+                    for (int sub = 1; sub < S::kSub; ++sub) {
+                        tmem_load_chunk<CW>(taddr + sub * BN + c * CW, r2);
+                        ptx::tmem_ld_wait();
+#pragma unroll
+                        for (int j = 0; j < CW; ++j)
+                            r[j] = __float_as_uint(__uint_as_float(r[j]) + __uint_as_float(r2[j]));
+                    }
+                }
                 ptx::tmem_ld_wait();
                 store_chunk<CW>(p, prow, t.tq * BN + c * CW, r);
             }
