@@ -19,7 +19,9 @@
 //               accumulator (for narrow tiles, into 2 or 4 partial accumulators in
 //               turn, summed by the epilogue)
 //   warps 2-5   epilogue: tcgen05.ld the accumulator (each warp owns one 32-lane TMEM
-//               subpartition), convert, store (or fp32 reduce for split K)
+//               subpartition), convert, and either stage 32 x 32 boxes in shared memory
+//               for TMA tensor stores (wide row-major tiles) or store directly (decode's
+//               transposed tiles, fp32 reductions for split K, unaligned outputs)
 //   warps 6-13  scale-factor writers, two sets of four taking alternate K tiles: each
 //               warp reads the scale atoms of a K tile from shared memory and writes
 //               them into its TMEM subpartition with tcgen05.st, so the tensor pipe
@@ -54,6 +56,8 @@ struct GemmParams {
     int32_t atomic;          // 1: fp32 reduction into out (split K)
     int32_t transpose_out;   // 1: out[q * ldo + p], 0: out[p * ldo + q]
     int32_t vec_ok;          // 1: out and ldo allow 16-byte vector stores
+    int32_t tma_store;       // 1: epilogue stages 32 x 32 output boxes in shared memory and
+                             //    writes them with TMA stores (row-major, not atomic, vec_ok)
     int* err;                // device error word
 };
 
@@ -88,6 +92,10 @@ struct GemmShape {
     static constexpr int kTmemCols = kTmemNeed <= 32 ? 32 : kTmemNeed <= 64 ? 64
                                    : kTmemNeed <= 128 ? 128 : kTmemNeed <= 256 ? 256 : 512;
     static constexpr int kChunkCols = BN < 32 ? BN : 32;    // epilogue TMEM load width
+    // Output staging for TMA stores (wide tiles only): one box of 32 rows x 64 bytes
+    // (32 bf16 or 16 fp32 columns) per epilogue warp.
+    static constexpr int kStageBoxBytes = 32 * 64;
+    static constexpr int kStagingBytes = BN >= 128 ? 4 * kStageBoxBytes : 0;
 };
 
 template <int BN, int STAGES>
@@ -97,7 +105,8 @@ struct GemmSmem {
     static constexpr int kOffQ = kOffP + STAGES * S::kPTileBytes;
     static constexpr int kOffSfP = kOffQ + STAGES * S::kQTileBytes;
     static constexpr int kOffSfQ = kOffSfP + STAGES * S::kSfChunkBytes;
-    static constexpr int kOffBar = kOffSfQ + STAGES * S::kQChunks * S::kSfChunkBytes;
+    static constexpr int kOffStaging = kOffSfQ + STAGES * S::kQChunks * S::kSfChunkBytes;   // 1 KB aligned
+    static constexpr int kOffBar = kOffStaging + S::kStagingBytes;
     static constexpr int kNumBars = 3 * STAGES + 4 + 1;
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;
     static constexpr int kBytes = kOffMisc + 16;
@@ -273,8 +282,8 @@ constexpr int kGemmThreads = 32 * (6 + 4 * kSfWarpSets);
 
 template <int BN, int STAGES>
 __global__ void __launch_bounds__(kGemmThreads, 1)
-    gemm_mxf4_kernel(const __grid_constant__ CUtensorMap tmap_p,
-                     const __grid_constant__ CUtensorMap tmap_q, const GemmParams p) {
+    gemm_mxf4_kernel(const __grid_constant__ CUtensorMap tmap_p, const __grid_constant__ CUtensorMap tmap_q,
+                     const __grid_constant__ CUtensorMap tmap_y, const GemmParams p) {
     using S = GemmShape<BN, STAGES>;
     using L = GemmSmem<BN, STAGES>;
     extern __shared__ uint8_t smem_raw[];
@@ -309,6 +318,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         ptx::fence_proxy_async_smem();
         ptx::prefetch_tensormap(&tmap_p);
         ptx::prefetch_tensormap(&tmap_q);
+        if (S::kStagingBytes > 0 && p.tma_store) ptx::prefetch_tensormap(&tmap_y);
     }
     if (warp == 1) {
         ptx::tmem_alloc(tmem_slot, S::kTmemCols);
@@ -500,6 +510,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         int acc = 0;
         uint32_t acc_phase = 0;
         constexpr int CW = S::kChunkCols;
+        const bool via_tma = S::kStagingBytes > 0 && p.tma_store;
+        const uint32_t staging = ptx::smem_u32(smem + L::kOffStaging) + quad * S::kStageBoxBytes;
         for (int u = blockIdx.x; u < p.total_units && !*abort; u += gridDim.x) {
             const Unit t = decode_unit(p, u);
             if (!wait_or_abort(&acc_full[acc], acc_phase, abort, p.err, kErrTimeoutEpilogue)) break;
@@ -522,11 +534,57 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     }
                 }
                 ptx::tmem_ld_wait();
-                store_chunk<CW>(p, prow, t.tq * BN + c * CW, r);
+                if (!via_tma) {
+                    store_chunk<CW>(p, prow, t.tq * BN + c * CW, r);
+                    continue;
+                }
+                if (c == BN / CW - 1) {
+                    // the accumulator is in registers: hand it back to the MMA warp now
+                    ptx::tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) ptx::mbar_arrive(&acc_empty[acc]);
+                }
+                // Stage this warp's 32 rows x 64 bytes box in shared memory in the tensor
+                // map's 64-byte-swizzled layout (row = lane; 16-byte piece j of the row at
+                // j ^ ((row >> 1) & 3)), then one lane stores the box. The buffer is
+                // rewritten only after the previous store from it has finished reading it.
+                const int boxes = p.out_bf16 ? 1 : 2;           // 32 columns = 64 or 128 bytes
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    if (h >= boxes) break;
+                    const int bx = t.tq * BN + c * CW + 16 * h, by = t.tp * S::kBM + quad * 32;
+                    if (bx >= p.q_rows || by >= p.p_rows) break;     // box wholly outside y
+                    if (lane == 0) ptx::bulk_wait_group_read<0>();
+                    __syncwarp();
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        uint32_t w[4];
+                        if (p.out_bf16) {
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                __nv_bfloat162 v = __floats2bfloat162_rn(__uint_as_float(r[8 * j + 2 * e]),
+                                                                         __uint_as_float(r[8 * j + 2 * e + 1]));
+                                w[e] = *reinterpret_cast<uint32_t*>(&v);
+                            }
+                        } else {
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) w[e] = r[16 * h + 4 * j + e];
+                        }
+                        ptx::sts128(staging + lane * 64 + ((j ^ ((lane >> 1) & 3)) << 4), w[0], w[1], w[2], w[3]);
+                    }
+                    ptx::fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        ptx::tma_store_2d(&tmap_y, staging, bx, by);
+                        ptx::bulk_commit_group();
+                    }
+                }
             }
-            ptx::tc_fence_before();
-            __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(&acc_empty[acc]);
+            if (!via_tma) {
+                ptx::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(&acc_empty[acc]);
+            }
             if (S::kNumAcc == 2) {
                 acc ^= 1;
                 if (acc == 0) acc_phase ^= 1;
@@ -534,6 +592,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 acc_phase ^= 1;
             }
         }
+        // the staging buffers must outlive the stores that read them
+        if (via_tma && lane == 0) ptx::bulk_wait_group_all();
+        __syncwarp();
     }
 
     ptx::tc_fence_before();

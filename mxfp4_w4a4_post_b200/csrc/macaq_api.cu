@@ -232,9 +232,23 @@ bool encode_codes_map(CUtensorMap* map, const uint8_t* codes, int64_t rows, int6
     return r == CUDA_SUCCESS;
 }
 
+// Output tensor map for the TMA-store epilogue: boxes of 32 rows x 64 bytes (32 bf16 or
+// 16 fp32 columns), 64-byte swizzle.
+bool encode_out_map(CUtensorMap* map, void* y, int64_t M, int64_t N, int64_t ldy, bool bf16) {
+    const int64_t esz = bf16 ? 2 : 4;
+    cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)M};
+    cuuint64_t strides[1] = {(cuuint64_t)(ldy * esz)};
+    cuuint32_t box[2] = {(cuuint32_t)(64 / esz), 32};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = g_encode(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, y, dims,
+                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                          CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 template <int BN, int STAGES>
-macaq_status launch_gemm_bn(const CUtensorMap& mp, const CUtensorMap& mq, const GemmParams& gp,
-                            int grid, cudaStream_t stream) {
+macaq_status launch_gemm_bn(const CUtensorMap& mp, const CUtensorMap& mq, const CUtensorMap& my,
+                            const GemmParams& gp, int grid, cudaStream_t stream) {
     using L = GemmSmem<BN, STAGES>;
     static_assert(L::kAlloc <= 232448, "shared memory budget");
     static std::atomic<uint64_t> configured_mask{0};
@@ -247,7 +261,8 @@ macaq_status launch_gemm_bn(const CUtensorMap& mp, const CUtensorMap& mq, const 
             return MACAQ_ERR_CUDA;
         configured_mask.fetch_or(bit);
     }
-    return launch_pdl(gemm_mxf4_kernel<BN, STAGES>, dim3(grid), dim3(kGemmThreads), L::kAlloc, stream, mp, mq, gp) ==
+    return launch_pdl(gemm_mxf4_kernel<BN, STAGES>, dim3(grid), dim3(kGemmThreads), L::kAlloc, stream, mp, mq, my,
+                      gp) ==
                    cudaSuccess
                ? MACAQ_OK
                : MACAQ_ERR_CUDA;
@@ -327,14 +342,19 @@ macaq_status run_gemm(const uint8_t* a_codes, const uint8_t* a_scales, int64_t M
         gp.atomic = 0;
         gp.out_bf16 = out == MACAQ_OUT_BF16 ? 1 : 0;
         gp.vec_ok = (aligned16(y) && (ldy * esz) % 16 == 0) ? 1 : 0;
+        // wide row-major tiles store through TMA (an aligned output is all it needs)
+        gp.tma_store = (!g.swap && g.bn >= 128 && gp.vec_ok) ? 1 : 0;
     }
+    CUtensorMap my;
+    std::memset(&my, 0, sizeof(my));
+    if (gp.tma_store && !encode_out_map(&my, y, M, N, ldy, out == MACAQ_OUT_BF16)) return MACAQ_ERR_CUDA;
 
     switch (g.bn) {
-        case 16: st = launch_gemm_bn<16, 8>(mp, mq, gp, g.grid, stream); break;
-        case 32: st = launch_gemm_bn<32, 8>(mp, mq, gp, g.grid, stream); break;
-        case 64: st = launch_gemm_bn<64, 8>(mp, mq, gp, g.grid, stream); break;
-        case 128: st = launch_gemm_bn<128, 6>(mp, mq, gp, g.grid, stream); break;
-        default: st = launch_gemm_bn<192, 5>(mp, mq, gp, g.grid, stream); break;
+        case 16: st = launch_gemm_bn<16, 8>(mp, mq, my, gp, g.grid, stream); break;
+        case 32: st = launch_gemm_bn<32, 8>(mp, mq, my, gp, g.grid, stream); break;
+        case 64: st = launch_gemm_bn<64, 8>(mp, mq, my, gp, g.grid, stream); break;
+        case 128: st = launch_gemm_bn<128, 6>(mp, mq, my, gp, g.grid, stream); break;
+        default: st = launch_gemm_bn<192, 5>(mp, mq, my, gp, g.grid, stream); break;
     }
     if (st != MACAQ_OK) return st;
     if (g.atomic) {

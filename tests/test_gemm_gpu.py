@@ -1,7 +1,8 @@
 """Parity of the block-scaled FP4 GEMM (tcgen05 kind::mxf4) with the oracle's fp64 sum
 of decoded products. One-hot operands pin the nibble order and the scale layout;
 random codes and scales cover every tile path (swapped decode tiles of width 16..128,
-prefill tiles of width 128/224, split K, ragged M/N/K)."""
+prefill tiles of width 128/192, split K, ragged M/N/K) and every output path (TMA tensor
+stores of staged boxes, direct stores, transposed stores, fp32 reductions)."""
 import numpy as np
 import pytest
 
@@ -111,3 +112,36 @@ def test_extreme_scales(mq):
     w, sw = random_mxfp4(rng, N, K, 240, 252)
     y = host(gpu_gemm(mq, a, sa, w, sw, K))
     assert_gemm_close(y, oracle.gemm_fp64(a, sa, w, sw, K), "extreme scales")
+
+
+# (M, N, K, dtype, extra columns of row padding): rows whose byte length is a multiple of
+# 16 go through the staged TMA-store epilogue (boxes clipped at ragged M and N edges),
+# others through direct stores; padding columns of a strided output stay untouched.
+OUTPUT_CASES = [
+    (300, 200, 512, "bf16", 0), (300, 200, 512, "f32", 0), (257, 333, 256, "bf16", 0),
+    (300, 200, 512, "bf16", 24), (300, 200, 512, "f32", 12), (640, 1000, 768, "bf16", 0),
+]
+
+
+@pytest.mark.parametrize("M,N,K,dt,pad", OUTPUT_CASES)
+def test_output_paths(mq, M, N, K, dt, pad):
+    import torch
+    rng = np.random.default_rng(M + 3 * N + K + pad)
+    a, sa = random_mxfp4(rng, M, K)
+    w, sw = random_mxfp4(rng, N, K)
+    y32 = host(gpu_gemm(mq, a, sa, w, sw, K, out="f32"))
+    rows = np.unique(np.concatenate([rng.choice(M, 40, replace=False), [0, M - 1]]))
+    assert_gemm_close(y32[rows], oracle.gemm_fp64(a, sa, w, sw, K, rows=rows), f"f32 {M}x{N}x{K}")
+    tdt = torch.bfloat16 if dt == "bf16" else torch.float32
+    big = torch.full((M, N + pad), float("nan"), dtype=tdt, device="cuda")
+    y = big[:, :N]
+    pw = mq.PreparedWeight(u8_dev(w), u8_dev(oracle.swizzle_scales(sw, K)),
+                           torch.ones(K, dtype=torch.float32, device="cuda"), N, K)
+    mq.gemm_mxfp4(u8_dev(a), u8_dev(oracle.swizzle_scales(sa, K)), M, pw, y=y)
+    torch.cuda.synchronize()
+    if pad:
+        assert torch.isnan(big[:, N:]).all().item(), "padding columns were written"
+    if dt == "bf16":
+        assert_bf16_matches_f32(y, torch.from_numpy(y32).cuda(), f"bf16 {M}x{N}x{K} pad {pad}")
+    else:
+        assert np.array_equal(host(y), y32), f"f32 {M}x{N}x{K} pad {pad}"
