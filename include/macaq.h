@@ -84,7 +84,8 @@ size_t macaq_codes_bytes(int64_t rows, int64_t K);
 size_t macaq_scales_bytes(int64_t rows, int64_t K);
 
 /* Device workspace macaq_gemm_mxfp4 needs for an M x N x K product with output
- * `out` (an fp32 split-K accumulator when the library splits K; may be 0). */
+ * `out`: when the library splits K, one fp32 sum per output tile, an arrival count per
+ * tile and a flag per CTA (the kernel clears what it needs itself); 0 otherwise. */
 size_t macaq_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, macaq_out_dtype out);
 
 /* Device workspace macaq_linear_w4a4 needs: the activation codes and scales, plus
@@ -133,7 +134,9 @@ macaq_status macaq_quant_act(const void* x_bf16, int64_t M, int64_t K, int64_t l
  *            to its element size (16-byte alignment of y and of ldy * element size
  *            enables vector stores)
  *   workspace device, >= macaq_gemm_workspace_bytes(M, N, K, out), 256-byte aligned
- *            (may be NULL when that size is 0); contents are scratch
+ *            (may be NULL when that size is 0). Contents are scratch and need no
+ *            clearing (each call tags its split-K flags with a value unique to the
+ *            call); two calls that may run at the same time must not share it.
  * M >= 1. Also the entry point for externally refined weight codes/scales. */
 macaq_status macaq_gemm_mxfp4(const uint8_t* a_codes, const uint8_t* a_scales, int64_t M,
                               const macaq_weight* w, void* y, int64_t ldy, macaq_out_dtype out,
@@ -160,7 +163,7 @@ macaq_status macaq_linear_w4a4(const void* x_bf16, int64_t M, int64_t ldx, const
  * libraries none of it, and latency-critical loops where allocating or freeing would
  * stall the device (cudaFree synchronises it) or could fail under memory pressure in the
  * middle of serving. This entry point takes no workspace: the activation codes, scales
- * and split-K accumulator live in one file-scope static device array of
+ * and split-K partial sums live in one file-scope static device array of
  * MACAQ_NOALLOC_SCRATCH_BYTES. The caller still passes x, the prepared weight and y,
  * with the same meaning, layout and alignment rules as macaq_linear_w4a4 (fused = 0).
  *
@@ -170,9 +173,10 @@ macaq_status macaq_linear_w4a4(const void* x_bf16, int64_t M, int64_t ldx, const
  * - The first call on each device looks up the array's device address (once per device,
  *   with that device current); make that first call before any stream capture.
  * - Every call on a device shares the one array, and the array keeps the last call's
- *   contents. Whatever must start at zero is cleared by each call on its stream. Calls
- *   whose executions overlap on the GPU (other streams, or no ordering between them)
- *   race on the array and give undefined results: order them on one stream.
+ *   contents. Nothing in it needs to start at zero: every call overwrites what it reads
+ *   and tags its split-K flags with a value unique to the call. Calls whose executions
+ *   overlap on the GPU (other streams, or no ordering between them) race on the array
+ *   and give undefined results: order them on one stream.
  * - Allocates nothing: no cudaMalloc, cudaFree or allocating library routine. */
 macaq_status macaq_linear_w4a4_noalloc(const void* x_bf16, int64_t M, int64_t ldx,
                                        const macaq_weight* w, void* y, int64_t ldy,

@@ -19,9 +19,11 @@
 //               accumulator (for narrow tiles, into 2 or 4 partial accumulators in
 //               turn, summed by the epilogue)
 //   warps 2-5   epilogue: tcgen05.ld the accumulator (each warp owns one 32-lane TMEM
-//               subpartition), convert, and either stage 32 x 32 boxes in shared memory
+//               subpartition), convert, and either stage 32-row boxes in shared memory
 //               for TMA tensor stores (wide row-major tiles) or store directly (decode's
-//               transposed tiles, fp32 reductions for split K, unaligned outputs)
+//               transposed tiles, unaligned outputs). With split K every split adds its
+//               fp32 partial into a workspace accumulator (zeroed by the kernel itself)
+//               with vector reductions; a small kernel then writes y from it.
 //   warps 6-13  scale-factor writers, two sets of four taking alternate K tiles: each
 //               warp reads the scale atoms of a K tile from shared memory and writes
 //               them into its TMEM subpartition with tcgen05.st, so the tensor pipe
@@ -29,7 +31,9 @@
 // Accumulators are double-buffered in TMEM when they fit, so the epilogue of one tile
 // overlaps the MMAs of the next. Every mbarrier wait is bounded by a wall-clock limit;
 // a kernel that gives up records an error code, drains what it issued, frees its TMEM
-// and returns.
+// and returns. The one split-K wait (for every CTA to have zeroed its slice of the
+// workspace, done first thing) always ends: all CTAs are resident at once (grid <= SMs,
+// one CTA per SM). It is bounded all the same.
 #pragma once
 
 #include <cstdint>
@@ -43,7 +47,7 @@ namespace macaq {
 struct GemmParams {
     const uint8_t* sf_p;     // scale atoms of P
     const uint8_t* sf_q;     // scale atoms of Q
-    void* out;               // output, or the fp32 accumulator when atomic
+    void* out;               // y, or the fp32 split-K accumulator when atomic
     int64_t ldo;             // leading dimension of out, elements
     int32_t p_rows, q_rows;  // logical rows of P and Q
     int32_t k_tiles;         // ceil(K / 256)
@@ -53,15 +57,28 @@ struct GemmParams {
     int32_t total_units;     // tiles_p * tiles_q * splits
     int32_t group_p;         // raster group height (in P tiles)
     int32_t out_bf16;        // 1: bf16 output, 0: fp32 (ignored when atomic)
-    int32_t atomic;          // 1: fp32 reduction into out (split K)
+    int32_t atomic;          // 1: split K, fp32 vector reductions into out
     int32_t transpose_out;   // 1: out[q * ldo + p], 0: out[p * ldo + q]
     int32_t vec_ok;          // 1: out and ldo allow 16-byte vector stores
     int32_t tma_store;       // 1: epilogue stages 32 x 32 output boxes in shared memory and
-                             //    writes them with TMA stores (row-major, not atomic, vec_ok)
+                             //    writes them with TMA stores (row-major tiles, vec_ok)
     int* err;                // device error word
+    // Split K (atomic): the accumulator `out` starts at zero without a separate memset.
+    // First thing, the epilogue warps of every CTA zero their slice of it and set their
+    // CTA's flag to `epoch` (a value unique to the call, so flags left by earlier calls
+    // never match); before its first reduction a CTA waits until every flag is set.
+    int64_t zero_vec4;               // 16-byte words of the accumulator
+    unsigned long long* cta_flags;   // [gridDim.x]
+    unsigned long long epoch;
 };
 
-enum : int { kErrTimeoutProducer = 1, kErrTimeoutMma = 2, kErrTimeoutEpilogue = 3, kErrSfOffset = 4 };
+enum : int {
+    kErrTimeoutProducer = 1,
+    kErrTimeoutMma = 2,
+    kErrTimeoutEpilogue = 3,
+    kErrSfOffset = 4,
+    kErrTimeoutSplit = 5
+};
 
 template <int BN, int STAGES>
 struct GemmShape {
@@ -91,7 +108,7 @@ struct GemmShape {
     static_assert(kTmemNeed <= 512, "tensor memory budget");
     static constexpr int kTmemCols = kTmemNeed <= 32 ? 32 : kTmemNeed <= 64 ? 64
                                    : kTmemNeed <= 128 ? 128 : kTmemNeed <= 256 ? 256 : 512;
-    static constexpr int kChunkCols = BN < 32 ? BN : 32;    // epilogue TMEM load width
+    static constexpr int kChunkCols = BN <= 32 ? 16 : 32;   // epilogue TMEM load width
     // Output staging for TMA stores (wide tiles only): one box of 32 rows x 64 bytes
     // (32 bf16 or 16 fp32 columns) per epilogue warp.
     static constexpr int kStageBoxBytes = 32 * 64;
@@ -160,7 +177,7 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
 }
 
 struct Unit {
-    int tp, tq, kt_begin, kt_end;
+    int tile, split, tp, tq, kt_begin, kt_end;
 };
 
 __device__ __forceinline__ Unit decode_unit(const GemmParams& p, int u) {
@@ -171,6 +188,8 @@ __device__ __forceinline__ Unit decode_unit(const GemmParams& p, int u) {
     const int r = tile - g * per_group;
     const int gp = min(p.group_p, p.tiles_p - g * p.group_p);
     Unit x;
+    x.tile = tile;
+    x.split = split;
     x.tp = g * p.group_p + r % gp;
     x.tq = r / gp;
     x.kt_begin = split * p.k_tiles_per_split;
@@ -255,6 +274,35 @@ __device__ __forceinline__ void store_chunk(const GemmParams& p, int prow, int q
             for (int j = 0; j < CW; ++j)
                 if (q_base + j < p.q_rows) o[j] = __uint_as_float(r[j]);
         }
+    }
+}
+
+// Split-K zeroing protocol (gpu scope): a CTA zeroes its slice, fences, and one thread
+// releases its flag; the epilogue lanes acquire every CTA's flag before reducing.
+__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long* f) {
+    unsigned long long v;
+    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(f) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_release_u64(unsigned long long* f, unsigned long long v) {
+    asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(f), "l"(v) : "memory");
+}
+// Wait (bounded, ~2 s) until *flag == epoch. On give-up record kErrTimeoutSplit, raise
+// the CTA abort flag and return false. Polls sleep briefly: the flag lives in L2.
+__device__ __noinline__ bool wait_split_flag(const unsigned long long* flag, unsigned long long epoch,
+                                             volatile int* abort, int* err) {
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t it = 0;; ++it) {
+        if (ld_acquire_u64(flag) == epoch) return true;
+        if ((it & 15) == 15) {
+            if (*abort) return false;
+            if (global_timer_ns() - t0 > 2000000000ull) {
+                atomicExch(err, kErrTimeoutSplit);
+                *abort = 1;
+                return false;
+            }
+        }
+        __nanosleep(128);
     }
 }
 
@@ -510,16 +558,83 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         int acc = 0;
         uint32_t acc_phase = 0;
         constexpr int CW = S::kChunkCols;
+        constexpr int NCH = BN / CW;
         const bool via_tma = S::kStagingBytes > 0 && p.tma_store;
         const uint32_t staging = ptx::smem_u32(smem + L::kOffStaging) + quad * S::kStageBoxBytes;
+        bool zeroed = false;
+        if (p.atomic) {
+            // zero this CTA's slice of the split-K accumulator, then flag it
+            const int et = threadIdx.x - 64;                     // 0..127 over warps 2-5
+            const int64_t per = (p.zero_vec4 + gridDim.x - 1) / gridDim.x;
+            const int64_t b0 = (int64_t)blockIdx.x * per, b1 = min(p.zero_vec4, b0 + per);
+            float4* z = reinterpret_cast<float4*>(p.out);
+            for (int64_t i = b0 + et; i < b1; i += 128) z[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+            __threadfence();
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+            if (et == 0) st_release_u64(p.cta_flags + blockIdx.x, p.epoch);
+        }
         for (int u = blockIdx.x; u < p.total_units && !*abort; u += gridDim.x) {
             const Unit t = decode_unit(p, u);
             if (!wait_or_abort(&acc_full[acc], acc_phase, abort, p.err, kErrTimeoutEpilogue)) break;
             ptx::tc_fence_after();
             const int prow = t.tp * S::kBM + quad * 32 + lane;
             const uint32_t taddr = tmem + acc * S::kAccStride + ((uint32_t)(quad * 32) << 16);
+            if (p.atomic && !zeroed) {
+                // once per kernel: every CTA has zeroed its slice of the accumulator
+                bool ok = true;
+                for (int i = lane; i < (int)gridDim.x && ok; i += 32)
+                    ok = wait_split_flag(p.cta_flags + i, p.epoch, abort, p.err);
+                if (!__all_sync(0xffffffffu, ok)) break;
+                zeroed = true;
+            }
+            // write chunk c of y from registers: staged TMA store or direct stores
+            auto emit = [&](int c, uint32_t (&r)[CW]) {
+                if constexpr (S::kStagingBytes > 0) {
+                    if (via_tma) {
+                        // Stage this warp's box of 32 rows x 64 bytes in shared memory in the
+                        // tensor map's 64-byte-swizzled layout (row = lane; 16-byte piece j of
+                        // the row at j ^ ((row >> 1) & 3)), then one lane stores the box. The
+                        // buffer is rewritten only after the previous store from it has been
+                        // read out.
+                        const int boxes = p.out_bf16 ? 1 : 2;     // 32 columns = 64 or 128 bytes
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            if (h >= boxes) break;
+                            const int bx = t.tq * BN + c * CW + 16 * h, by = t.tp * S::kBM + quad * 32;
+                            if (bx >= p.q_rows || by >= p.p_rows) break;   // box wholly outside y
+                            if (lane == 0) ptx::bulk_wait_group_read<0>();
+                            __syncwarp();
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) {
+                                uint32_t w[4];
+                                if (p.out_bf16) {
+#pragma unroll
+                                    for (int e = 0; e < 4; ++e) {
+                                        __nv_bfloat162 v = __floats2bfloat162_rn(
+                                            __uint_as_float(r[8 * j + 2 * e]), __uint_as_float(r[8 * j + 2 * e + 1]));
+                                        w[e] = *reinterpret_cast<uint32_t*>(&v);
+                                    }
+                                } else {
+#pragma unroll
+                                    for (int e = 0; e < 4; ++e) w[e] = r[16 * h + 4 * j + e];
+                                }
+                                ptx::sts128(staging + lane * 64 + ((j ^ ((lane >> 1) & 3)) << 4), w[0], w[1], w[2],
+                                            w[3]);
+                            }
+                            ptx::fence_proxy_async_smem();
+                            __syncwarp();
+                            if (lane == 0) {
+                                ptx::tma_store_2d(&tmap_y, staging, bx, by);
+                                ptx::bulk_commit_group();
+                            }
+                        }
+                        return;
+                    }
+                }
+                store_chunk<CW>(p, prow, t.tq * BN + c * CW, r);
+            };
 #pragma unroll 1
-            for (int c = 0; c < BN / CW; ++c) {
+            for (int c = 0; c < NCH; ++c) {
                 uint32_t r[CW];
                 tmem_load_chunk<CW>(taddr + c * CW, r);
                 if (S::kSub > 1) {
@@ -534,56 +649,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     }
                 }
                 ptx::tmem_ld_wait();
-                if (!via_tma) {
-                    store_chunk<CW>(p, prow, t.tq * BN + c * CW, r);
-                    continue;
-                }
-                if (c == BN / CW - 1) {
+                if (c == NCH - 1) {
                     // the accumulator is in registers: hand it back to the MMA warp now
                     ptx::tc_fence_before();
                     __syncwarp();
                     if (lane == 0) ptx::mbar_arrive(&acc_empty[acc]);
                 }
-                // Stage this warp's 32 rows x 64 bytes box in shared memory in the tensor
-                // map's 64-byte-swizzled layout (row = lane; 16-byte piece j of the row at
-                // j ^ ((row >> 1) & 3)), then one lane stores the box. The buffer is
-                // rewritten only after the previous store from it has finished reading it.
-                const int boxes = p.out_bf16 ? 1 : 2;           // 32 columns = 64 or 128 bytes
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    if (h >= boxes) break;
-                    const int bx = t.tq * BN + c * CW + 16 * h, by = t.tp * S::kBM + quad * 32;
-                    if (bx >= p.q_rows || by >= p.p_rows) break;     // box wholly outside y
-                    if (lane == 0) ptx::bulk_wait_group_read<0>();
-                    __syncwarp();
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        uint32_t w[4];
-                        if (p.out_bf16) {
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                __nv_bfloat162 v = __floats2bfloat162_rn(__uint_as_float(r[8 * j + 2 * e]),
-                                                                         __uint_as_float(r[8 * j + 2 * e + 1]));
-                                w[e] = *reinterpret_cast<uint32_t*>(&v);
-                            }
-                        } else {
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) w[e] = r[16 * h + 4 * j + e];
-                        }
-                        ptx::sts128(staging + lane * 64 + ((j ^ ((lane >> 1) & 3)) << 4), w[0], w[1], w[2], w[3]);
-                    }
-                    ptx::fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0) {
-                        ptx::tma_store_2d(&tmap_y, staging, bx, by);
-                        ptx::bulk_commit_group();
-                    }
-                }
-            }
-            if (!via_tma) {
-                ptx::tc_fence_before();
-                __syncwarp();
-                if (lane == 0) ptx::mbar_arrive(&acc_empty[acc]);
+                emit(c, r);
             }
             if (S::kNumAcc == 2) {
                 acc ^= 1;

@@ -5,6 +5,7 @@
 
 #include <algorithm>
 #include <atomic>
+#include <chrono>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -160,64 +161,103 @@ struct GemmPlan {
     int splits, kps;
     int group_p;
     int grid;
-    bool atomic;
 };
 
+// Estimated SM cycles per 256-wide K tile of a 128 x bn tile: the four MMAs take about
+// 2.4 bn cycles at the measured tensor rate, and a K tile costs ~400 cycles of copies,
+// barriers and issue however narrow it is.
+inline double ktile_cycles(int bn) { return std::max(400.0, 2.42 * bn); }
+// Extra cost of splitting K: zeroing the accumulator and the finalize kernel that
+// converts it (~4 us), plus the fp32 reductions of every unit's 128 x bn tile, which
+// L2 absorbs at an estimated 800 bytes per cycle.
+constexpr double kSplitCycles = 8000.0;
+constexpr double kReduceBytesPerCycle = 800.0;
+
 GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, int num_sms) {
-    GemmPlan g{};
-    g.k_tiles = (int)cdiv(K, 256);
-    int64_t p_rows, q_rows;
-    if (M <= 128) {
-        g.swap = true;
-        g.bn = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : 128;
-        p_rows = N;
-        q_rows = M;
-    } else {
-        g.swap = false;
-        g.bn = N <= 128 ? 128 : 192;
-        p_rows = M;
-        q_rows = N;
+    GemmPlan best{};
+    double best_cost = 0.0;
+    const int k_tiles = (int)cdiv(K, 256);
+    // Decode (M <= 128): weights take the MMA's 128-row side, the tokens its N.
+    // Otherwise activations take the 128-row side and weights come in 128- or
+    // 192-row tiles.
+    const bool swap = M <= 128;
+    int widths[2] = {0, 0};
+    if (swap)
+        widths[0] = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : 128;
+    else if (N <= 128)
+        widths[0] = 128;
+    else {
+        widths[0] = 192;
+        widths[1] = 128;
     }
-    g.tiles_p = (int)cdiv(p_rows, 128);
-    g.tiles_q = (int)cdiv(q_rows, g.bn);
-    const int64_t tiles = (int64_t)g.tiles_p * g.tiles_q;
-    // Split K when the tiles alone fill the SMs poorly. Score each split count by its
-    // wave efficiency times kps / (kps + 1) (one K tile of pipeline fill per unit), and
-    // take a larger split count only when it scores 2% better.
-    auto score = [&](int s) {
-        const int kps = (int)cdiv(g.k_tiles, s);
-        const int64_t units = tiles * cdiv(g.k_tiles, kps);
-        const double eff = (double)units / (double)(cdiv(units, num_sms) * num_sms);
-        return eff * (double)kps / (double)(kps + 1);
-    };
-    g.splits = 1;
-    if (tiles < 2 * (int64_t)num_sms && g.k_tiles > 1) {
-        double best = score(1);
-        const int max_splits = std::max(1, g.k_tiles / 2);
-        for (int s = 2; s <= max_splits; ++s) {
-            const double sc = score(s);
-            if (sc > best * 1.02) {
-                best = sc;
-                g.splits = s;
+    for (int wi = 0; wi < 2 && widths[wi] != 0; ++wi) {
+        GemmPlan g{};
+        g.swap = swap;
+        g.k_tiles = k_tiles;
+        g.bn = widths[wi];
+        g.tiles_p = (int)cdiv(swap ? N : M, 128);
+        g.tiles_q = (int)cdiv(swap ? M : N, g.bn);
+        const int64_t tiles = (int64_t)g.tiles_p * g.tiles_q;
+        // time = rounds of units over the SMs x K tiles per unit x cycles per K tile,
+        // plus the cost of splitting; K tiles per unit stay >= 2
+        const int max_splits = std::max(1, k_tiles / 2);
+        for (int s = 1; s <= max_splits; ++s) {
+            const int kps = (int)cdiv(k_tiles, s);
+            const int splits = (int)cdiv(k_tiles, kps);
+            if (splits != s) continue;
+            if (splits > 1 && M > 65535) break;        // the finalize grid has one row per block row
+            const int64_t units = tiles * splits;
+            const double cost =
+                (double)cdiv(units, num_sms) * kps * ktile_cycles(g.bn) +
+                (splits > 1 ? kSplitCycles + (double)units * 128 * g.bn * 4 / kReduceBytesPerCycle : 0.0);
+            if (best.bn == 0 || cost < best_cost * 0.98) {
+                best = g;
+                best.splits = splits;
+                best.kps = kps;
+                best_cost = cost;
             }
         }
     }
-    g.kps = (int)cdiv(g.k_tiles, g.splits);
-    g.splits = (int)cdiv(g.k_tiles, g.kps);
-    g.atomic = g.splits > 1;
-    g.group_p = std::min(g.tiles_p, 16);
-    const int64_t units = tiles * g.splits;
-    g.grid = (int)std::min<int64_t>(units, num_sms);
-    return g;
+    best.group_p = std::min(best.tiles_p, 16);
+    best.grid = (int)std::min<int64_t>((int64_t)best.tiles_p * best.tiles_q * best.splits, num_sms);
+    return best;
 }
 
 // Row stride (elements) of the fp32 split-K accumulator: a multiple of 4 so that the
 // epilogue's 16-byte vector reductions stay aligned.
 inline int64_t acc_ld(int64_t N) { return round_up(N, 4); }
 
+// Split-K workspace: the fp32 accumulator (M x acc_ld(N)), then one 8-byte flag per CTA.
+struct SplitWorkspace {
+    size_t acc_bytes, flag_bytes;
+};
+SplitWorkspace split_workspace(const GemmPlan& g, int64_t M, int64_t N) {
+    SplitWorkspace w{0, 0};
+    if (g.splits > 1) {
+        w.acc_bytes = (size_t)round_up(M * acc_ld(N) * 4, 256);
+        w.flag_bytes = (size_t)round_up((int64_t)g.grid * 8, 256);
+    }
+    return w;
+}
+
 size_t gemm_workspace(int64_t M, int64_t N, int64_t K, int num_sms) {
-    const GemmPlan g = plan_gemm(M, N, K, num_sms);
-    return g.atomic ? (size_t)round_up(M * acc_ld(N) * 4, 256) : 0;
+    const SplitWorkspace w = split_workspace(plan_gemm(M, N, K, num_sms), M, N);
+    return w.acc_bytes + w.flag_bytes;
+}
+
+// Split-K flags are set to a value unique to each call, so a flag left by an earlier
+// call (or whatever the workspace held) is never taken for a fresh one: 32 bits of a
+// per-process salt from the clock, then a call counter.
+unsigned long long next_epoch() {
+    static std::atomic<unsigned long long> counter{0};
+    static const unsigned long long salt = [] {
+        unsigned long long t = (unsigned long long)std::chrono::steady_clock::now().time_since_epoch().count();
+        t ^= t >> 33;
+        t *= 0xff51afd7ed558ccdull;
+        t ^= t >> 33;
+        return (t | 1ull) << 32;
+    }();
+    return salt + counter.fetch_add(1) + 1;
 }
 
 bool encode_codes_map(CUtensorMap* map, const uint8_t* codes, int64_t rows, int64_t K, int box_rows) {
@@ -268,19 +308,34 @@ macaq_status launch_gemm_bn(const CUtensorMap& mp, const CUtensorMap& mq, const 
                : MACAQ_ERR_CUDA;
 }
 
-__global__ void finalize_kernel(const float* __restrict__ acc, int64_t lda, int64_t M, int64_t N, void* y,
-                                int64_t ldy, int bf16) {
+// Split K: converts the fp32 accumulator (row stride lda, a multiple of 4) into y, four
+// columns per thread; blockIdx.y is the row (split-K products have few rows).
+__global__ void finalize_kernel(const float* __restrict__ acc, int64_t lda, int N, void* y, int64_t ldy, int bf16,
+                                int vec) {
     ptx::griddep_wait();
     ptx::griddep_launch_dependents();
-    const int64_t total = M * N;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
-         i += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t m = i / N, n = i - m * N;
-        const float v = acc[m * lda + n];
-        if (bf16)
-            static_cast<__nv_bfloat16*>(y)[m * ldy + n] = __float2bfloat16_rn(v);
+    const int n = (blockIdx.x * blockDim.x + threadIdx.x) * 4;
+    if (n >= N) return;
+    const int64_t m = blockIdx.y;
+    const float4 v = *reinterpret_cast<const float4*>(acc + m * lda + n);
+    const float f[4] = {v.x, v.y, v.z, v.w};
+    if (bf16) {
+        __nv_bfloat16* o = static_cast<__nv_bfloat16*>(y) + m * ldy + n;
+        if (vec && n + 4 <= N) {
+            __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y), hi = __floats2bfloat162_rn(v.z, v.w);
+            uint2 w;
+            w.x = *reinterpret_cast<uint32_t*>(&lo);
+            w.y = *reinterpret_cast<uint32_t*>(&hi);
+            *reinterpret_cast<uint2*>(o) = w;
+        } else {
+            for (int j = 0; j < 4 && n + j < N; ++j) o[j] = __float2bfloat16_rn(f[j]);
+        }
+    } else {
+        float* o = static_cast<float*>(y) + m * ldy + n;
+        if (vec && n + 4 <= N)
+            *reinterpret_cast<float4*>(o) = v;
         else
-            static_cast<float*>(y)[m * ldy + n] = v;
+            for (int j = 0; j < 4 && n + j < N; ++j) o[j] = f[j];
     }
 }
 
@@ -327,21 +382,26 @@ macaq_status run_gemm(const uint8_t* a_codes, const uint8_t* a_scales, int64_t M
     gp.group_p = g.group_p;
     gp.transpose_out = g.swap ? 1 : 0;
     gp.err = dev->err_ptr;
-    if (g.atomic) {
-        if (cudaMemsetAsync(workspace, 0, (size_t)(M * acc_ld(N) * 4), stream) != cudaSuccess)
-            return MACAQ_ERR_CUDA;
+    const int64_t esz = out == MACAQ_OUT_BF16 ? 2 : 4;
+    const int y_vec = (aligned16(y) && (ldy * esz) % 16 == 0) ? 1 : 0;
+    if (g.splits > 1) {
+        // fp32 reductions into the workspace accumulator, zeroed by the kernel itself
+        const SplitWorkspace sw = split_workspace(g, M, N);
         gp.out = workspace;
         gp.ldo = acc_ld(N);
         gp.atomic = 1;
         gp.out_bf16 = 0;
         gp.vec_ok = 1;
+        gp.tma_store = 0;
+        gp.zero_vec4 = M * acc_ld(N) * 4 / 16;
+        gp.cta_flags = reinterpret_cast<unsigned long long*>(static_cast<uint8_t*>(workspace) + sw.acc_bytes);
+        gp.epoch = next_epoch();
     } else {
-        const int64_t esz = out == MACAQ_OUT_BF16 ? 2 : 4;
         gp.out = y;
         gp.ldo = ldy;
         gp.atomic = 0;
         gp.out_bf16 = out == MACAQ_OUT_BF16 ? 1 : 0;
-        gp.vec_ok = (aligned16(y) && (ldy * esz) % 16 == 0) ? 1 : 0;
+        gp.vec_ok = y_vec;
         // wide row-major tiles store through TMA (an aligned output is all it needs)
         gp.tma_store = (!g.swap && g.bn >= 128 && gp.vec_ok) ? 1 : 0;
     }
@@ -356,14 +416,12 @@ macaq_status run_gemm(const uint8_t* a_codes, const uint8_t* a_scales, int64_t M
         case 128: st = launch_gemm_bn<128, 6>(mp, mq, my, gp, g.grid, stream); break;
         default: st = launch_gemm_bn<192, 5>(mp, mq, my, gp, g.grid, stream); break;
     }
-    if (st != MACAQ_OK) return st;
-    if (g.atomic) {
-        const int64_t total = M * N;
-        const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>(cdiv(total, 256), (int64_t)dev->num_sms * 8));
-        if (launch_pdl(finalize_kernel, dim3(blocks), dim3(256), 0, stream, static_cast<const float*>(workspace),
-                       acc_ld(N), M, N, y, ldy, out == MACAQ_OUT_BF16 ? 1 : 0) != cudaSuccess)
-            return MACAQ_ERR_CUDA;
-    }
+    if (st != MACAQ_OK || g.splits == 1) return st;
+    // split K (planned only for M <= 65535): one grid row per output row
+    const dim3 fgrid((unsigned)cdiv(cdiv(N, 4), 256), (unsigned)M);
+    if (launch_pdl(finalize_kernel, fgrid, dim3(256), 0, stream, static_cast<const float*>(workspace), acc_ld(N),
+                   (int)N, y, ldy, out == MACAQ_OUT_BF16 ? 1 : 0, y_vec) != cudaSuccess)
+        return MACAQ_ERR_CUDA;
     return MACAQ_OK;
 }
 

@@ -115,11 +115,13 @@ def test_extreme_scales(mq):
 
 
 # (M, N, K, dtype, extra columns of row padding): rows whose byte length is a multiple of
-# 16 go through the staged TMA-store epilogue (boxes clipped at ragged M and N edges),
-# others through direct stores; padding columns of a strided output stay untouched.
+# 16 go through the staged TMA-store epilogue (boxes clipped at ragged M and N edges) or
+# the finalize kernel's vector stores, others through scalar stores; padding columns of a
+# strided output stay untouched.
 OUTPUT_CASES = [
     (300, 200, 512, "bf16", 0), (300, 200, 512, "f32", 0), (257, 333, 256, "bf16", 0),
     (300, 200, 512, "bf16", 24), (300, 200, 512, "f32", 12), (640, 1000, 768, "bf16", 0),
+    (16, 256, 25600, "bf16", 8), (64, 640, 12288, "f32", 3),     # split K, finalize kernel
 ]
 
 
@@ -130,7 +132,7 @@ def test_output_paths(mq, M, N, K, dt, pad):
     a, sa = random_mxfp4(rng, M, K)
     w, sw = random_mxfp4(rng, N, K)
     y32 = host(gpu_gemm(mq, a, sa, w, sw, K, out="f32"))
-    rows = np.unique(np.concatenate([rng.choice(M, 40, replace=False), [0, M - 1]]))
+    rows = np.unique(np.concatenate([rng.choice(M, min(M, 40), replace=False), [0, M - 1]]))
     assert_gemm_close(y32[rows], oracle.gemm_fp64(a, sa, w, sw, K, rows=rows), f"f32 {M}x{N}x{K}")
     tdt = torch.bfloat16 if dt == "bf16" else torch.float32
     big = torch.full((M, N + pad), float("nan"), dtype=tdt, device="cuda")
@@ -144,4 +146,29 @@ def test_output_paths(mq, M, N, K, dt, pad):
     if dt == "bf16":
         assert_bf16_matches_f32(y, torch.from_numpy(y32).cuda(), f"bf16 {M}x{N}x{K} pad {pad}")
     else:
-        assert np.array_equal(host(y), y32), f"f32 {M}x{N}x{K} pad {pad}"
+        # not compared bit for bit with y32: split-K reductions add in no fixed order
+        assert_gemm_close(host(y)[rows], oracle.gemm_fp64(a, sa, w, sw, K, rows=rows), f"f32 {M}x{N}x{K} pad {pad}")
+
+
+@pytest.mark.parametrize("M,N,K", [(16, 256, 25600), (256, 384, 16384), (64, 640, 12288)])
+def test_split_k_workspace_reuse(mq, M, N, K):
+    """Split-K shapes (few tiles, deep K: every split adds into an fp32 accumulator the
+    kernel zeroes itself, then a small kernel writes y): two calls with different
+    activations share one workspace that starts filled with 0xFF bytes; both must match
+    the oracle."""
+    import torch
+    rng = np.random.default_rng(M + N + K)
+    need = mq.gemm_workspace_bytes(M, N, K, torch.float32)
+    assert need > 0, "shape expected to split K"
+    ws = torch.full((need,), 0xFF, dtype=torch.uint8, device="cuda")
+    w, sw = random_mxfp4(rng, N, K)
+    pw = mq.PreparedWeight(u8_dev(w), u8_dev(oracle.swizzle_scales(sw, K)),
+                           torch.ones(K, dtype=torch.float32, device="cuda"), N, K)
+    for call in range(2):
+        a, sa = random_mxfp4(rng, M, K)
+        y = mq.gemm_mxfp4(u8_dev(a), u8_dev(oracle.swizzle_scales(sa, K)), M, pw,
+                          out_dtype=torch.float32, workspace=ws)
+        torch.cuda.synchronize()
+        rows = np.arange(M) if M <= 64 else np.unique(np.concatenate([rng.choice(M, 40, replace=False), [0, M - 1]]))
+        assert_gemm_close(host(y)[rows], oracle.gemm_fp64(a, sa, w, sw, K, rows=rows), f"split K call {call}")
+    assert mq.device_error() == 0
