@@ -71,13 +71,15 @@ DEFAULT_WORKLOAD = "llama3_8b_gate_up_prefill_4096x14336x4096"
 def parse_args(argv=None):
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=2000)
+    p.add_argument("--steps", type=int, default=500)
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--workload", default=DEFAULT_WORKLOAD)
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
-    p.add_argument("--sample-rows", type=int, default=16, help="oracle sample size (rows of x)")
+    p.add_argument("--sample-rows", type=int, default=None,
+                   help="oracle sample size in rows of x (default: 128 for the CPU baseline of the GPU arm; "
+                        "for --impl reference, as many rows per step, up to 16, as keep the run within ~150 s)")
     return p.parse_args(argv)
 
 
@@ -351,7 +353,7 @@ def run_ours(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(L, x, W, s, args.sample_rows)
+        cpu = cpu_baseline(L, x, W, s, args.sample_rows or 128)
 
     result = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -425,16 +427,22 @@ def run_reference(args):
     if rank != 0:
         return None
     L = workloads_by_name()[args.workload]
-    x, W, s = wl.draw_x(L, rows=args.sample_rows), wl.draw_W(L), wl.draw_s(L)
+    x, W, s = wl.draw_x(L, rows=16), wl.draw_W(L), wl.draw_s(L)
     wc, ws, _ = oracle.prepare_weight(W, s)
-    prep_rows = max(1, int(round(L.N * args.sample_rows / L.M)))
+    rows = args.sample_rows
+    if rows is None:
+        # size each step's sample so that warm-up + timed steps stay within ~150 s
+        t1 = oracle_sample(L, x, wc, ws, W, s, 1, max(1, int(round(L.N / L.M))))
+        rows = int(max(1, min(16, 150.0 / (max(1, args.steps + args.warmup) * t1))))
+    rows = min(rows, x.shape[0])
+    prep_rows = max(1, int(round(L.N * rows / L.M)))
     for _ in range(args.warmup):
-        oracle_sample(L, x, wc, ws, W, s, args.sample_rows, prep_rows)
-    times = [oracle_sample(L, x, wc, ws, W, s, args.sample_rows, prep_rows) for _ in range(args.steps)]
+        oracle_sample(L, x, wc, ws, W, s, rows, prep_rows)
+    times = [oracle_sample(L, x, wc, ws, W, s, rows, prep_rows) for _ in range(args.steps)]
     t = sum(times) / len(times)
-    flops = 2.0 * args.sample_rows * L.N * L.K
+    flops = 2.0 * rows * L.N * L.K
     value = flops / t / 1e12
-    sample = (f"{args.sample_rows} of {L.M} rows of x per step (quantise + fp64 GEMM against all {L.N} "
+    sample = (f"{rows} of {L.M} rows of x per step (quantise + fp64 GEMM against all {L.N} "
               f"prepared weight rows) plus the matching {prep_rows}-row share of the weight preparation")
     result = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
