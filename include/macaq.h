@@ -88,8 +88,8 @@ size_t macaq_scales_bytes(int64_t rows, int64_t K);
  * tile and a flag per CTA (the kernel clears what it needs itself); 0 otherwise. */
 size_t macaq_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, macaq_out_dtype out);
 
-/* Device workspace macaq_linear_w4a4 needs: the activation codes and scales, plus
- * the GEMM workspace, each 256-byte aligned inside the block. */
+/* Device workspace macaq_linear_w4a4 needs: the activation codes and scales, per-CTA
+ * flags of the fused transform, and the GEMM workspace, each 256-byte aligned. */
 size_t macaq_linear_workspace_bytes(int64_t M, int64_t N, int64_t K, macaq_out_dtype out);
 
 /* ------------------------------------------------------------ compute --------- */
@@ -142,10 +142,16 @@ macaq_status macaq_gemm_mxfp4(const uint8_t* a_codes, const uint8_t* a_scales, i
                               const macaq_weight* w, void* y, int64_t ldy, macaq_out_dtype out,
                               void* workspace, size_t ws_bytes, macaq_stream stream);
 
-/* The whole online layer: macaq_quant_act into the workspace, then macaq_gemm_mxfp4.
- *   fused     must be 0 (a variant quantising inside the GEMM producer is not built;
- *             nonzero returns MACAQ_ERR_UNSUPPORTED)
- *   workspace device, >= macaq_linear_workspace_bytes(M, N, K, out), 256-byte aligned
+/* The whole online layer: the activation transform of macaq_quant_act into the
+ * workspace, then the GEMM of macaq_gemm_mxfp4.
+ *   fused     0: two launches (macaq_quant_act's kernel, then the GEMM).
+ *             1: for M <= 128 (decode) one launch: the GEMM kernel quantises the
+ *             activations itself (each CTA a share, while its first weight tiles load)
+ *             with the same bit-exact transform and encoding; for M > 128 as 0.
+ *             Other values return MACAQ_ERR_INVALID_ARG.
+ *   workspace device, >= macaq_linear_workspace_bytes(M, N, K, out), 256-byte aligned;
+ *             it starts with the activation codes (macaq_codes_bytes(M, K) bytes) and,
+ *             256-byte aligned after them, the scales (macaq_scales_bytes(M, K) bytes)
  * Other arguments as for macaq_quant_act / macaq_gemm_mxfp4. */
 macaq_status macaq_linear_w4a4(const void* x_bf16, int64_t M, int64_t ldx, const macaq_weight* w,
                                void* y, int64_t ldy, macaq_out_dtype out, int fused,

@@ -41,6 +41,7 @@
 #include <cuda_bf16.h>
 
 #include "ptx_sm100.cuh"
+#include "quant_kernel.cuh"
 
 namespace macaq {
 
@@ -70,6 +71,18 @@ struct GemmParams {
     int64_t zero_vec4;               // 16-byte words of the accumulator
     unsigned long long* cta_flags;   // [gridDim.x]
     unsigned long long epoch;
+    // Fused activation transform (decode, Q = activations): first thing, the epilogue
+    // warps of every CTA quantise their share of the activation blocks into the Q codes
+    // and scales (the transform and encoding of macaq_quant_act) and then set the CTA's
+    // flag as above; the producer issues the Q side of its copies only once every flag
+    // is set (the weight side of its first fills goes ahead meanwhile).
+    int32_t fused;
+    const uint16_t* fx;              // bf16 activations [f_rows x f_K], row stride fx_ld
+    int64_t fx_ld;
+    const float* f_mult;             // inv_s [f_K]
+    uint8_t* f_codes;                // [f_rows x f_K/2]
+    uint8_t* f_scales;               // atom layout, 128-row slabs x f_kb_pad blocks
+    int32_t f_rows, f_K, f_kb_pad;
 };
 
 enum : int {
@@ -325,6 +338,44 @@ __device__ __forceinline__ void tmem_load_chunk<16>(uint32_t taddr, uint32_t (&r
         : "r"(taddr));
 }
 
+// This CTA's share of the fused activation transform: one 32-element block per thread
+// and step over the 128-row slab(s) x f_kb_pad blocks of the Q operand. Blocks of real
+// rows and columns get codes and their scale byte; padding blocks get scale byte 0.
+__device__ __forceinline__ void fused_quant_share(const GemmParams& p, int et) {
+    const int kb = p.f_K >> 5;
+    const int64_t rows_pad = ((int64_t)p.f_rows + 127) / 128 * 128;
+    const int64_t total = rows_pad * p.f_kb_pad;
+    const int64_t per = (total + gridDim.x - 1) / gridDim.x;
+    const int64_t b0 = (int64_t)blockIdx.x * per, b1 = min(total, b0 + per);
+    for (int64_t i = b0 + et; i < b1; i += 128) {
+        const int row = (int)(i / p.f_kb_pad);
+        const int b = (int)(i - (int64_t)row * p.f_kb_pad);
+        uint32_t sbyte = 0;
+        if (row < p.f_rows && b < kb) {
+            const uint4* xs = reinterpret_cast<const uint4*>(p.fx + (int64_t)row * p.fx_ld + (int64_t)b * 32);
+            const float4* ms = reinterpret_cast<const float4*>(p.f_mult + (int64_t)b * 32);
+            uint64_t T[16];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const uint4 v = __ldg(xs + j);
+                const float4 m0 = __ldg(ms + 2 * j), m1 = __ldg(ms + 2 * j + 1);
+                const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+                const uint64_t mm[4] = {pk(m0.x, m0.y), pk(m0.z, m0.w), pk(m1.x, m1.y), pk(m1.z, m1.w)};
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    T[4 * j + q] = mul2(pk(__uint_as_float(w[q] << 16), __uint_as_float(w[q] & 0xFFFF0000u)), mm[q]);
+            }
+            uint32_t packed[4];
+            sbyte = encode_block(T, packed);
+            *reinterpret_cast<uint4*>(p.f_codes + (int64_t)row * (p.f_K >> 1) + (int64_t)b * 16) =
+                make_uint4(packed[0], packed[1], packed[2], packed[3]);
+        }
+        const int64_t o = ((int64_t)(row >> 7) * (p.f_kb_pad >> 2) + (b >> 2)) * 512 + (row & 31) * 16 +
+                          ((row >> 5) & 3) * 4 + (b & 3);
+        p.f_scales[o] = (uint8_t)sbyte;
+    }
+}
+
 constexpr int kSfWarpSets = 2;                                // scale-writer sets
 constexpr int kGemmThreads = 32 * (6 + 4 * kSfWarpSets);
 
@@ -389,6 +440,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         uint32_t phase = 0;
         uint32_t issued_mask = 0, issued_phase = 0;
         const int q_slabs = (p.q_rows + 127) / 128;
+        // Q side of one fill: codes tile and scale chunks
+        auto issue_q = [&](int st, int kt, int q0, int slab0, int nchunks) {
+            ptx::tma_load_2d(smem + L::kOffQ + st * S::kQTileBytes, &tmap_q, &full[st], kt * S::kBKBytes, q0);
+            for (int c = 0; c < nchunks; ++c)
+                ptx::bulk_load(smem + L::kOffSfQ + (st * S::kQChunks + c) * S::kSfChunkBytes,
+                               p.sf_q + ((int64_t)(slab0 + c) * p.kb4_pad + 2 * kt) * 512, S::kSfChunkBytes,
+                               &full[st]);
+        };
+        bool q_ready = !p.fused;
+        int deferred = 0;                   // fills of the first unit still without their Q side
         for (int u = blockIdx.x; u < p.total_units; u += gridDim.x) {
             if (cta_aborted(abort)) break;
             const Unit t = decode_unit(p, u);
@@ -403,20 +464,28 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     ptx::mbar_arrive_expect_tx(&full[stage], bytes);
                     ptx::tma_load_2d(smem + L::kOffP + stage * S::kPTileBytes, &tmap_p, &full[stage],
                                      kt * S::kBKBytes, t.tp * S::kBM);
-                    ptx::tma_load_2d(smem + L::kOffQ + stage * S::kQTileBytes, &tmap_q, &full[stage],
-                                     kt * S::kBKBytes, q0);
                     ptx::bulk_load(smem + L::kOffSfP + stage * S::kSfChunkBytes,
                                    p.sf_p + ((int64_t)t.tp * p.kb4_pad + 2 * kt) * 512,
                                    S::kSfChunkBytes, &full[stage]);
-                    for (int c = 0; c < nchunks; ++c)
-                        ptx::bulk_load(smem + L::kOffSfQ + (stage * S::kQChunks + c) * S::kSfChunkBytes,
-                                       p.sf_q + ((int64_t)(slab0 + c) * p.kb4_pad + 2 * kt) * 512,
-                                       S::kSfChunkBytes, &full[stage]);
+                    if (q_ready) issue_q(stage, kt, q0, slab0, nchunks);
                 }
                 __syncwarp();
                 issued_mask |= 1u << stage;
                 issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
                 if (++stage == STAGES) { stage = 0; phase ^= 1; }
+                if (!q_ready && (++deferred == STAGES || kt + 1 == t.kt_end)) {
+                    // every CTA's share of the quantised activations is in memory: give
+                    // the deferred fills (stages 0.. of the first unit) their Q side
+                    bool fl = true;
+                    for (int i = lane; i < (int)gridDim.x && fl; i += 32)
+                        fl = wait_split_flag(p.cta_flags + i, p.epoch, abort, p.err);
+                    if (!__all_sync(0xffffffffu, fl)) { ok = false; break; }
+                    ptx::fence_proxy_async_global();
+                    if (leader)
+                        for (int d = 0; d < deferred; ++d) issue_q(d, t.kt_begin + d, q0, slab0, nchunks);
+                    __syncwarp();
+                    q_ready = true;
+                }
             }
             if (!ok) break;
         }
@@ -562,13 +631,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const bool via_tma = S::kStagingBytes > 0 && p.tma_store;
         const uint32_t staging = ptx::smem_u32(smem + L::kOffStaging) + quad * S::kStageBoxBytes;
         bool zeroed = false;
-        if (p.atomic) {
-            // zero this CTA's slice of the split-K accumulator, then flag it
+        if (p.atomic || p.fused) {
             const int et = threadIdx.x - 64;                     // 0..127 over warps 2-5
-            const int64_t per = (p.zero_vec4 + gridDim.x - 1) / gridDim.x;
-            const int64_t b0 = (int64_t)blockIdx.x * per, b1 = min(p.zero_vec4, b0 + per);
-            float4* z = reinterpret_cast<float4*>(p.out);
-            for (int64_t i = b0 + et; i < b1; i += 128) z[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (p.atomic) {
+                // zero this CTA's slice of the split-K accumulator
+                const int64_t per = (p.zero_vec4 + gridDim.x - 1) / gridDim.x;
+                const int64_t b0 = (int64_t)blockIdx.x * per, b1 = min(p.zero_vec4, b0 + per);
+                float4* z = reinterpret_cast<float4*>(p.out);
+                for (int64_t i = b0 + et; i < b1; i += 128) z[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+            if (p.fused) fused_quant_share(p, et);
+            ptx::fence_proxy_async_global();
             __threadfence();
             asm volatile("bar.sync 1, 128;" ::: "memory");
             if (et == 0) st_release_u64(p.cta_flags + blockIdx.x, p.epoch);

@@ -347,9 +347,23 @@ macaq_status check_weight(const macaq_weight* w) {
     return MACAQ_OK;
 }
 
+// Activation transform fused into the GEMM kernel: the kernel quantises x (with w's
+// inv_s) into a_codes / a_scales itself before it loads them; `flags` holds one 8-byte
+// flag per CTA.
+struct FusedAct {
+    const void* x;
+    int64_t ldx;
+    unsigned long long* flags;
+};
+constexpr size_t kFusedFlagBytes = 8192;                 // up to 1024 CTAs
+// Largest M the fused transform takes (decode): every CTA then quantises a small share,
+// one 128-row slab of blocks in all, while the weight tiles stream in. Larger M runs the
+// transform as its own kernel, which uses every thread of the GPU for it.
+constexpr int64_t kFusedMaxRows = 128;
+
 macaq_status run_gemm(const uint8_t* a_codes, const uint8_t* a_scales, int64_t M,
                       const macaq_weight* w, void* y, int64_t ldy, macaq_out_dtype out,
-                      void* workspace, size_t ws_bytes, cudaStream_t stream) {
+                      void* workspace, size_t ws_bytes, cudaStream_t stream, const FusedAct* fa = nullptr) {
     DeviceInfo* dev = nullptr;
     macaq_status st = device_info(&dev);
     if (st != MACAQ_OK) return st;
@@ -405,16 +419,34 @@ macaq_status run_gemm(const uint8_t* a_codes, const uint8_t* a_scales, int64_t M
         // wide row-major tiles store through TMA (an aligned output is all it needs)
         gp.tma_store = (!g.swap && g.bn >= 128 && gp.vec_ok) ? 1 : 0;
     }
+    int grid = g.grid;
+    if (fa) {
+        // one CTA per SM however few tiles there are: CTAs without a unit still take
+        // their share of the activation transform
+        grid = dev->num_sms;
+        if ((size_t)grid * 8 > kFusedFlagBytes) return MACAQ_ERR_UNSUPPORTED_SHAPE;
+        gp.fused = 1;
+        gp.fx = static_cast<const uint16_t*>(fa->x);
+        gp.fx_ld = fa->ldx;
+        gp.f_mult = w->inv_s;
+        gp.f_codes = const_cast<uint8_t*>(a_codes);
+        gp.f_scales = const_cast<uint8_t*>(a_scales);
+        gp.f_rows = (int32_t)M;
+        gp.f_K = (int32_t)K;
+        gp.f_kb_pad = (int32_t)round_up(K / 32, 8);
+        gp.cta_flags = fa->flags;              // also the split-K zeroing flags
+        if (gp.epoch == 0) gp.epoch = next_epoch();
+    }
     CUtensorMap my;
     std::memset(&my, 0, sizeof(my));
     if (gp.tma_store && !encode_out_map(&my, y, M, N, ldy, out == MACAQ_OUT_BF16)) return MACAQ_ERR_CUDA;
 
     switch (g.bn) {
-        case 16: st = launch_gemm_bn<16, 8>(mp, mq, my, gp, g.grid, stream); break;
-        case 32: st = launch_gemm_bn<32, 8>(mp, mq, my, gp, g.grid, stream); break;
-        case 64: st = launch_gemm_bn<64, 8>(mp, mq, my, gp, g.grid, stream); break;
-        case 128: st = launch_gemm_bn<128, 6>(mp, mq, my, gp, g.grid, stream); break;
-        default: st = launch_gemm_bn<192, 5>(mp, mq, my, gp, g.grid, stream); break;
+        case 16: st = launch_gemm_bn<16, 8>(mp, mq, my, gp, grid, stream); break;
+        case 32: st = launch_gemm_bn<32, 8>(mp, mq, my, gp, grid, stream); break;
+        case 64: st = launch_gemm_bn<64, 8>(mp, mq, my, gp, grid, stream); break;
+        case 128: st = launch_gemm_bn<128, 6>(mp, mq, my, gp, grid, stream); break;
+        default: st = launch_gemm_bn<192, 5>(mp, mq, my, gp, grid, stream); break;
     }
     if (st != MACAQ_OK || g.splits == 1) return st;
     // split K (planned only for M <= 65535): one grid row per output row
@@ -463,19 +495,22 @@ size_t macaq_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, macaq_out_dty
     return gemm_workspace(M, N, K, sms);
 }
 
+// macaq_linear_w4a4's workspace: activation codes | scales | per-CTA flags of the fused
+// transform | the GEMM's own workspace, each 256-byte aligned.
 static size_t linear_ws_parts(int64_t M, int64_t N, int64_t K, macaq_out_dtype out, size_t* off_scales,
-                              size_t* off_gemm) {
+                              size_t* off_flags, size_t* off_gemm) {
     const size_t codes = (size_t)round_up((int64_t)macaq_codes_bytes(M, K), 256);
     const size_t scales = (size_t)round_up((int64_t)macaq_scales_bytes(M, K), 256);
     *off_scales = codes;
-    *off_gemm = codes + scales;
-    return codes + scales + macaq_gemm_workspace_bytes(M, N, K, out);
+    *off_flags = codes + scales;
+    *off_gemm = codes + scales + kFusedFlagBytes;
+    return *off_gemm + macaq_gemm_workspace_bytes(M, N, K, out);
 }
 
 size_t macaq_linear_workspace_bytes(int64_t M, int64_t N, int64_t K, macaq_out_dtype out) {
     if (M < 1 || N < 1 || K < 32) return 0;
-    size_t a, b;
-    return linear_ws_parts(M, N, K, out, &a, &b);
+    size_t a, b, c;
+    return linear_ws_parts(M, N, K, out, &a, &b, &c);
 }
 
 macaq_status macaq_prepare_weight(const void* W_bf16, int64_t N, int64_t K, int64_t ldw, const float* s,
@@ -510,17 +545,23 @@ macaq_status macaq_linear_w4a4(const void* x_bf16, int64_t M, int64_t ldx, const
                                macaq_stream stream) {
     macaq_status st = check_gemm_args(M, w, y, ldy, out);
     if (st != MACAQ_OK) return st;
-    if (fused != 0) return MACAQ_ERR_UNSUPPORTED;
+    if (fused != 0 && fused != 1) return MACAQ_ERR_INVALID_ARG;
     if (!w->inv_s) return MACAQ_ERR_INVALID_ARG;
     st = check_quant_args(x_bf16, M, w->K, ldx, w->inv_s, w->codes, w->scales);
     if (st != MACAQ_OK) return st;
-    size_t off_scales, off_gemm;
-    const size_t need = linear_ws_parts(M, w->N, w->K, out, &off_scales, &off_gemm);
+    size_t off_scales, off_flags, off_gemm;
+    const size_t need = linear_ws_parts(M, w->N, w->K, out, &off_scales, &off_flags, &off_gemm);
     if (!workspace || ws_bytes < need) return MACAQ_ERR_WORKSPACE;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255) != 0) return MACAQ_ERR_MISALIGNED;
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     uint8_t* a_codes = ws;
     uint8_t* a_scales = ws + off_scales;
+    if (fused == 1 && M <= kFusedMaxRows) {
+        // one launch: the GEMM kernel quantises the activations itself
+        const FusedAct fa{x_bf16, ldx, reinterpret_cast<unsigned long long*>(ws + off_flags)};
+        return run_gemm(a_codes, a_scales, M, w, y, ldy, out, ws + off_gemm, ws_bytes - off_gemm,
+                        (cudaStream_t)stream, &fa);
+    }
     st = launch_quant(x_bf16, M, w->K, ldx, w->inv_s, a_codes, a_scales, nullptr, nullptr, (cudaStream_t)stream);
     if (st != MACAQ_OK) return st;
     return run_gemm(a_codes, a_scales, M, w, y, ldy, out, ws + off_gemm, ws_bytes - off_gemm, (cudaStream_t)stream);

@@ -109,6 +109,63 @@ __device__ __forceinline__ uint32_t cvt_e2m1x8(uint64_t p0, uint64_t p1, uint64_
     return cvt_e2m1x8(a);
 }
 
+__device__ __forceinline__ float absmax3(float a, float b, float c) { return max3(fabsf(a), fabsf(b), fabsf(c)); }
+
+// The block transform and encoding for one block held as T[j] = elements (2j, 2j+1)
+// of u = x * mult: the butterfly, the shared exponent and the E2M1 codes (element i in nibble i % 8 of
+// packed[i / 8]). Returns the scale byte e + 127. T is overwritten.
+__device__ __forceinline__ uint32_t encode_block(uint64_t (&T)[16], uint32_t (&packed)[4]) {
+    const float c = __uint_as_float(0x3E3504F3u);        // nearest fp32 to 1/sqrt(32)
+    // butterfly stage h = 1 combines the two halves of each pair
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+        float a, d;
+        upk(T[j], a, d);
+        T[j] = pk(__fadd_rn(a, d), __fsub_rn(a, d));
+    }
+    // stages h = 2, 4, 8, 16 pair T[j] with T[j + h/2], two elements per instruction
+#pragma unroll
+    for (int hp = 1; hp < 16; hp <<= 1) {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            if (j & hp) continue;
+            const uint64_t A = T[j], B = T[j + hp];
+            T[j] = add2(A, B);
+            T[j + hp] = sub2(A, B);
+        }
+    }
+
+    // max |t| as a three-level tree (the order of a max does not change its value)
+    float a[32];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) upk(T[j], a[2 * j], a[2 * j + 1]);
+    float m[11];
+#pragma unroll
+    for (int i = 0; i < 10; ++i) m[i] = absmax3(a[3 * i], a[3 * i + 1], a[3 * i + 2]);
+    m[10] = fmaxf(fabsf(a[30]), fabsf(a[31]));
+    const float tmax = max3(max3(m[0], m[1], m[2]), max3(m[3], m[4], m[5]),
+                            max3(max3(m[6], m[7], m[8]), m[9], m[10]));
+    const float amax = __fmul_rn(tmax, c);
+    const int biased = (int)(__float_as_uint(amax) >> 23);
+    const int e = max(biased - 129, -127);        // biased == 0 (zero / subnormal) -> -127
+    if (e >= -123 && e <= 123) {
+        const float k = __uint_as_float(0x3E3504F3u - ((uint32_t)e << 23));   // c * 2^-e
+        const uint64_t kk = pk(k, k);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            packed[i] = cvt_e2m1x8(mul2(T[4 * i], kk), mul2(T[4 * i + 1], kk), mul2(T[4 * i + 2], kk),
+                                   mul2(T[4 * i + 3], kk));
+    } else {
+        const float inv = __uint_as_float((uint32_t)(127 - e) << 23);      // 2^-e
+        const uint64_t cc = pk(c, c), ii = pk(inv, inv);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            packed[i] = cvt_e2m1x8(mul2(mul2(T[4 * i], cc), ii), mul2(mul2(T[4 * i + 1], cc), ii),
+                                   mul2(mul2(T[4 * i + 2], cc), ii), mul2(mul2(T[4 * i + 3], cc), ii));
+    }
+    return (uint32_t)(e + 127);
+}
+
 constexpr int kQuantThreads = 256;
 constexpr int kQuantStages = 4;
 constexpr uint32_t kQuantStageBytes = kQuantThreads * 64;
@@ -122,8 +179,6 @@ __device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src, uint3
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
-
-__device__ __forceinline__ float absmax3(float a, float b, float c) { return max3(fabsf(a), fabsf(b), fabsf(c)); }
 
 __global__ void __launch_bounds__(kQuantThreads, 2) quant_rows_kernel(QuantParams p) {
     extern __shared__ __align__(16) uint8_t qsmem[];
@@ -139,7 +194,6 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_rows_kernel(QuantParam
     const int rows = (int)p.rows, rows_pad = (int)p.rows_pad;
     const int b = chunk * 32 + lane;                     // block index in the row
     const bool col_live = b < (int)(p.K >> 5);
-    const float c = __uint_as_float(0x3E3504F3u);        // nearest fp32 to 1/sqrt(32)
 
     // Copy pipeline. Rows past the end and blocks past K are zero-filled instead of
     // branched around: they give zero blocks, whose scale byte 0 is exactly what the
@@ -225,56 +279,8 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_rows_kernel(QuantParam
         rslot += kQuantStageBytes;
         if (rslot == slot_end) rslot = slot0;
 
-        // butterfly stage h = 1 combines the two halves of each pair
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-            float a, d;
-            upk(T[j], a, d);
-            T[j] = pk(__fadd_rn(a, d), __fsub_rn(a, d));
-        }
-        // stages h = 2, 4, 8, 16 pair T[j] with T[j + h/2], two elements per instruction
-#pragma unroll
-        for (int hp = 1; hp < 16; hp <<= 1) {
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                if (j & hp) continue;
-                const uint64_t A = T[j], B = T[j + hp];
-                T[j] = add2(A, B);
-                T[j + hp] = sub2(A, B);
-            }
-        }
-
-        // max |t| as a three-level tree (the order of a max does not change its value)
-        float a[32];
-#pragma unroll
-        for (int j = 0; j < 16; ++j) upk(T[j], a[2 * j], a[2 * j + 1]);
-        float m[11];
-#pragma unroll
-        for (int i = 0; i < 10; ++i) m[i] = absmax3(a[3 * i], a[3 * i + 1], a[3 * i + 2]);
-        m[10] = fmaxf(fabsf(a[30]), fabsf(a[31]));
-        const float tmax = max3(max3(m[0], m[1], m[2]), max3(m[3], m[4], m[5]),
-                                max3(max3(m[6], m[7], m[8]), m[9], m[10]));
-        const float amax = __fmul_rn(tmax, c);
-        const int biased = (int)(__float_as_uint(amax) >> 23);
-        const int e = max(biased - 129, -127);        // biased == 0 (zero / subnormal) -> -127
-        const uint32_t sbyte = (uint32_t)(e + 127);
-
         uint32_t packed[4];
-        if (e >= -123 && e <= 123) {
-            const float k = __uint_as_float(0x3E3504F3u - ((uint32_t)e << 23));   // c * 2^-e
-            const uint64_t kk = pk(k, k);
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-                packed[i] = cvt_e2m1x8(mul2(T[4 * i], kk), mul2(T[4 * i + 1], kk), mul2(T[4 * i + 2], kk),
-                                       mul2(T[4 * i + 3], kk));
-        } else {
-            const float inv = __uint_as_float((uint32_t)(127 - e) << 23);      // 2^-e
-            const uint64_t cc = pk(c, c), ii = pk(inv, inv);
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-                packed[i] = cvt_e2m1x8(mul2(mul2(T[4 * i], cc), ii), mul2(mul2(T[4 * i + 1], cc), ii),
-                                       mul2(mul2(T[4 * i + 2], cc), ii), mul2(mul2(T[4 * i + 3], cc), ii));
-        }
+        const uint32_t sbyte = encode_block(T, packed);
 
         if (col_live && row < rows)
             *reinterpret_cast<uint4*>(cdst) = make_uint4(packed[0], packed[1], packed[2], packed[3]);

@@ -130,3 +130,34 @@ def test_strided_activations(mq):
 
 def test_device_error_word_is_clear(mq):
     assert mq.device_error() == 0
+
+
+# (M, N, K): decode shapes for the fused transform (one launch), a split-K shape (the
+# kernel also zeroes its accumulator), and a K whose block count needs scale padding.
+FUSED_CASES = [(1, 25600, 5120), (16, 25600, 5120), (64, 4096, 5120), (128, 1024, 768),
+               (16, 256, 25600), (7, 300, 800)]
+
+
+@pytest.mark.parametrize("M,N,K", FUSED_CASES)
+def test_fused_transform(mq, M, N, K):
+    """macaq_linear_w4a4 with fused = 1: the activation codes and scales the GEMM kernel
+    leaves in the workspace are bit-exact against the oracle, and y is within the GEMM
+    tolerance; a second call on the same workspace gives the same."""
+    import torch
+    L = wl.with_shape(wl.tiny_layer(), M=M, N=N, K=K)
+    W, s = wl.draw_W(L), wl.draw_s(L)
+    pw = mq.prepare_weight(bf16_dev(W), f32_dev(s))
+    rwc, rws, rinv = oracle.prepare_weight(W, s)
+    need = mq.linear_workspace_bytes(M, N, K, torch.float32)
+    ws = torch.full((need,), 0xFF, dtype=torch.uint8, device="cuda")
+    cb = mq.codes_bytes(M, K)
+    off_scales = (cb + 255) // 256 * 256
+    for seed in (21, 22):
+        x = wl.draw_x(wl.with_shape(L, seed=seed))
+        y = mq.linear(bf16_dev(x), pw, out_dtype=torch.float32, workspace=ws, fused=True)
+        torch.cuda.synchronize()
+        rac, ras = oracle.quant_rows(x, rinv)
+        assert_codes_equal(host(ws[:cb]).reshape(M, K // 2), rac, f"fused codes {M}x{K}")
+        assert_scales_equal(host(ws[off_scales:off_scales + mq.scales_bytes(M, K)]), ras, K, f"fused scales {M}x{K}")
+        assert_gemm_close(host(y), oracle.gemm_fp64(rac, ras, rwc, rws, K), f"fused {M}x{N}x{K} seed {seed}")
+    assert mq.device_error() == 0
