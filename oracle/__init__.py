@@ -60,6 +60,18 @@ def lib():
         L.oracle_dequant_rows.restype = None
         L.oracle_transform_rows_f64.argtypes = [P, I64, I64, P, ctypes.c_double, P]
         L.oracle_transform_rows_f64.restype = None
+        L.oracle_transform_block_f32.argtypes = [P, P, I64, P]
+        L.oracle_transform_block_f32.restype = None
+        L.oracle_hessian_blocks.argtypes = [P, I64, I64, I64, P, P]
+        L.oracle_hessian_blocks.restype = None
+        L.oracle_block_error.argtypes = [P, P]
+        L.oracle_block_error.restype = ctypes.c_double
+        L.oracle_block_error_at.argtypes = [P, ctypes.c_int, P, P]
+        L.oracle_block_error_at.restype = ctypes.c_double
+        L.oracle_search_block.argtypes = [P, P, P, P]
+        L.oracle_search_block.restype = None
+        L.oracle_prepare_weight_hessian.argtypes = [P, I64, I64, I64, P, P, P, P, P]
+        L.oracle_prepare_weight_hessian.restype = None
         _lib = L
     return _lib
 
@@ -131,6 +143,63 @@ def prepare_weight(W_bf16, s):
     scales = np.empty((N, K // 32), np.uint8)
     inv_s = np.empty(K, np.float32)
     lib().oracle_prepare_weight(_p(W), N, K, K, _p(s), _p(codes), _p(scales), _p(inv_s))
+    return codes, scales, inv_s
+
+
+def transform_block(x_row_bf16, mult, b):
+    """The fp32 transformed block b of one row (fwht32 of x * mult)."""
+    x = _c(x_row_bf16, np.uint16)
+    m = _c(mult, np.float32)
+    v = np.empty(32, np.float32)
+    lib().oracle_transform_block_f32(_p(x), _p(m), int(b), _p(v))
+    return v
+
+
+def hessian_blocks(x_bf16, inv_s):
+    """x_bf16: uint16 [T, K]; returns H float64 [K/32, 32, 32]."""
+    x = _c(x_bf16, np.uint16)
+    m = _c(inv_s, np.float32)
+    T, K = x.shape
+    H = np.empty((K // 32, 32, 32), np.float64)
+    lib().oracle_hessian_blocks(_p(x), T, K, K, _p(m), _p(H))
+    return H
+
+
+def block_error(d, H):
+    dd = _c(d, np.float64)
+    Hh = _c(H, np.float64)
+    return lib().oracle_block_error(_p(dd), _p(Hh))
+
+
+def block_error_at(v, e, H):
+    vv = _c(v, np.float32)
+    Hh = _c(H, np.float64)
+    codes = np.empty(16, np.uint8)
+    err = lib().oracle_block_error_at(_p(vv), int(e), _p(Hh), _p(codes))
+    return err, codes
+
+
+def search_block(v, H):
+    """Returns (codes uint8 [16], scale byte)."""
+    vv = _c(v, np.float32)
+    Hh = _c(H, np.float64)
+    codes = np.empty(16, np.uint8)
+    sc = np.empty(1, np.uint8)
+    lib().oracle_search_block(_p(vv), _p(Hh), _p(codes), _p(sc))
+    return codes, int(sc[0])
+
+
+def prepare_weight_hessian(W_bf16, s, H):
+    """Returns (codes [N, K/2], scales [N, K/32] row-major, inv_s float32 [K])."""
+    W = _c(W_bf16, np.uint16)
+    s = _c(s, np.float32)
+    N, K = W.shape
+    Hh = _c(H, np.float64)
+    assert Hh.shape == (K // 32, 32, 32)
+    codes = np.empty((N, K // 2), np.uint8)
+    scales = np.empty((N, K // 32), np.uint8)
+    inv_s = np.empty(K, np.float32)
+    lib().oracle_prepare_weight_hessian(_p(W), N, K, K, _p(s), _p(Hh), _p(codes), _p(scales), _p(inv_s))
     return codes, scales, inv_s
 
 

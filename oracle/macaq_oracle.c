@@ -177,9 +177,14 @@ void oracle_quant_rows(const uint16_t* x, int64_t rows, int64_t K, int64_t ld,
     }
 }
 
+/* inv_s = RN32(1 / s), one IEEE fp32 division per channel. */
+static void inverse_scales(const float* s, int64_t K, float* inv_s) {
+    for (int64_t k = 0; k < K; ++k) inv_s[k] = 1.0f / s[k];
+}
+
 void oracle_prepare_weight(const uint16_t* W, int64_t N, int64_t K, int64_t ld,
                            const float* s, uint8_t* codes, uint8_t* scales, float* inv_s) {
-    for (int64_t k = 0; k < K; ++k) inv_s[k] = 1.0f / s[k];
+    inverse_scales(s, K, inv_s);
     oracle_quant_rows(W, N, K, ld, s, codes, scales);
 }
 
@@ -272,6 +277,93 @@ void oracle_transform_rows_f64(const double* x, int64_t rows, int64_t K, const d
                 }
                 out[r * K + 32 * b + j] = acc / norm;
             }
+        }
+    }
+}
+
+/* ----------------------------------------- Hessian exponent search ---------- */
+
+void oracle_transform_block_f32(const uint16_t* x_row, const float* mult, int64_t b, float v[32]) {
+    for (int i = 0; i < 32; ++i) {
+        int64_t k = 32 * b + i;
+        v[i] = oracle_bf16_to_f32(x_row[k]) * mult[k];
+    }
+    oracle_fwht32_f32(v);
+}
+
+void oracle_hessian_blocks(const uint16_t* x, int64_t T, int64_t K, int64_t ld, const float* inv_s,
+                           double* H) {
+    int64_t Kb = K / 32;
+    memset(H, 0, (size_t)(Kb * 32 * 32) * sizeof(double));
+    for (int64_t t = 0; t < T; ++t) {
+        for (int64_t b = 0; b < Kb; ++b) {
+            float v[32];
+            oracle_transform_block_f32(x + t * ld, inv_s, b, v);
+            double* Hb = H + b * 32 * 32;
+            for (int i = 0; i < 32; ++i)
+                for (int j = 0; j < 32; ++j) Hb[i * 32 + j] += (double)v[i] * (double)v[j];
+        }
+    }
+}
+
+double oracle_block_error(const double d[32], const double H[32 * 32]) {
+    double err = 0.0;
+    for (int i = 0; i < 32; ++i) {
+        double r = 0.0;
+        for (int j = 0; j < 32; ++j) r += H[i * 32 + j] * d[j];
+        err += d[i] * r;
+    }
+    return err;
+}
+
+double oracle_block_error_at(const float v[32], int e, const double H[32 * 32], uint8_t codes16[16]) {
+    float inv = ldexpf(1.0f, -e);
+    double d[32];
+    for (int j = 0; j < 16; ++j) {
+        uint8_t lo = oracle_e2m1_encode(v[2 * j] * inv);
+        uint8_t hi = oracle_e2m1_encode(v[2 * j + 1] * inv);
+        codes16[j] = (uint8_t)((hi << 4) | lo);             /* element 2j in the low nibble */
+        d[2 * j] = (double)v[2 * j] - ldexp(oracle_e2m1_decode(lo), e);
+        d[2 * j + 1] = (double)v[2 * j + 1] - ldexp(oracle_e2m1_decode(hi), e);
+    }
+    return oracle_block_error(d, H);
+}
+
+void oracle_search_block(const float v[32], const double H[32 * 32], uint8_t codes16[16], uint8_t* scale) {
+    float amax = 0.0f;
+    for (int i = 0; i < 32; ++i) {
+        float a = fabsf(v[i]);
+        if (a > amax) amax = a;
+    }
+    int e0 = oracle_e8m0_exponent(amax);
+    int cand[3] = {e0, e0 + 1, e0 - 1};
+    int best_e = e0;
+    double best = 0.0;
+    int have = 0;
+    for (int c = 0; c < 3; ++c) {
+        int e = cand[c];
+        if (e < -127 || e > 127) continue;
+        uint8_t tmp[16];
+        double err = oracle_block_error_at(v, e, H, tmp);
+        if (!have || err < best) {
+            best = err;
+            best_e = e;
+            memcpy(codes16, tmp, 16);
+            have = 1;
+        }
+    }
+    *scale = (uint8_t)(best_e + 127);
+}
+
+void oracle_prepare_weight_hessian(const uint16_t* W, int64_t N, int64_t K, int64_t ld, const float* s,
+                                   const double* H, uint8_t* codes, uint8_t* scales, float* inv_s) {
+    int64_t Kb = K / 32;
+    inverse_scales(s, K, inv_s);
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t b = 0; b < Kb; ++b) {
+            float v[32];
+            oracle_transform_block_f32(W + n * ld, s, b, v);
+            oracle_search_block(v, H + b * 32 * 32, codes + n * (K / 2) + 16 * b, scales + n * Kb + b);
         }
     }
 }

@@ -105,6 +105,45 @@ void oracle_dequant_rows(const uint8_t* codes, const uint8_t* scales, int64_t ro
 void oracle_transform_rows_f64(const double* x, int64_t rows, int64_t K, const double* mult,
                                double norm, double* out);
 
+/* ------------------------------------------------------------------------------
+ * Hessian exponent search for weight blocks (the "Hessian exponent search" step of the
+ * ablation paragraph of the openai-hub.com article, between round-to-nearest and the
+ * micro-rotation; its error model is the second-order form
+ *   dL ~ 1/2 (w - w_hat)^T H (w - w_hat)
+ * of the Flip-Refinement paragraph of the zicq.com articles). Reading taken: H is the
+ * Gram matrix X'^T X' of calibration activations in the transformed basis (the fp32
+ * values oracle_quant_rows quantises), restricted to its 32 x 32 diagonal blocks, and
+ * each weight block keeps the exponent, among e0 (the floor rule), e0 + 1 and e0 - 1,
+ * with the smallest d^T H_b d, d = w' - dec(codes) 2^e.
+ * ---------------------------------------------------------------------------- */
+
+/* The transformed block v (32 fp32 values) of row r, block b: fwht32 of x * mult. */
+void oracle_transform_block_f32(const uint16_t* x_row, const float* mult, int64_t b, float v[32]);
+
+/* H[b][i][j] = sum_t v_t[i] v_t[j] over the calibration rows t = 0 .. T-1 (ascending),
+ * v_t the transformed block b of row t under multiplier inv_s. fp64: each product of
+ * two fp32 values is exact, so only the running sum rounds. H: [K/32][32][32]. */
+void oracle_hessian_blocks(const uint16_t* x, int64_t T, int64_t K, int64_t ld, const float* inv_s,
+                           double* H);
+
+/* d^T H d for one block, fp64: sum over i ascending of d[i] * r[i], where
+ * r[i] = sum over j ascending of H[i][j] * d[j]; every product and sum rounded on its own. */
+double oracle_block_error(const double d[32], const double H[32 * 32]);
+
+/* Encode v under exponent e (codes of v * 2^-e, as the floor-rule path encodes) and
+ * return d^T H d with d = v - dec(codes) * 2^e (exact in fp64). */
+double oracle_block_error_at(const float v[32], int e, const double H[32 * 32], uint8_t codes16[16]);
+
+/* One block of the search: candidates e0, e0 + 1, e0 - 1 (those within [-127, 127]), in
+ * that order; a candidate replaces the current choice only with a strictly smaller
+ * error. Writes the 16 code bytes and the scale byte e + 127. */
+void oracle_search_block(const float v[32], const double H[32 * 32], uint8_t codes16[16], uint8_t* scale);
+
+/* Weight preparation with the exponent search: as oracle_prepare_weight, with every
+ * block of every row chosen by oracle_search_block under H[b]. */
+void oracle_prepare_weight_hessian(const uint16_t* W, int64_t N, int64_t K, int64_t ld, const float* s,
+                                   const double* H, uint8_t* codes, uint8_t* scales, float* inv_s);
+
 #ifdef __cplusplus
 }
 #endif

@@ -325,4 +325,152 @@ def pin_storage():
     assert bits == golden_storage_bits()
 
 
+# ------------------------------------------------ Hessian exponent search -----
+
+def _np_block_codes(v, e):
+    """Codes of v * 2^-e by the brute-force encoder, and their values dec * 2^e."""
+    q = (v.astype(np.float64) * 2.0 ** (-e)).astype(np.float32)
+    codes = np.array([bf_e2m1_encode(qq) for qq in q], np.uint8)
+    table = golden_e2m1()
+    vals = np.array([(-1.0 if c & 8 else 1.0) * table[c & 7] for c in codes]) * 2.0 ** e
+    return codes, vals
+
+
+def _np_search(v, H):
+    """Independent restatement of the search: errors in fp64 by numpy, candidates in the
+    order e0, e0 + 1, e0 - 1, a later one kept only when strictly better."""
+    e0 = bf_e8m0(float(np.abs(v).max()))
+    best = None
+    for e in (e0, e0 + 1, e0 - 1):
+        if not -127 <= e <= 127:
+            continue
+        codes, vals = _np_block_codes(v, e)
+        d = v.astype(np.float64) - vals
+        err = float(d @ H @ d)
+        if best is None or err < best[0] * (1 - 1e-12) - 1e-300:
+            best = (err, e, codes)
+    return best
+
+
+def _random_psd(rng, n=32):
+    A = rng.standard_normal((n, 2 * n))
+    return A @ A.T / (2 * n)
+
+
+def pin_transform_block():
+    rng = np.random.default_rng(20)
+    xi, xb, mult = _exact_rows(rng, 3, 96)
+    for r in range(3):
+        for b in range(3):
+            t = H32 @ (xi[r, 32 * b:32 * b + 32].astype(np.float64) * mult[32 * b:32 * b + 32])   # exact
+            v = (np.float32(t) * C32).astype(np.float32)
+            assert np.array_equal(oracle.transform_block(xb[r], mult, b), v), (r, b)
+
+
+def pin_hessian_blocks():
+    rng = np.random.default_rng(21)
+    T, K = 12, 128
+    x = rng.standard_t(3, size=(T, K)).astype(np.float32)
+    x[:, 9] *= 30
+    xb = (x.view(np.uint32) >> 16).astype(np.uint16)
+    inv_s = (np.float32(1.0) / np.exp(rng.normal(0, 0.5, K)).astype(np.float32)).astype(np.float32)
+    H = oracle.hessian_blocks(xb, inv_s)
+    for b in range(K // 32):
+        V = np.stack([oracle.transform_block(xb[t], inv_s, b) for t in range(T)]).astype(np.float64)
+        ref = V.T @ V                                  # library matmul
+        assert np.allclose(H[b], ref, rtol=1e-13, atol=1e-300), b
+        assert np.array_equal(H[b], H[b].T), b          # same products both ways
+    # small integers: every sum is exact
+    xi, xb2, mult = _exact_rows(rng, 5, 64)
+    H2 = oracle.hessian_blocks(xb2, mult)
+    for b in range(2):
+        V = np.stack([oracle.transform_block(xb2[t], mult, b) for t in range(5)]).astype(np.float64)
+        assert np.array_equal(H2[b], V.T @ V), b
+
+
+def pin_block_error():
+    rng = np.random.default_rng(22)
+    d = rng.integers(-9, 10, 32).astype(np.float64)
+    A = rng.integers(-5, 6, (32, 32))
+    H = (A + A.T).astype(np.float64)
+    assert oracle.block_error(d, H) == float(d @ H @ d)            # integers: exact
+    d = rng.standard_normal(32)
+    H = _random_psd(rng)
+    assert math.isclose(oracle.block_error(d, H), float(d @ H @ d), rel_tol=1e-12)
+
+
+def pin_block_error_at():
+    rng = np.random.default_rng(23)
+    for trial in range(20):
+        v = (rng.standard_t(3, 32) * 2.0 ** rng.integers(-6, 7)).astype(np.float32)
+        H = _random_psd(rng)
+        e0 = bf_e8m0(float(np.abs(v).max()))
+        for e in (e0 - 1, e0, e0 + 1):
+            err, codes = oracle.block_error_at(v, e, H)
+            ref_codes, vals = _np_block_codes(v, e)
+            assert np.array_equal(codes, pack_nibbles(ref_codes[None, :])[0]), (trial, e)
+            d = v.astype(np.float64) - vals
+            assert math.isclose(err, float(d @ H @ d), rel_tol=1e-11, abs_tol=1e-300), (trial, e)
+
+
+def pin_search_block():
+    rng = np.random.default_rng(24)
+    picked = {0: 0, 1: 0, -1: 0}
+    for trial in range(300):
+        v = (rng.standard_t(3, 32) * 2.0 ** rng.integers(-8, 8)).astype(np.float32)
+        if trial % 3 == 0:
+            v[rng.integers(32)] *= 12                  # an outlier
+        H = np.eye(32) if trial % 2 == 0 else _random_psd(rng)
+        codes, scale = oracle.search_block(v, H)
+        e0 = bf_e8m0(float(np.abs(v).max()))
+        err_ref, e_ref, codes_ref = _np_search(v, H)
+        assert scale == e_ref + 127, (trial, scale - 127, e_ref)
+        assert np.array_equal(codes, pack_nibbles(codes_ref[None, :])[0]), trial
+        err_e0 = _np_search(v, np.zeros((32, 32)))[0]
+        picked[e_ref - e0] += 1
+        # never worse than the floor rule under the same H
+        _, vals0 = _np_block_codes(v, e0)
+        d0 = v.astype(np.float64) - vals0
+        assert err_ref <= float(d0 @ H @ d0) * (1 + 1e-12), trial
+        assert err_e0 == 0.0
+    assert picked[0] > 0 and picked[1] > 0, picked
+    # H = 0: every candidate ties, the floor rule stays
+    v = (rng.standard_normal(32) * 5).astype(np.float32)
+    codes, scale = oracle.search_block(v, np.zeros((32, 32)))
+    assert scale == bf_e8m0(float(np.abs(v).max())) + 127
+    # planted: an outlier whose coordinate H ignores makes e0 - 1 the best choice (it
+    # clips the outlier at no cost and halves the step for the rest)
+    v = np.full(32, 0.37, np.float32) * np.where(np.arange(32) % 2 == 0, 1, -1).astype(np.float32)
+    v[0] = np.float32(7.9)
+    Hd = np.eye(32)
+    Hd[0, 0] = 0.0
+    codes, scale = oracle.search_block(v, Hd)
+    assert scale - 127 == bf_e8m0(7.9) - 1, scale - 127
+    # planted: values just under 8 * 2^e0 saturate to 6 at e0; e0 + 1 is better under H = I
+    v = np.full(32, 7.75, np.float32)
+    codes, scale = oracle.search_block(v, np.eye(32))
+    assert scale - 127 == bf_e8m0(7.75) + 1, scale - 127
+
+
+def pin_prepare_weight_hessian():
+    rng = np.random.default_rng(25)
+    N, K = 7, 96
+    W = rng.normal(0, 0.02, (N, K)).astype(np.float32)
+    Wb = (W.view(np.uint32) >> 16).astype(np.uint16)
+    s = np.exp(rng.normal(0, 0.5, K)).astype(np.float32)
+    # H = 0: the floor rule everywhere, i.e. plain prepare_weight
+    c0, s0, inv0 = oracle.prepare_weight_hessian(Wb, s, np.zeros((K // 32, 32, 32)))
+    c1, s1, inv1 = oracle.prepare_weight(Wb, s)
+    assert np.array_equal(c0, c1) and np.array_equal(s0, s1) and np.array_equal(inv0, inv1)
+    # general H: every block is the numpy search of its transformed block
+    H = np.stack([_random_psd(rng) for _ in range(K // 32)])
+    c2, s2, _ = oracle.prepare_weight_hessian(Wb, s, H)
+    for n in range(N):
+        for b in range(K // 32):
+            v = oracle.transform_block(Wb[n], s, b)
+            _, e, codes = _np_search(v, H[b])
+            assert s2[n, b] == e + 127, (n, b)
+            assert np.array_equal(c2[n, 16 * b:16 * b + 16], pack_nibbles(codes[None, :])[0]), (n, b)
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

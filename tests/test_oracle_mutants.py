@@ -39,6 +39,15 @@ MUTANTS = [
     ("decode_exponent_bias", "ldexp(1.0 + 0.5 * m, ex - 1)", "ldexp(1.0 + 0.5 * m, ex)"),
     ("transform_f64_index", "acc += x[r * K + k] * mult[k] * (double)oracle_hadamard_entry(i, j);",
      "acc += x[r * K + k] * mult[k] * (double)oracle_hadamard_entry(j, i & 15);"),
+    ("hessian_diagonal_only", "for (int j = 0; j < 32; ++j) Hb[i * 32 + j] += (double)v[i] * (double)v[j];",
+     "Hb[i * 32 + i] += (double)v[i] * (double)v[i];"),
+    ("block_error_index", "for (int j = 0; j < 32; ++j) r += H[i * 32 + j] * d[j];",
+     "for (int j = 0; j < 32; ++j) r += H[i * 32 + j] * d[i];"),
+    ("error_at_exponent_sign", "d[2 * j] = (double)v[2 * j] - ldexp(oracle_e2m1_decode(lo), e);",
+     "d[2 * j] = (double)v[2 * j] - ldexp(oracle_e2m1_decode(lo), -e);"),
+    ("search_nibble_order", "codes16[j] = (uint8_t)((hi << 4) | lo);", "codes16[j] = (uint8_t)((lo << 4) | hi);"),
+    ("search_ties_replace", "if (!have || err < best) {", "if (!have || err <= best) {"),
+    ("search_no_lower_candidate", "int cand[3] = {e0, e0 + 1, e0 - 1};", "int cand[3] = {e0, e0 + 1, e0 + 1};"),
 ]
 
 
