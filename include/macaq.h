@@ -157,6 +157,44 @@ macaq_status macaq_linear_w4a4(const void* x_bf16, int64_t M, int64_t ldx, const
                                void* y, int64_t ldy, macaq_out_dtype out, int fused,
                                void* workspace, size_t ws_bytes, macaq_stream stream);
 
+/* ------------------------------------------ Hessian exponent search (offline) --- */
+
+/* The "Hessian exponent search" step of the ablation paragraph of the openai-hub.com
+ * article, with the second-order error model dL ~ 1/2 (w - w_hat)^T H (w - w_hat) of the
+ * Flip-Refinement paragraphs of the zicq.com articles. H is taken as the Gram matrix
+ * of calibration activations in the transformed basis, restricted to its 32 x 32
+ * diagonal blocks; each weight block keeps, of the exponents e0 (the floor rule), e0 + 1
+ * and e0 - 1, the one with the smallest d^T H_b d. Only the weight bytes change: the
+ * result feeds macaq_gemm_mxfp4 / macaq_linear_w4a4 like macaq_prepare_weight's. */
+
+/* Bytes of the H block array for K: (K/32) * 32 * 32 doubles (0 if K % 32 != 0). */
+size_t macaq_hessian_bytes(int64_t K);
+
+/* H[b][i][j] = sum over t = 0 .. T-1 (in that order) of v_t[32b+i] * v_t[32b+j], fp64,
+ * where v_t is calibration row t after the online transform of macaq_quant_act with
+ * inv_s = RN32(1/s) (the fp32 values before quantisation). Each product of two fp32
+ * values is exact in fp64, so only the running sum rounds: the result is bit-identical
+ * to that sequential definition.
+ *   x_bf16  device bf16 [T x K], row stride ldx (ldx >= K, ldx % 8 == 0), 16-byte aligned
+ *   s       device fp32 [K], 16-byte aligned
+ *   H       device fp64, macaq_hessian_bytes(K), 16-byte aligned, row-major [K/32][32][32]
+ * T >= 1, K % 32 == 0. */
+macaq_status macaq_hessian_blocks(const void* x_bf16, int64_t T, int64_t K, int64_t ldx, const float* s, double* H,
+                                  macaq_stream stream);
+
+/* macaq_prepare_weight with the exponent search: for every 32-block of every row of
+ * W' = W diag(s) Hb, candidates e0, e0 + 1, e0 - 1 (within [-127, 127]); for each, the
+ * round-to-nearest codes of fp32(v * 2^-e) and d = v - dec(codes) 2^e (exact in fp64);
+ * error = sum_i d_i * (sum_j H_b[i][j] * d_j), i and j ascending, every fp64 product and
+ * sum rounded on its own; a later candidate replaces the choice only when its error is
+ * strictly smaller. Codes, scales (same layout and padding as macaq_prepare_weight) and
+ * inv_s are written; bit-identical to that definition.
+ *   H       device fp64 [K/32][32][32] (from macaq_hessian_blocks or the caller)
+ * Other arguments as for macaq_prepare_weight. */
+macaq_status macaq_prepare_weight_hessian(const void* W_bf16, int64_t N, int64_t K, int64_t ldw, const float* s,
+                                          const double* H, uint8_t* w_codes, uint8_t* w_scales, float* inv_s_out,
+                                          macaq_stream stream);
+
 /* Largest scratch the no-allocation variant below can use: 16 MiB, held in a static
  * device array on every GPU that loads this library, for as long as it stays loaded. */
 #define MACAQ_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)

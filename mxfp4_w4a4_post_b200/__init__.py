@@ -57,6 +57,9 @@ def lib():
             "macaq_quant_act": (I, [P, I64, I64, I64, P, P, P, P]),
             "macaq_gemm_mxfp4": (I, [P, P, I64, ctypes.POINTER(MacaqWeight), P, I64, I, P, SZ, P]),
             "macaq_linear_w4a4": (I, [P, I64, I64, ctypes.POINTER(MacaqWeight), P, I64, I, I, P, SZ, P]),
+            "macaq_hessian_bytes": (SZ, [I64]),
+            "macaq_hessian_blocks": (I, [P, I64, I64, I64, P, P, P]),
+            "macaq_prepare_weight_hessian": (I, [P, I64, I64, I64, P, P, P, P, P, P]),
             "macaq_get_device_error": (I, []),
             "macaq_status_string": (ctypes.c_char_p, [I]),
             "macaq_version": (I, []),
@@ -149,6 +152,42 @@ def prepare_weight(W, s, out=None):
     st = lib().macaq_prepare_weight(W.data_ptr(), N, K, W.stride(0), s.data_ptr(), out.codes.data_ptr(),
                                     out.scales.data_ptr(), out.inv_s.data_ptr(), _stream_ptr(dev))
     _check(st, "macaq_prepare_weight")
+    return out
+
+
+def hessian_blocks(x, s, H=None):
+    """Calibration activations x: bf16 [T, K]; s: fp32 [K]. Returns the fp64 Gram blocks
+    H [K/32, 32, 32] of the transformed rows (the input of prepare_weight_hessian)."""
+    torch = _torch()
+    _require(x, torch.bfloat16, "x")
+    _require(s, torch.float32, "s")
+    T, K = x.shape
+    if H is None:
+        H = torch.empty((K // 32, 32, 32), dtype=torch.float64, device=x.device)
+    st = lib().macaq_hessian_blocks(x.data_ptr(), T, K, x.stride(0), s.data_ptr(), H.data_ptr(),
+                                    _stream_ptr(x.device))
+    _check(st, "macaq_hessian_blocks")
+    return H
+
+
+def prepare_weight_hessian(W, s, H, out=None):
+    """prepare_weight with the Hessian exponent search over e0, e0 + 1, e0 - 1 per block."""
+    torch = _torch()
+    _require(W, torch.bfloat16, "W")
+    _require(s, torch.float32, "s")
+    N, K = W.shape
+    dev = W.device
+    if not (isinstance(H, torch.Tensor) and H.is_cuda and H.dtype == torch.float64 and H.is_contiguous()
+            and tuple(H.shape) == (K // 32, 32, 32)):
+        raise ValueError("H must be a contiguous float64 CUDA tensor [K/32, 32, 32]")
+    if out is None:
+        out = PreparedWeight(torch.empty((N, K // 2), dtype=torch.uint8, device=dev),
+                             torch.empty(scales_bytes(N, K), dtype=torch.uint8, device=dev),
+                             torch.empty(K, dtype=torch.float32, device=dev), N, K)
+    st = lib().macaq_prepare_weight_hessian(W.data_ptr(), N, K, W.stride(0), s.data_ptr(), H.data_ptr(),
+                                            out.codes.data_ptr(), out.scales.data_ptr(), out.inv_s.data_ptr(),
+                                            _stream_ptr(dev))
+    _check(st, "macaq_prepare_weight_hessian")
     return out
 
 

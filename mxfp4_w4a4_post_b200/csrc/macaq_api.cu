@@ -13,6 +13,7 @@
 
 #include "macaq.h"
 #include "gemm_kernel.cuh"
+#include "hessian_kernel.cuh"
 #include "quant_kernel.cuh"
 
 namespace macaq {
@@ -604,6 +605,47 @@ macaq_status macaq_linear_w4a4_noalloc(const void* x_bf16, int64_t M, int64_t ld
         scratch = g_noalloc_ptr[dev];
     }
     return macaq_linear_w4a4(x_bf16, M, ldx, w, y, ldy, out, 0, scratch, MACAQ_NOALLOC_SCRATCH_BYTES, stream);
+}
+
+size_t macaq_hessian_bytes(int64_t K) {
+    if (K < 32 || K % 32 != 0) return 0;
+    return (size_t)(K / 32) * 32 * 32 * sizeof(double);
+}
+
+macaq_status macaq_hessian_blocks(const void* x_bf16, int64_t T, int64_t K, int64_t ldx, const float* s, double* H,
+                                  macaq_stream stream) {
+    if (!x_bf16 || !s || !H) return MACAQ_ERR_INVALID_ARG;
+    if (T < 1 || K < 32 || ldx < K) return MACAQ_ERR_INVALID_ARG;
+    if (K % 32 != 0 || T > kMaxRows || K > kMaxK) return MACAQ_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(x_bf16) || !aligned16(s) || !aligned16(H) || ldx % 8 != 0) return MACAQ_ERR_MISALIGNED;
+    DeviceInfo* dev = nullptr;
+    macaq_status st = device_info(&dev);
+    if (st != MACAQ_OK) return st;
+    HessianParams hp{static_cast<const uint16_t*>(x_bf16), s, H, T, K, ldx};
+    return launch_pdl(hessian_blocks_kernel, dim3((unsigned)(K / 32)), dim3(1024), 0, (cudaStream_t)stream, hp) ==
+                   cudaSuccess
+               ? MACAQ_OK
+               : MACAQ_ERR_CUDA;
+}
+
+macaq_status macaq_prepare_weight_hessian(const void* W_bf16, int64_t N, int64_t K, int64_t ldw, const float* s,
+                                          const double* H, uint8_t* w_codes, uint8_t* w_scales, float* inv_s_out,
+                                          macaq_stream stream) {
+    macaq_status st = check_quant_args(W_bf16, N, K, ldw, s, w_codes, w_scales);
+    if (st != MACAQ_OK) return st;
+    if (!H || !inv_s_out) return MACAQ_ERR_INVALID_ARG;
+    if (!aligned16(H) || !aligned16(inv_s_out)) return MACAQ_ERR_MISALIGNED;
+    const int64_t slabs = round_up(N, 128) / 128;
+    if (slabs > 65535) return MACAQ_ERR_UNSUPPORTED_SHAPE;
+    DeviceInfo* dev = nullptr;
+    st = device_info(&dev);
+    if (st != MACAQ_OK) return st;
+    HessianPrepParams hp{static_cast<const uint16_t*>(W_bf16), s, H, w_codes, w_scales, inv_s_out, N, K, ldw,
+                         round_up(K / 32, 8)};
+    const dim3 grid((unsigned)hp.kb_pad, (unsigned)slabs);
+    return launch_pdl(prepare_weight_hessian_kernel, grid, dim3(128), 0, (cudaStream_t)stream, hp) == cudaSuccess
+               ? MACAQ_OK
+               : MACAQ_ERR_CUDA;
 }
 
 macaq_status macaq_get_device_error(void) {

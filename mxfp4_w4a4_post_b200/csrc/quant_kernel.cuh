@@ -114,9 +114,11 @@ __device__ __forceinline__ float absmax3(float a, float b, float c) { return max
 // The block transform and encoding for one block held as T[j] = elements (2j, 2j+1)
 // of u = x * mult: the butterfly, the shared exponent and the E2M1 codes (element i in nibble i % 8 of
 // packed[i / 8]). Returns the scale byte e + 127. T is overwritten.
-__device__ __forceinline__ uint32_t encode_block(uint64_t (&T)[16], uint32_t (&packed)[4]) {
-    const float c = __uint_as_float(0x3E3504F3u);        // nearest fp32 to 1/sqrt(32)
-    // butterfly stage h = 1 combines the two halves of each pair
+// The unnormalised 32-point butterfly on T[j] = elements (2j, 2j+1): stages
+// h = 1, 2, 4, 8, 16, pairs (a + b, a - b) with a at the lower index, fp32 round to
+// nearest at every step.
+__device__ __forceinline__ void butterfly_block(uint64_t (&T)[16]) {
+    // stage h = 1 combines the two halves of each pair
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
         float a, d;
@@ -134,6 +136,11 @@ __device__ __forceinline__ uint32_t encode_block(uint64_t (&T)[16], uint32_t (&p
             T[j + hp] = sub2(A, B);
         }
     }
+}
+
+__device__ __forceinline__ uint32_t encode_block(uint64_t (&T)[16], uint32_t (&packed)[4]) {
+    const float c = __uint_as_float(0x3E3504F3u);        // nearest fp32 to 1/sqrt(32)
+    butterfly_block(T);
 
     // max |t| as a three-level tree (the order of a max does not change its value)
     float a[32];
