@@ -1,0 +1,136 @@
+"""Per-call timing of the library on the seeded workloads, for the per-shape figures and
+the ncu captures that back them.
+
+    python -m mxfp4_w4a4_post_b200.timing list
+    python -m mxfp4_w4a4_post_b200.timing {quant,gemm,linear,hessian} WORKLOAD [--reps R]
+                                          [--warmup W] [--fused] [--calib T]
+
+Inputs are the workload's seeded synthetic tensors (workloads.py), resident on the
+device. Before every timed call L2 is flushed by a 256 MiB write and a read of the same
+buffer; each call is timed with CUDA events on the current stream and the mean is
+printed, one line per measured call:
+    quant    macaq_quant_act on x (weights prepared first)
+    gemm     macaq_gemm_mxfp4 on the quantised x and the prepared weight
+    linear   macaq_linear_w4a4 (fused = 0, or 1 with --fused)
+    hessian  macaq_hessian_blocks on T calibration rows (the workload's activation model
+             with another seed) and macaq_prepare_weight_hessian on the weight
+"""
+import argparse
+import sys
+
+import numpy as np
+
+from . import workloads as wl
+
+L2_FLUSH_BYTES = 256 << 20
+
+
+def all_workloads():
+    ws = {L.name: L for L in wl.all_single_layers()}
+    ws.update({L.name: L for L in wl.qwen3_32b_layer_decode(256)})
+    return ws
+
+
+def _bf16(torch, a, dev):
+    return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+
+
+def _time(torch, fn, flush, reps, warmup):
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    total = 0.0
+    for i in range(reps):
+        flush.fill_(i & 0xFF)
+        flush.view(torch.int32).max()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        fn()
+        b.record()
+        torch.cuda.synchronize()
+        total += a.elapsed_time(b) * 1e-3
+    return total / reps
+
+
+def main(argv=None):
+    p = argparse.ArgumentParser()
+    p.add_argument("what", choices=["list", "quant", "gemm", "linear", "hessian"])
+    p.add_argument("workload", nargs="?")
+    p.add_argument("--reps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--fused", action="store_true")
+    p.add_argument("--calib", type=int, default=2048, help="calibration rows for `hessian`")
+    a = p.parse_args(argv)
+    ws = all_workloads()
+    if a.what == "list":
+        print("\n".join(ws))
+        return 0
+    if a.workload not in ws:
+        p.error(f"unknown workload {a.workload!r}; see `list`")
+    import torch
+    import mxfp4_w4a4_post_b200 as mq
+    L = ws[a.workload]
+    dev = torch.device("cuda", torch.cuda.current_device())
+    M, N, K = L.M, L.N, L.K
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    W, s = _bf16(torch, wl.draw_W(L), dev), torch.from_numpy(wl.draw_s(L)).to(dev)
+    pw = mq.prepare_weight(W, s)
+    out = torch.bfloat16 if L.out_dtype == "bf16" else torch.float32
+    line = f"{L.name} M={M} N={N} K={K}"
+    # the C-ABI calls with their arguments marshalled once, so that host-side Python
+    # time stays out of the measured intervals
+    import ctypes
+    lib = mq.lib()
+    stream = ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+    cw = pw.c_struct()
+    oc = mq.OUT_BF16 if out == torch.bfloat16 else mq.OUT_F32
+
+    def call(fn, *args):
+        st = fn(*args)
+        if st != 0:
+            raise mq.MacaqError(st, fn.__name__)
+
+    if a.what in ("quant", "gemm", "linear"):
+        x = _bf16(torch, wl.draw_x(L), dev)
+        codes, scales = mq.quant_act(x, pw.inv_s)
+        y = torch.empty((M, N), dtype=out, device=dev)
+        if a.what == "quant":
+            args = (x.data_ptr(), M, K, x.stride(0), pw.inv_s.data_ptr(), codes.data_ptr(), scales.data_ptr(), stream)
+            t = _time(torch, lambda: call(lib.macaq_quant_act, *args), flush, a.reps, a.warmup)
+            print(f"{line} quant_act {t * 1e6:.2f} us {M * K * 2.53125 / t / 1e9:.1f} GB/s")
+        elif a.what == "gemm":
+            nws = mq.gemm_workspace_bytes(M, N, K, out)
+            ws_t = torch.empty(max(256, nws), dtype=torch.uint8, device=dev)
+            args = (codes.data_ptr(), scales.data_ptr(), M, ctypes.byref(cw), y.data_ptr(), y.stride(0), oc,
+                    ws_t.data_ptr(), ws_t.numel(), stream)
+            t = _time(torch, lambda: call(lib.macaq_gemm_mxfp4, *args), flush, a.reps, a.warmup)
+            print(f"{line} gemm_mxfp4 {t * 1e6:.2f} us {2.0 * M * N * K / t / 1e12:.1f} TFLOP/s "
+                  f"{(N * K + M * K) * 0.53125 / t / 1e9:.1f} GB/s of operands")
+        else:
+            ws_t = torch.empty(mq.linear_workspace_bytes(M, N, K, out), dtype=torch.uint8, device=dev)
+            args = (x.data_ptr(), M, x.stride(0), ctypes.byref(cw), y.data_ptr(), y.stride(0), oc,
+                    1 if a.fused else 0, ws_t.data_ptr(), ws_t.numel(), stream)
+            t = _time(torch, lambda: call(lib.macaq_linear_w4a4, *args), flush, a.reps, a.warmup)
+            print(f"{line} linear_w4a4 fused={int(a.fused)} {t * 1e6:.2f} us {2.0 * M * N * K / t / 1e12:.1f} TFLOP/s")
+    else:
+        from dataclasses import replace
+        xc = _bf16(torch, wl.draw_x(replace(L, M=a.calib, seed=L.seed + 100)), dev)
+        H = mq.hessian_blocks(xc, s)
+        hargs = (xc.data_ptr(), a.calib, K, xc.stride(0), s.data_ptr(), H.data_ptr(), stream)
+        t_h = _time(torch, lambda: call(lib.macaq_hessian_blocks, *hargs), flush, a.reps, a.warmup)
+        out_w = mq.prepare_weight_hessian(W, s, H)
+        pargs = (W.data_ptr(), N, K, W.stride(0), s.data_ptr(), H.data_ptr(), out_w.codes.data_ptr(),
+                 out_w.scales.data_ptr(), out_w.inv_s.data_ptr(), stream)
+        t_p = _time(torch, lambda: call(lib.macaq_prepare_weight_hessian, *pargs), flush, a.reps, a.warmup)
+        print(f"{line} hessian_blocks T={a.calib} {t_h * 1e6:.1f} us "
+              f"{2.0 * a.calib * K * 32 / t_h / 1e12:.2f} TFLOP/s fp64")
+        print(f"{line} prepare_weight_hessian {t_p * 1e6:.1f} us "
+              f"{N * (K // 32) * 3 * 2048 / t_p / 1e12:.2f} TFLOP/s fp64")
+    if mq.device_error() != 0:
+        print("device error word set", file=sys.stderr)
+        return 1
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())
