@@ -72,6 +72,12 @@ def lib():
         L.oracle_search_block.restype = None
         L.oracle_prepare_weight_hessian.argtypes = [P, I64, I64, I64, P, P, P, P, P]
         L.oracle_prepare_weight_hessian.restype = None
+        L.oracle_hessian_full.argtypes = [P, I64, I64, I64, P, P]
+        L.oracle_hessian_full.restype = None
+        L.oracle_flip_refine_row.argtypes = [P, P, I64, P, P, ctypes.c_int]
+        L.oracle_flip_refine_row.restype = ctypes.c_int
+        L.oracle_flip_refine.argtypes = [P, I64, I64, I64, P, P, P, P, ctypes.c_int, P]
+        L.oracle_flip_refine.restype = None
         _lib = L
     return _lib
 
@@ -201,6 +207,40 @@ def prepare_weight_hessian(W_bf16, s, H):
     inv_s = np.empty(K, np.float32)
     lib().oracle_prepare_weight_hessian(_p(W), N, K, K, _p(s), _p(Hh), _p(codes), _p(scales), _p(inv_s))
     return codes, scales, inv_s
+
+
+def hessian_full(x_bf16, inv_s):
+    """Full K x K Gram matrix of the transformed rows of x (fp64)."""
+    x = _c(x_bf16, np.uint16)
+    m = _c(inv_s, np.float32)
+    T, K = x.shape
+    H = np.empty((K, K), np.float64)
+    lib().oracle_hessian_full(_p(x), T, K, K, _p(m), _p(H))
+    return H
+
+
+def flip_refine_row(wv, H, codes_row, scales_row, max_rounds):
+    """Returns (refined codes [K/2], number of moves)."""
+    w = _c(wv, np.float32)
+    Hh = _c(H, np.float64)
+    c = np.array(codes_row, np.uint8, copy=True)
+    sr = _c(scales_row, np.uint8)
+    n = lib().oracle_flip_refine_row(_p(w), _p(Hh), w.size, _p(c), _p(sr), int(max_rounds))
+    return c, n
+
+
+def flip_refine(W_bf16, s, H, codes, scales_rowmajor, max_rounds):
+    """Returns (refined codes [N, K/2], moves int32 [N])."""
+    W = _c(W_bf16, np.uint16)
+    s = _c(s, np.float32)
+    N, K = W.shape
+    Hh = _c(H, np.float64)
+    assert Hh.shape == (K, K)
+    c = np.array(codes, np.uint8, copy=True)
+    sc = _c(scales_rowmajor, np.uint8)
+    moves = np.empty(N, np.int32)
+    lib().oracle_flip_refine(_p(W), N, K, K, _p(s), _p(Hh), _p(c), _p(sc), int(max_rounds), _p(moves))
+    return c, moves
 
 
 def scale_rows_padded(rows):

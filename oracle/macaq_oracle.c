@@ -367,3 +367,98 @@ void oracle_prepare_weight_hessian(const uint16_t* W, int64_t N, int64_t K, int6
         }
     }
 }
+
+/* ----------------------------------------------------- Flip-Refinement ------ */
+
+void oracle_hessian_full(const uint16_t* x, int64_t T, int64_t K, int64_t ld, const float* inv_s, double* H) {
+    int64_t Kb = K / 32;
+    float* v = (float*)malloc((size_t)K * sizeof(float));
+    memset(H, 0, (size_t)(K * K) * sizeof(double));
+    for (int64_t t = 0; t < T; ++t) {
+        for (int64_t b = 0; b < Kb; ++b) oracle_transform_block_f32(x + t * ld, inv_s, b, v + 32 * b);
+        for (int64_t i = 0; i < K; ++i)
+            for (int64_t j = 0; j < K; ++j) H[i * K + j] += (double)v[i] * (double)v[j];
+    }
+    free(v);
+}
+
+/* The 15 signed E2M1 values in increasing order; index 7 is zero. */
+static const double kFlipGrid[15] = {-6.0, -4.0, -3.0, -2.0, -1.5, -1.0, -0.5, 0.0,
+                                     0.5,  1.0,  1.5,  2.0,  3.0,  4.0,  6.0};
+
+static int flip_index(uint8_t code) {
+    int m = code & 7;
+    if (m == 0) return 7;
+    return (code & 8) ? 7 - m : 7 + m;
+}
+
+static uint8_t flip_code(int index) {
+    if (index == 7) return 0;
+    return index > 7 ? (uint8_t)(index - 7) : (uint8_t)(8 | (7 - index));
+}
+
+int oracle_flip_refine_row(const float* wv, const double* H, int64_t K, uint8_t* codes, const uint8_t* scales_row,
+                           int max_rounds) {
+    double* e = (double*)malloc((size_t)K * sizeof(double));
+    double* g = (double*)malloc((size_t)K * sizeof(double));
+    int* idx = (int*)malloc((size_t)K * sizeof(int));
+    for (int64_t k = 0; k < K; ++k) {
+        uint8_t byte = codes[k / 2];
+        uint8_t code = (k & 1) ? (uint8_t)(byte >> 4) : (uint8_t)(byte & 0xF);
+        idx[k] = flip_index(code);
+        e[k] = (double)wv[k] - ldexp(kFlipGrid[idx[k]], (int)scales_row[k / 32] - 127);
+    }
+    for (int64_t j = 0; j < K; ++j) {
+        double acc = 0.0;
+        for (int64_t k = 0; k < K; ++k) acc = fma(H[j * K + k], e[k], acc);
+        g[j] = acc;
+    }
+    int moves = 0;
+    for (int round = 0; round < max_rounds; ++round) {
+        double best = 0.0;
+        int64_t bk = -1;
+        int bdir = 0;
+        double bdelta = 0.0;
+        for (int64_t k = 0; k < K; ++k) {
+            int sc = (int)scales_row[k / 32] - 127;
+            for (int dir = -1; dir <= 1; dir += 2) {
+                int ni = idx[k] + dir;
+                if (ni < 0 || ni > 14) continue;
+                double delta = ldexp(kFlipGrid[ni] - kFlipGrid[idx[k]], sc);
+                double a = delta * delta;
+                double b2 = a * H[k * K + k];
+                double c = (2.0 * delta) * g[k];
+                double dE = b2 - c;
+                if (dE < best) {
+                    best = dE;
+                    bk = k;
+                    bdir = dir;
+                    bdelta = delta;
+                }
+            }
+        }
+        if (bk < 0) break;
+        idx[bk] += bdir;
+        uint8_t nc = flip_code(idx[bk]);
+        uint8_t* byte = &codes[bk / 2];
+        *byte = (bk & 1) ? (uint8_t)((*byte & 0x0F) | (nc << 4)) : (uint8_t)((*byte & 0xF0) | nc);
+        e[bk] -= bdelta;
+        for (int64_t j = 0; j < K; ++j) g[j] = fma(-bdelta, H[bk * K + j], g[j]);
+        ++moves;
+    }
+    free(idx);
+    free(g);
+    free(e);
+    return moves;
+}
+
+void oracle_flip_refine(const uint16_t* W, int64_t N, int64_t K, int64_t ld, const float* s, const double* H,
+                        uint8_t* codes, const uint8_t* scales, int max_rounds, int32_t* moves) {
+    int64_t Kb = K / 32;
+    float* wv = (float*)malloc((size_t)K * sizeof(float));
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t b = 0; b < Kb; ++b) oracle_transform_block_f32(W + n * ld, s, b, wv + 32 * b);
+        moves[n] = oracle_flip_refine_row(wv, H, K, codes + n * (K / 2), scales + n * Kb, max_rounds);
+    }
+    free(wv);
+}

@@ -144,6 +144,40 @@ void oracle_search_block(const float v[32], const double H[32 * 32], uint8_t cod
 void oracle_prepare_weight_hessian(const uint16_t* W, int64_t N, int64_t K, int64_t ld, const float* s,
                                    const double* H, uint8_t* codes, uint8_t* scales, float* inv_s);
 
+/* ------------------------------------------------------------------------------
+ * Flip-Refinement of weight codes (the Flip-Refinement paragraphs of the zicq.com
+ * articles and of the openai-hub.com article: starting from quantised weights, each
+ * round moves, for every output row, the one code whose move to an adjacent
+ * representable value lowers the second-order error most; a row stops when no such move
+ * lowers it). Reading taken: the error of row n is E = e^T H e, e = w' - w_hat (the
+ * transformed weight row minus its dequantised codes), H the full K x K Gram matrix of
+ * the transformed calibration rows; block scales stay fixed; the representable values of
+ * a coordinate are the 15 signed E2M1 values times its block scale. With g = H e, moving
+ * coordinate k by delta changes E by delta^2 H_kk - 2 delta g_k, and g then changes by
+ * -delta H[k, :].
+ * ---------------------------------------------------------------------------- */
+
+/* H[i][j] = sum_t v_t[i] v_t[j] over all K columns (t ascending), fp64, K x K. */
+void oracle_hessian_full(const uint16_t* x, int64_t T, int64_t K, int64_t ld, const float* inv_s, double* H);
+
+/* One row. wv: the K transformed fp32 weight values; codes: K/2 bytes, refined in place;
+ * scales_row: K/32 E8M0 bytes (row-major); at most max_rounds moves. fp64 throughout:
+ *   e_k = wv_k - value(code_k) 2^(scale - 127)                   (exact)
+ *   g_j = fma chain over k ascending of H[j][k] * e_k, from 0
+ *   for each k ascending, first the lower then the higher neighbour value:
+ *     delta = (neighbour - value) 2^(scale - 127)                 (exact)
+ *     dE = (delta * delta) * H[k][k] - (2 delta) * g_k           (each op rounded)
+ *   the first strictly smallest dE < 0 is taken (none: the row stops);
+ *   then e_k -= delta and g_j = fma(-delta, H[k][j], g_j) for every j.
+ * A move to the value 0 writes code 0 (+0). Returns the number of moves. */
+int oracle_flip_refine_row(const float* wv, const double* H, int64_t K, uint8_t* codes, const uint8_t* scales_row,
+                           int max_rounds);
+
+/* Every row of a prepared weight: wv from W and s by the weight transform, codes
+ * (N x K/2) refined in place, scales row-major (N x K/32); moves[n] receives the count. */
+void oracle_flip_refine(const uint16_t* W, int64_t N, int64_t K, int64_t ld, const float* s, const double* H,
+                        uint8_t* codes, const uint8_t* scales, int max_rounds, int32_t* moves);
+
 #ifdef __cplusplus
 }
 #endif

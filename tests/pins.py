@@ -473,4 +473,147 @@ def pin_prepare_weight_hessian():
             assert np.array_equal(c2[n, 16 * b:16 * b + 16], pack_nibbles(codes[None, :])[0]), (n, b)
 
 
+# ------------------------------------------------------------ Flip-Refinement ---
+
+FLIP_GRID = np.array([-6, -4, -3, -2, -1.5, -1, -0.5, 0, 0.5, 1, 1.5, 2, 3, 4, 6], np.float64)
+
+
+def _decode_row(codes_row, scales_row, K):
+    """Dequantised row from the golden E2M1 table and the E8M0 bytes."""
+    table = golden_e2m1()
+    nib = np.empty(K, np.uint8)
+    nib[0::2] = codes_row & 0xF
+    nib[1::2] = codes_row >> 4
+    vals = np.array([(-1.0 if c & 8 else 1.0) * table[c & 7] for c in nib])
+    return vals * 2.0 ** (np.repeat(scales_row.astype(np.int64), 32) - 127)
+
+
+def _local_gains(wv, H, codes_row, scales_row):
+    """Every adjacent move's change of e^T H e, by numpy (grid positions from values)."""
+    K = wv.size
+    what = _decode_row(codes_row, scales_row, K)
+    step = 2.0 ** (np.repeat(scales_row.astype(np.int64), 32) - 127)
+    e = wv.astype(np.float64) - what
+    g = H @ e
+    gains = []
+    for k in range(K):
+        pos = int(np.argmin(np.abs(FLIP_GRID - what[k] / step[k])))
+        for d in (-1, 1):
+            if 0 <= pos + d <= 14:
+                delta = (FLIP_GRID[pos + d] - FLIP_GRID[pos]) * step[k]
+                gains.append(delta * delta * H[k, k] - 2 * delta * g[k])
+    return np.array(gains), float(e @ H @ e)
+
+
+def pin_hessian_full():
+    rng = np.random.default_rng(30)
+    T, K = 9, 96
+    x = rng.standard_t(3, size=(T, K)).astype(np.float32)
+    xb = (x.view(np.uint32) >> 16).astype(np.uint16)
+    inv_s = np.exp(rng.normal(0, 0.5, K)).astype(np.float32)
+    H = oracle.hessian_full(xb, inv_s)
+    V = np.concatenate([np.stack([oracle.transform_block(xb[t], inv_s, b) for b in range(K // 32)]).reshape(-1)[None]
+                        for t in range(T)]).astype(np.float64)
+    assert np.allclose(H, V.T @ V, rtol=1e-13, atol=1e-300)
+    assert np.array_equal(H, H.T)
+    Hb = oracle.hessian_blocks(xb, inv_s)
+    for b in range(K // 32):                          # same products, same order
+        assert np.array_equal(H[32 * b:32 * b + 32, 32 * b:32 * b + 32], Hb[b]), b
+    _, xb2, mult = _exact_rows(rng, 4, 64)
+    H2 = oracle.hessian_full(xb2, mult)
+    V2 = np.concatenate([np.stack([oracle.transform_block(xb2[t], mult, b) for b in range(2)]).reshape(-1)[None]
+                         for t in range(4)]).astype(np.float64)
+    assert np.array_equal(H2, V2.T @ V2)
+
+
+def pin_flip_refine_special_cases():
+    rng = np.random.default_rng(31)
+    N, K = 5, 64
+    W = rng.normal(0, 0.02, (N, K)).astype(np.float32)
+    Wb = (W.view(np.uint32) >> 16).astype(np.uint16)
+    s = np.exp(rng.normal(0, 0.5, K)).astype(np.float32)
+    c, sc, _ = oracle.prepare_weight(Wb, s)
+    # diagonal H: coordinates are independent and round-to-nearest is already optimal
+    Hd = np.diag(rng.uniform(0.1, 3.0, K))
+    c1, m1 = oracle.flip_refine(Wb, s, Hd, c, sc, 1000)
+    assert (m1 == 0).all() and np.array_equal(c1, c)
+    # H = 0: no move lowers the error strictly
+    c2, m2 = oracle.flip_refine(Wb, s, np.zeros((K, K)), c, sc, 1000)
+    assert (m2 == 0).all() and np.array_equal(c2, c)
+    # planted, worked by hand: H = I except H01 = H10 = 0.9, w' = (0.74, 0.70, 0, ...), scale
+    # 2^0; round to nearest gives (0.5, 0.5), e = (0.24, 0.20), g = H e = (0.42, 0.416); the
+    # best move takes coordinate 0 up to 1.0 (dE = 0.25 - 0.42 = -0.17, against -0.166 for
+    # coordinate 1), g becomes (-0.08, -0.034) and no move helps any more
+    H = np.eye(32)
+    H[0, 1] = H[1, 0] = 0.9
+    wv = np.zeros(32, np.float32)
+    wv[0], wv[1] = 0.74, 0.70
+    codes = np.zeros(16, np.uint8)
+    codes[0] = 0x11                                 # codes 1 | 1 << 4: values 0.5, 0.5
+    out, n = oracle.flip_refine_row(wv, H, codes, np.array([127], np.uint8), 100)
+    assert n == 1 and out[0] == 0x12 and (out[1:] == 0).all(), (n, out[:2])
+
+
+def pin_flip_refine_local_optimum():
+    rng = np.random.default_rng(32)
+    N, K, T = 6, 96, 40
+    W = rng.normal(0, 0.02, (N, K)).astype(np.float32)
+    Wb = (W.view(np.uint32) >> 16).astype(np.uint16)
+    s = np.exp(rng.normal(0, 0.5, K)).astype(np.float32)
+    x = rng.standard_t(3, size=(T, K)).astype(np.float32)
+    x[:, 7] *= 20
+    xb = (x.view(np.uint32) >> 16).astype(np.uint16)
+    H = oracle.hessian_full(xb, (np.float32(1.0) / s).astype(np.float32))
+    c, sc, _ = oracle.prepare_weight(Wb, s)
+    c2, moves = oracle.flip_refine(Wb, s, H, c, sc, 10000)
+    assert moves.sum() > 0
+    for n in range(N):
+        wv = np.concatenate([oracle.transform_block(Wb[n], s, b) for b in range(K // 32)])
+        g0, e0 = _local_gains(wv, H, c[n], sc[n])
+        g1, e1 = _local_gains(wv, H, c2[n], sc[n])
+        assert e1 <= e0 * (1 + 1e-12), n              # never worse than round to nearest
+        assert (g1 >= -1e-9 * max(e0, 1e-300)).all(), (n, g1.min())   # no improving move left
+        assert int((c2[n] != c[n]).sum()) <= 2 * moves[n]
+    # a cap on the rounds is honoured
+    c3, m3 = oracle.flip_refine(Wb, s, H, c, sc, 1)
+    assert (m3 <= 1).all() and (m3 == np.minimum(moves, 1)).all()
+
+
+def pin_flip_refine_brute_force():
+    """Three coupled coordinates in one block, the rest zero: every code triple is
+    enumerated; the refined triple is no worse than round to nearest, is a local
+    optimum, and starting from the global optimum no move is made."""
+    rng = np.random.default_rng(33)
+    for trial in range(6):
+        A = rng.standard_normal((3, 3))
+        H = np.eye(32)
+        H[:3, :3] = A @ A.T + 0.05 * np.eye(3)
+        wv = np.zeros(32, np.float32)
+        wv[:3] = rng.uniform(-2.5, 2.5, 3).astype(np.float32)
+        sc = np.array([127], np.uint8)
+        best = None
+        for i in range(15):
+            for j in range(15):
+                for k in range(15):
+                    d = wv[:3].astype(np.float64) - FLIP_GRID[[i, j, k]]
+                    E = float(d @ H[:3, :3] @ d)
+                    if best is None or E < best[0]:
+                        best = (E, (i, j, k))
+        def codes_of(idx):
+            nib = np.zeros(32, np.uint8)
+            for p_, gi in enumerate(idx):
+                v = FLIP_GRID[gi]
+                m = {0.0: 0, 0.5: 1, 1.0: 2, 1.5: 3, 2.0: 4, 3.0: 5, 4.0: 6, 6.0: 7}[abs(v)]
+                nib[p_] = m | (8 if v < 0 and m else 0)
+            return (nib[0::2] | (nib[1::2] << 4)).astype(np.uint8)
+        rtn = tuple(int(np.argmin(np.abs(FLIP_GRID - float(w)))) for w in wv[:3])
+        out, n = oracle.flip_refine_row(wv, H, codes_of(rtn), sc, 1000)
+        gains, E = _local_gains(wv, H, out, sc)
+        _, E_rtn = _local_gains(wv, H, codes_of(rtn), sc)
+        assert best[0] <= E + 1e-12 and E <= E_rtn + 1e-12, trial
+        assert (gains >= -1e-12).all(), trial
+        out2, n2 = oracle.flip_refine_row(wv, H, codes_of(best[1]), sc, 1000)
+        assert n2 == 0 and np.array_equal(out2, codes_of(best[1])), trial
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

@@ -48,6 +48,14 @@ MUTANTS = [
     ("search_nibble_order", "codes16[j] = (uint8_t)((hi << 4) | lo);", "codes16[j] = (uint8_t)((lo << 4) | hi);"),
     ("search_ties_replace", "if (!have || err < best) {", "if (!have || err <= best) {"),
     ("search_no_lower_candidate", "int cand[3] = {e0, e0 + 1, e0 - 1};", "int cand[3] = {e0, e0 + 1, e0 + 1};"),
+    ("flip_gain_sign", "double dE = b2 - c;", "double dE = b2 + c;"),
+    ("flip_update_sign", "g[j] = fma(-bdelta, H[bk * K + j], g[j]);", "g[j] = fma(bdelta, H[bk * K + j], g[j]);"),
+    ("flip_ties_accepted", "if (dE < best) {", "if (dE <= best) {"),
+    ("flip_neighbour", "int ni = idx[k] + dir;", "int ni = idx[k] + 2 * dir;"),
+    ("flip_error_sign", "e[k] = (double)wv[k] - ldexp(kFlipGrid[idx[k]], (int)scales_row[k / 32] - 127);",
+     "e[k] = (double)wv[k] + ldexp(kFlipGrid[idx[k]], (int)scales_row[k / 32] - 127);"),
+    ("hessian_full_diagonal", "for (int64_t j = 0; j < K; ++j) H[i * K + j] += (double)v[i] * (double)v[j];",
+     "H[i * K + i] += (double)v[i] * (double)v[i];"),
 ]
 
 
