@@ -195,6 +195,50 @@ macaq_status macaq_prepare_weight_hessian(const void* W_bf16, int64_t N, int64_t
                                           const double* H, uint8_t* w_codes, uint8_t* w_scales, float* inv_s_out,
                                           macaq_stream stream);
 
+/* ------------------------------------------------ Flip-Refinement (offline) ----- */
+
+/* The Flip-Refinement paragraphs of the zicq.com and openai-hub.com articles: after
+ * quantisation, each round moves, for every output row, the one code whose step to an
+ * adjacent representable value lowers the second-order error most; a row stops when no
+ * step lowers it. Error of row n: e^T H e, e = w' - w_hat (transformed weights minus the
+ * dequantised codes), H the full K x K Gram matrix of transformed calibration rows
+ * (macaq_hessian_full). Block scales stay fixed; codes move along the 15 signed E2M1
+ * values. Only weight codes change: the result feeds the same GEMM. */
+
+/* Workspace of macaq_hessian_full: the fp32 transformed calibration rows (T x K). */
+size_t macaq_hessian_full_workspace_bytes(int64_t T, int64_t K);
+
+/* H[i][j] = sum over t = 0 .. T-1 (in that order) of v_t[i] * v_t[j], fp64, K x K,
+ * v_t calibration row t after the online transform with inv_s = RN32(1/s); exactly
+ * symmetric (both halves from the same products). Bit-identical to that sequential
+ * definition (products of two fp32 values are exact in fp64).
+ *   x_bf16 [T x K] (ldx >= K, ldx % 8 == 0), s [K], H [K x K] fp64: device, 16-byte aligned
+ *   workspace >= macaq_hessian_full_workspace_bytes(T, K), 16-byte aligned
+ * K % 32 == 0, K <= 8192. */
+macaq_status macaq_hessian_full(const void* x_bf16, int64_t T, int64_t K, int64_t ldx, const float* s, double* H,
+                                void* workspace, size_t ws_bytes, macaq_stream stream);
+
+/* Workspace of macaq_flip_refine: transformed weight rows (fp32) and their initial
+ * gradients (fp64), N x K each. */
+size_t macaq_flip_workspace_bytes(int64_t N, int64_t K);
+
+/* Flip-Refinement of a prepared weight's codes, in place, rows in parallel. Per row, fp64:
+ *   e_k = w'_k - dec(code_k) 2^(scale - 127) (exact); g_j = fma chain over k ascending
+ *   of H[j][k] e_k from 0; per round, for k ascending, lower then higher neighbour:
+ *   delta = (neighbour - value) 2^(scale - 127), dE = (delta delta) H_kk - (2 delta) g_k
+ *   (each operation rounded); the first strictly smallest dE < 0 is applied (code
+ *   changed, a move to 0 writing +0), then g_j = fma(-delta, H[k][j], g_j); the row stops
+ *   when no dE < 0 remains or after max_rounds moves. Bit-identical to that definition.
+ *   W_bf16, s      the weight and channel scales macaq_prepare_weight(_hessian) was given
+ *   H              device fp64 [K x K], symmetric (as macaq_hessian_full writes it)
+ *   w_codes        device [N x K/2], refined in place; w_scales: its scale atoms
+ *   moves          device int32 [N]: the number of moves made in each row
+ *   workspace      >= macaq_flip_workspace_bytes(N, K), 16-byte aligned
+ * K % 32 == 0, K <= 8192, max_rounds >= 0. */
+macaq_status macaq_flip_refine(const void* W_bf16, int64_t N, int64_t K, int64_t ldw, const float* s, const double* H,
+                               uint8_t* w_codes, const uint8_t* w_scales, int max_rounds, int32_t* moves,
+                               void* workspace, size_t ws_bytes, macaq_stream stream);
+
 /* Largest scratch the no-allocation variant below can use: 16 MiB, held in a static
  * device array on every GPU that loads this library, for as long as it stays loaded. */
 #define MACAQ_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)

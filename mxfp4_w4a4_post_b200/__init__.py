@@ -60,6 +60,10 @@ def lib():
             "macaq_hessian_bytes": (SZ, [I64]),
             "macaq_hessian_blocks": (I, [P, I64, I64, I64, P, P, P]),
             "macaq_prepare_weight_hessian": (I, [P, I64, I64, I64, P, P, P, P, P, P]),
+            "macaq_hessian_full_workspace_bytes": (SZ, [I64, I64]),
+            "macaq_hessian_full": (I, [P, I64, I64, I64, P, P, P, SZ, P]),
+            "macaq_flip_workspace_bytes": (SZ, [I64, I64]),
+            "macaq_flip_refine": (I, [P, I64, I64, I64, P, P, P, P, I, P, P, SZ, P]),
             "macaq_get_device_error": (I, []),
             "macaq_status_string": (ctypes.c_char_p, [I]),
             "macaq_version": (I, []),
@@ -189,6 +193,41 @@ def prepare_weight_hessian(W, s, H, out=None):
                                             _stream_ptr(dev))
     _check(st, "macaq_prepare_weight_hessian")
     return out
+
+
+def hessian_full(x, s, H=None):
+    """Calibration activations x: bf16 [T, K]; s: fp32 [K]. Returns the full fp64 Gram
+    matrix H [K, K] of the transformed rows (the input of flip_refine)."""
+    torch = _torch()
+    _require(x, torch.bfloat16, "x")
+    _require(s, torch.float32, "s")
+    T, K = x.shape
+    if H is None:
+        H = torch.empty((K, K), dtype=torch.float64, device=x.device)
+    nws = lib().macaq_hessian_full_workspace_bytes(T, K)
+    ws = torch.empty(max(nws, 256), dtype=torch.uint8, device=x.device)
+    st = lib().macaq_hessian_full(x.data_ptr(), T, K, x.stride(0), s.data_ptr(), H.data_ptr(), ws.data_ptr(),
+                                  ws.numel(), _stream_ptr(x.device))
+    _check(st, "macaq_hessian_full")
+    return H
+
+
+def flip_refine(W, s, H, w, max_rounds=1 << 20, workspace=None):
+    """Flip-Refinement of the prepared weight w's codes, in place. Returns the number of
+    moves per row (int32 CUDA tensor [N])."""
+    torch = _torch()
+    _require(W, torch.bfloat16, "W")
+    _require(s, torch.float32, "s")
+    N, K = W.shape
+    dev = W.device
+    moves = torch.empty(N, dtype=torch.int32, device=dev)
+    need = lib().macaq_flip_workspace_bytes(N, K)
+    ws, ws_bytes = _workspace(need, dev, workspace)
+    st = lib().macaq_flip_refine(W.data_ptr(), N, K, W.stride(0), s.data_ptr(), H.data_ptr(), w.codes.data_ptr(),
+                                 w.scales.data_ptr(), int(max_rounds), moves.data_ptr(), ws.data_ptr(), ws_bytes,
+                                 _stream_ptr(dev))
+    _check(st, "macaq_flip_refine")
+    return moves
 
 
 def quant_act(x, inv_s, codes=None, scales=None):

@@ -12,6 +12,7 @@
 #include <numeric>
 
 #include "macaq.h"
+#include "flip_kernel.cuh"
 #include "gemm_kernel.cuh"
 #include "hessian_kernel.cuh"
 #include "quant_kernel.cuh"
@@ -80,6 +81,7 @@ inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 // Limits that keep every index inside 32 bits where the kernels use int.
 constexpr int64_t kMaxRows = (int64_t)1 << 30;
 constexpr int64_t kMaxK = (int64_t)1 << 24;
+constexpr int64_t kMaxFlipK = 8192;     // Flip-Refinement keeps a row's gradient in shared memory
 
 // --------------------------------------------------------------------- quant ---
 
@@ -646,6 +648,83 @@ macaq_status macaq_prepare_weight_hessian(const void* W_bf16, int64_t N, int64_t
     return launch_pdl(prepare_weight_hessian_kernel, grid, dim3(128), 0, (cudaStream_t)stream, hp) == cudaSuccess
                ? MACAQ_OK
                : MACAQ_ERR_CUDA;
+}
+
+size_t macaq_hessian_full_workspace_bytes(int64_t T, int64_t K) {
+    if (T < 1 || K < 32 || K % 32 != 0) return 0;
+    return (size_t)round_up(T * K * 4, 256);
+}
+
+macaq_status macaq_hessian_full(const void* x_bf16, int64_t T, int64_t K, int64_t ldx, const float* s, double* H,
+                                void* workspace, size_t ws_bytes, macaq_stream stream) {
+    if (!x_bf16 || !s || !H) return MACAQ_ERR_INVALID_ARG;
+    if (T < 1 || K < 32 || ldx < K) return MACAQ_ERR_INVALID_ARG;
+    if (K % 32 != 0 || T > kMaxRows || K > kMaxFlipK) return MACAQ_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(x_bf16) || !aligned16(s) || !aligned16(H) || ldx % 8 != 0) return MACAQ_ERR_MISALIGNED;
+    const size_t need = macaq_hessian_full_workspace_bytes(T, K);
+    if (!workspace || ws_bytes < need) return MACAQ_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return MACAQ_ERR_MISALIGNED;
+    DeviceInfo* dev = nullptr;
+    macaq_status st = device_info(&dev);
+    if (st != MACAQ_OK) return st;
+    cudaStream_t cs = (cudaStream_t)stream;
+    float* xt = static_cast<float*>(workspace);
+    TransformParams tp{static_cast<const uint16_t*>(x_bf16), s, xt, T, K, ldx, 1};
+    const int64_t blocks = std::min<int64_t>(cdiv(T * (K / 32), 128), (int64_t)dev->num_sms * 16);
+    if (launch_pdl(transform_rows_kernel, dim3((unsigned)blocks), dim3(128), 0, cs, tp) != cudaSuccess)
+        return MACAQ_ERR_CUDA;
+    const int64_t nb = K / 32;
+    GramParams gp{xt, H, T, K};
+    if (launch_pdl(gram_tile_kernel, dim3((unsigned)(nb * (nb + 1) / 2)), dim3(1024), 0, cs, gp) != cudaSuccess)
+        return MACAQ_ERR_CUDA;
+    return MACAQ_OK;
+}
+
+size_t macaq_flip_workspace_bytes(int64_t N, int64_t K) {
+    if (N < 1 || K < 32 || K % 32 != 0) return 0;
+    return (size_t)round_up(N * K * 4, 256) + (size_t)round_up(N * K * 8, 256);
+}
+
+macaq_status macaq_flip_refine(const void* W_bf16, int64_t N, int64_t K, int64_t ldw, const float* s, const double* H,
+                               uint8_t* w_codes, const uint8_t* w_scales, int max_rounds, int32_t* moves,
+                               void* workspace, size_t ws_bytes, macaq_stream stream) {
+    macaq_status st = check_quant_args(W_bf16, N, K, ldw, s, w_codes, w_scales);
+    if (st != MACAQ_OK) return st;
+    if (!H || !moves || max_rounds < 0) return MACAQ_ERR_INVALID_ARG;
+    if (K > kMaxFlipK || cdiv(N, 64) > 65535) return MACAQ_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(H) || !aligned16(moves)) return MACAQ_ERR_MISALIGNED;
+    const size_t need = macaq_flip_workspace_bytes(N, K);
+    if (!workspace || ws_bytes < need) return MACAQ_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return MACAQ_ERR_MISALIGNED;
+    DeviceInfo* dev = nullptr;
+    st = device_info(&dev);
+    if (st != MACAQ_OK) return st;
+    cudaStream_t cs = (cudaStream_t)stream;
+    float* wv = static_cast<float*>(workspace);
+    double* G = reinterpret_cast<double*>(static_cast<uint8_t*>(workspace) + round_up(N * K * 4, 256));
+    const int64_t kb_pad = round_up(K / 32, 8);
+    TransformParams tp{static_cast<const uint16_t*>(W_bf16), s, wv, N, K, ldw, 0};
+    const int64_t blocks = std::min<int64_t>(cdiv(N * (K / 32), 128), (int64_t)dev->num_sms * 16);
+    if (launch_pdl(transform_rows_kernel, dim3((unsigned)blocks), dim3(128), 0, cs, tp) != cudaSuccess)
+        return MACAQ_ERR_CUDA;
+    FlipGradParams fg{wv, w_codes, w_scales, H, G, N, K, kb_pad};
+    if (launch_pdl(flip_gradient_kernel, dim3((unsigned)cdiv(K, 64), (unsigned)cdiv(N, 64)), dim3(256), 0, cs, fg) !=
+        cudaSuccess)
+        return MACAQ_ERR_CUDA;
+    const size_t smem = flip_rounds_smem(K);
+    static std::atomic<uint64_t> configured{0};
+    int devid = 0;
+    cudaGetDevice(&devid);
+    if (!(configured.load() & (1ull << (devid & 63)))) {
+        if (cudaFuncSetAttribute(flip_rounds_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)flip_rounds_smem(kMaxFlipK)) != cudaSuccess)
+            return MACAQ_ERR_CUDA;
+        configured.fetch_or(1ull << (devid & 63));
+    }
+    FlipRoundParams fr{wv, w_codes, w_scales, H, G, moves, N, K, kb_pad, max_rounds};
+    if (launch_pdl(flip_rounds_kernel, dim3((unsigned)N), dim3(kFlipThreads), smem, cs, fr) != cudaSuccess)
+        return MACAQ_ERR_CUDA;
+    return MACAQ_OK;
 }
 
 macaq_status macaq_get_device_error(void) {

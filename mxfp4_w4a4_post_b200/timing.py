@@ -2,8 +2,8 @@
 the ncu captures that back them.
 
     python -m mxfp4_w4a4_post_b200.timing list
-    python -m mxfp4_w4a4_post_b200.timing {quant,gemm,linear,hessian} WORKLOAD [--reps R]
-                                          [--warmup W] [--fused] [--calib T]
+    python -m mxfp4_w4a4_post_b200.timing {quant,gemm,linear,hessian,flip} WORKLOAD [--reps R]
+                                          [--warmup W] [--fused] [--calib T] [--rounds R]
 
 Inputs are the workload's seeded synthetic tensors (workloads.py), resident on the
 device. Before every timed call L2 is flushed by a 256 MiB write and a read of the same
@@ -14,6 +14,9 @@ printed, one line per measured call:
     linear   macaq_linear_w4a4 (fused = 0, or 1 with --fused)
     hessian  macaq_hessian_blocks on T calibration rows (the workload's activation model
              with another seed) and macaq_prepare_weight_hessian on the weight
+    flip     macaq_hessian_full on T calibration rows, then macaq_flip_refine of the
+             prepared weight (each timed call starts again from the round-to-nearest
+             codes, restored before the flush); also prints the moves per row
 """
 import argparse
 import sys
@@ -54,12 +57,13 @@ def _time(torch, fn, flush, reps, warmup):
 
 def main(argv=None):
     p = argparse.ArgumentParser()
-    p.add_argument("what", choices=["list", "quant", "gemm", "linear", "hessian"])
+    p.add_argument("what", choices=["list", "quant", "gemm", "linear", "hessian", "flip"])
     p.add_argument("workload", nargs="?")
     p.add_argument("--reps", type=int, default=20)
     p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--fused", action="store_true")
-    p.add_argument("--calib", type=int, default=2048, help="calibration rows for `hessian`")
+    p.add_argument("--calib", type=int, default=2048, help="calibration rows for `hessian` and `flip`")
+    p.add_argument("--rounds", type=int, default=256, help="move cap per row for `flip`")
     a = p.parse_args(argv)
     ws = all_workloads()
     if a.what == "list":
@@ -112,6 +116,40 @@ def main(argv=None):
                     1 if a.fused else 0, ws_t.data_ptr(), ws_t.numel(), stream)
             t = _time(torch, lambda: call(lib.macaq_linear_w4a4, *args), flush, a.reps, a.warmup)
             print(f"{line} linear_w4a4 fused={int(a.fused)} {t * 1e6:.2f} us {2.0 * M * N * K / t / 1e12:.1f} TFLOP/s")
+    elif a.what == "flip":
+        from dataclasses import replace
+        xc = _bf16(torch, wl.draw_x(replace(L, M=a.calib, seed=L.seed + 100)), dev)
+        hws = torch.empty(lib.macaq_hessian_full_workspace_bytes(a.calib, K), dtype=torch.uint8, device=dev)
+        H = torch.empty((K, K), dtype=torch.float64, device=dev)
+        hargs = (xc.data_ptr(), a.calib, K, xc.stride(0), s.data_ptr(), H.data_ptr(), hws.data_ptr(), hws.numel(),
+                 stream)
+        t_h = _time(torch, lambda: call(lib.macaq_hessian_full, *hargs), flush, a.reps, a.warmup)
+        codes0 = pw.codes.clone()
+        fws = torch.empty(lib.macaq_flip_workspace_bytes(N, K), dtype=torch.uint8, device=dev)
+        moves = torch.empty(N, dtype=torch.int32, device=dev)
+        fargs = (W.data_ptr(), N, K, W.stride(0), s.data_ptr(), H.data_ptr(), pw.codes.data_ptr(),
+                 pw.scales.data_ptr(), a.rounds, moves.data_ptr(), fws.data_ptr(), fws.numel(), stream)
+
+        def refine():
+            call(lib.macaq_flip_refine, *fargs)
+
+        total = 0.0
+        for i in range(a.warmup + a.reps):
+            pw.codes.copy_(codes0)
+            flush.fill_(i & 0xFF)
+            flush.view(torch.int32).max()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            refine()
+            e1.record()
+            torch.cuda.synchronize()
+            if i >= a.warmup:
+                total += e0.elapsed_time(e1) * 1e-3
+        t_f = total / a.reps
+        mv = moves.float()
+        print(f"{line} hessian_full T={a.calib} {t_h * 1e6:.1f} us")
+        print(f"{line} flip_refine rounds<={a.rounds} {t_f * 1e6:.1f} us, moves per row mean "
+              f"{mv.mean().item():.1f} max {int(mv.max().item())}")
     else:
         from dataclasses import replace
         xc = _bf16(torch, wl.draw_x(replace(L, M=a.calib, seed=L.seed + 100)), dev)
