@@ -64,6 +64,8 @@ def lib():
             "macaq_hessian_full": (I, [P, I64, I64, I64, P, P, P, SZ, P]),
             "macaq_flip_workspace_bytes": (SZ, [I64, I64]),
             "macaq_flip_refine": (I, [P, I64, I64, I64, P, P, P, P, I, P, P, SZ, P]),
+            "macaq_grouped_linear_workspace_bytes": (SZ, [P, I64, I64]),
+            "macaq_grouped_linear_w4a4": (I, [P, I64, P, I64, P, P, I64, I, P, SZ, P]),
             "macaq_get_device_error": (I, []),
             "macaq_status_string": (ctypes.c_char_p, [I]),
             "macaq_version": (I, []),
@@ -228,6 +230,29 @@ def flip_refine(W, s, H, w, max_rounds=1 << 20, workspace=None):
                                  _stream_ptr(dev))
     _check(st, "macaq_flip_refine")
     return moves
+
+
+def grouped_linear(x, offsets, weights, out_dtype=None, y=None, workspace=None):
+    """MoE experts: rows offsets[g] .. offsets[g+1] - 1 of x go through weights[g]."""
+    torch = _torch()
+    _require(x, torch.bfloat16, "x")
+    G = len(weights)
+    if len(offsets) != G + 1:
+        raise ValueError("offsets must have len(weights) + 1 entries")
+    offs = (ctypes.c_int64 * (G + 1))(*[int(o) for o in offsets])
+    ws_structs = (MacaqWeight * G)(*[w.c_struct() for w in weights])
+    N, K = weights[0].N, weights[0].K
+    M = int(offsets[-1])
+    out_dtype = out_dtype or torch.bfloat16
+    dev = x.device
+    if y is None:
+        y = torch.empty((M, N), dtype=out_dtype, device=dev)
+    need = lib().macaq_grouped_linear_workspace_bytes(offs, G, K)
+    ws, ws_bytes = _workspace(need, dev, workspace)
+    st = lib().macaq_grouped_linear_w4a4(x.data_ptr(), x.stride(0), offs, G, ws_structs, y.data_ptr(), y.stride(0),
+                                         _out_code(y.dtype), ws.data_ptr(), ws_bytes, _stream_ptr(dev))
+    _check(st, "macaq_grouped_linear_w4a4")
+    return y
 
 
 def quant_act(x, inv_s, codes=None, scales=None):

@@ -45,6 +45,12 @@
 
 namespace macaq {
 
+struct GemmGroup {
+    int32_t unit_begin, rows, row_p, row_y;
+    const uint8_t* sf_q;
+    int64_t pad;
+};
+
 struct GemmParams {
     const uint8_t* sf_p;     // scale atoms of P
     const uint8_t* sf_q;     // scale atoms of Q
@@ -83,6 +89,14 @@ struct GemmParams {
     uint8_t* f_codes;                // [f_rows x f_K/2]
     uint8_t* f_scales;               // atom layout, 128-row slabs x f_kb_pad blocks
     int32_t f_rows, f_K, f_kb_pad;
+    // Grouped GEMM (groups > 0; prefill orientation, no split K): group g multiplies the
+    // g_rows[g] activation rows starting at P row g_row_p[g] (a multiple of 128: groups
+    // sit in whole scale slabs) by its own weight (tensor map g_tmaps[g], scale atoms
+    // g_sf_q[g]) and writes y rows g_row_y[g] ..; its units are g_unit_begin[g] ..
+    // g_unit_begin[g + 1] - 1, P tiles fastest.
+    int32_t groups;
+    const GemmGroup* g_desc;         // [groups]
+    const CUtensorMap* g_tmaps;      // [groups], 64-byte aligned
 };
 
 enum : int {
@@ -191,9 +205,38 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
 
 struct Unit {
     int tile, split, tp, tq, kt_begin, kt_end;
+    int p_row0;                    // first P row of the tile in the P tensor map
+    int out_row0;                  // output row of the tile's P row 0
+    int rows;                      // valid P rows from p_row0 on (the tile's group)
+    const CUtensorMap* tmap_q;     // Q tensor map of the tile
+    const uint8_t* sf_q;           // Q scale atoms of the tile
 };
 
-__device__ __forceinline__ Unit decode_unit(const GemmParams& p, int u) {
+__device__ __forceinline__ Unit decode_unit(const GemmParams& p, int u, const CUtensorMap* tmap_q) {
+    if (p.groups > 0) {
+        // the group whose units contain u: binary search over the unit offsets
+        int lo = 0, hi = p.groups - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (p.g_desc[mid].unit_begin <= u) lo = mid; else hi = mid - 1;
+        }
+        const GemmGroup gd = p.g_desc[lo];
+        const int tiles_p = (gd.rows + 127) >> 7;
+        const int lu = u - gd.unit_begin;
+        Unit x;
+        x.tile = u;
+        x.split = 0;
+        x.tp = lu % tiles_p;
+        x.tq = lu / tiles_p;
+        x.kt_begin = 0;
+        x.kt_end = p.k_tiles;
+        x.p_row0 = gd.row_p + x.tp * 128;
+        x.out_row0 = gd.row_y + x.tp * 128;
+        x.rows = gd.rows - x.tp * 128;
+        x.tmap_q = p.g_tmaps + lo;
+        x.sf_q = gd.sf_q;
+        return x;
+    }
     const int tile = u / p.splits;
     const int split = u - tile * p.splits;
     const int per_group = p.group_p * p.tiles_q;
@@ -207,12 +250,20 @@ __device__ __forceinline__ Unit decode_unit(const GemmParams& p, int u) {
     x.tq = r / gp;
     x.kt_begin = split * p.k_tiles_per_split;
     x.kt_end = min(p.k_tiles, x.kt_begin + p.k_tiles_per_split);
+    x.p_row0 = x.tp * 128;
+    x.out_row0 = x.tp * 128;
+    x.rows = p.p_rows - x.tp * 128;
+    x.tmap_q = tmap_q;
+    x.sf_q = p.sf_q;
     return x;
 }
 
+// Writes one chunk of output row `prow` (a P row; the output column of it when
+// transposed) if `valid`.
 template <int CW>
-__device__ __forceinline__ void store_chunk(const GemmParams& p, int prow, int q_base, const uint32_t (&r)[CW]) {
-    if (prow >= p.p_rows) return;
+__device__ __forceinline__ void store_chunk(const GemmParams& p, int prow, bool valid, int q_base,
+                                            const uint32_t (&r)[CW]) {
+    if (!valid) return;
     if (p.transpose_out) {
         // out[q, prow]: for each column the 32 lanes of the warp write consecutive prow
         if (p.atomic) {
@@ -416,7 +467,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         ptx::fence_mbar_init();
         ptx::fence_proxy_async_smem();
         ptx::prefetch_tensormap(&tmap_p);
-        ptx::prefetch_tensormap(&tmap_q);
+        if (p.groups == 0) ptx::prefetch_tensormap(&tmap_q);
         if (S::kStagingBytes > 0 && p.tma_store) ptx::prefetch_tensormap(&tmap_y);
     }
     if (warp == 1) {
@@ -441,18 +492,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         uint32_t issued_mask = 0, issued_phase = 0;
         const int q_slabs = (p.q_rows + 127) / 128;
         // Q side of one fill: codes tile and scale chunks
-        auto issue_q = [&](int st, int kt, int q0, int slab0, int nchunks) {
-            ptx::tma_load_2d(smem + L::kOffQ + st * S::kQTileBytes, &tmap_q, &full[st], kt * S::kBKBytes, q0);
+        auto issue_q = [&](const Unit& t, int st, int kt, int q0, int slab0, int nchunks) {
+            ptx::tma_load_2d(smem + L::kOffQ + st * S::kQTileBytes, t.tmap_q, &full[st], kt * S::kBKBytes, q0);
             for (int c = 0; c < nchunks; ++c)
                 ptx::bulk_load(smem + L::kOffSfQ + (st * S::kQChunks + c) * S::kSfChunkBytes,
-                               p.sf_q + ((int64_t)(slab0 + c) * p.kb4_pad + 2 * kt) * 512, S::kSfChunkBytes,
+                               t.sf_q + ((int64_t)(slab0 + c) * p.kb4_pad + 2 * kt) * 512, S::kSfChunkBytes,
                                &full[st]);
         };
         bool q_ready = !p.fused;
         int deferred = 0;                   // fills of the first unit still without their Q side
         for (int u = blockIdx.x; u < p.total_units; u += gridDim.x) {
             if (cta_aborted(abort)) break;
-            const Unit t = decode_unit(p, u);
+            const Unit t = decode_unit(p, u, &tmap_q);
             const int q0 = t.tq * BN;
             const int slab0 = q0 / 128;
             const int nchunks = min(S::kQChunks, q_slabs - slab0);
@@ -463,11 +514,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 if (leader) {
                     ptx::mbar_arrive_expect_tx(&full[stage], bytes);
                     ptx::tma_load_2d(smem + L::kOffP + stage * S::kPTileBytes, &tmap_p, &full[stage],
-                                     kt * S::kBKBytes, t.tp * S::kBM);
+                                     kt * S::kBKBytes, t.p_row0);
                     ptx::bulk_load(smem + L::kOffSfP + stage * S::kSfChunkBytes,
-                                   p.sf_p + ((int64_t)t.tp * p.kb4_pad + 2 * kt) * 512,
+                                   p.sf_p + ((int64_t)(t.p_row0 >> 7) * p.kb4_pad + 2 * kt) * 512,
                                    S::kSfChunkBytes, &full[stage]);
-                    if (q_ready) issue_q(stage, kt, q0, slab0, nchunks);
+                    if (q_ready) issue_q(t, stage, kt, q0, slab0, nchunks);
                 }
                 __syncwarp();
                 issued_mask |= 1u << stage;
@@ -482,7 +533,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     if (!__all_sync(0xffffffffu, fl)) { ok = false; break; }
                     ptx::fence_proxy_async_global();
                     if (leader)
-                        for (int d = 0; d < deferred; ++d) issue_q(d, t.kt_begin + d, q0, slab0, nchunks);
+                        for (int d = 0; d < deferred; ++d) issue_q(t, d, t.kt_begin + d, q0, slab0, nchunks);
                     __syncwarp();
                     q_ready = true;
                 }
@@ -515,7 +566,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         bool issued = false;
         for (int u = blockIdx.x; u < p.total_units; u += gridDim.x) {
             if (cta_aborted(abort)) break;
-            const Unit t = decode_unit(p, u);
+            const Unit t = decode_unit(p, u, &tmap_q);
             const uint32_t q_off = (uint32_t)((t.tq * BN) % 128) / 32;
             if ((q_off & 1) != 0 || q_off * 32 + (BN < 32 ? 32 : BN) > 128 * S::kQChunks) {
                 // never planned: a scale-factor column offset the MMA is not given
@@ -585,7 +636,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         uint32_t phase = 0;
         uint32_t kt_count = 0;
         for (int u = blockIdx.x; u < p.total_units && !*abort; u += gridDim.x) {
-            const Unit t = decode_unit(p, u);
+            const Unit t = decode_unit(p, u, &tmap_q);
             bool ok = true;
             for (int kt = t.kt_begin; kt < t.kt_end; ++kt, ++kt_count) {
                 // Every set waits for every fill, in order, even those it does not
@@ -647,10 +698,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             if (et == 0) st_release_u64(p.cta_flags + blockIdx.x, p.epoch);
         }
         for (int u = blockIdx.x; u < p.total_units && !*abort; u += gridDim.x) {
-            const Unit t = decode_unit(p, u);
+            const Unit t = decode_unit(p, u, &tmap_q);
             if (!wait_or_abort(&acc_full[acc], acc_phase, abort, p.err, kErrTimeoutEpilogue)) break;
             ptx::tc_fence_after();
-            const int prow = t.tp * S::kBM + quad * 32 + lane;
+            const int prow = t.out_row0 + quad * 32 + lane;      // output row (transposed: column)
+            const bool row_ok = quad * 32 + lane < t.rows;
             const uint32_t taddr = tmem + acc * S::kAccStride + ((uint32_t)(quad * 32) << 16);
             if (p.atomic && !zeroed) {
                 // once per kernel: every CTA has zeroed its slice of the accumulator
@@ -673,7 +725,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
                         for (int h = 0; h < 2; ++h) {
                             if (h >= boxes) break;
-                            const int bx = t.tq * BN + c * CW + 16 * h, by = t.tp * S::kBM + quad * 32;
+                            const int bx = t.tq * BN + c * CW + 16 * h, by = t.out_row0 + quad * 32;
                             if (bx >= p.q_rows || by >= p.p_rows) break;   // box wholly outside y
                             if (lane == 0) ptx::bulk_wait_group_read<0>();
                             __syncwarp();
@@ -704,7 +756,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         return;
                     }
                 }
-                store_chunk<CW>(p, prow, t.tq * BN + c * CW, r);
+                store_chunk<CW>(p, prow, row_ok, t.tq * BN + c * CW, r);
             };
 #pragma unroll 1
             for (int c = 0; c < NCH; ++c) {

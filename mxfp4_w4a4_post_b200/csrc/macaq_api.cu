@@ -10,6 +10,7 @@
 #include <cstring>
 #include <mutex>
 #include <numeric>
+#include <vector>
 
 #include "macaq.h"
 #include "flip_kernel.cuh"
@@ -607,6 +608,145 @@ macaq_status macaq_linear_w4a4_noalloc(const void* x_bf16, int64_t M, int64_t ld
         scratch = g_noalloc_ptr[dev];
     }
     return macaq_linear_w4a4(x_bf16, M, ldx, w, y, ldy, out, 0, scratch, MACAQ_NOALLOC_SCRATCH_BYTES, stream);
+}
+
+// ------------------------------------------------------------- grouped (MoE) ---
+
+namespace {
+
+// Padded row layout of the grouped activations: group g's rows start at the multiple of
+// 128 after the previous group's, so every group owns whole scale slabs.
+struct GroupedLayout {
+    int64_t rows_pad_total = 0;
+    size_t off_scales = 0, off_tmaps = 0, off_desc = 0, total = 0;
+};
+
+bool grouped_layout(const int64_t* offsets, int64_t G, int64_t K, GroupedLayout* L) {
+    if (!offsets || G < 1 || G > 4096 || K < 32 || K % 32 != 0) return false;
+    int64_t rows = 0;
+    for (int64_t g = 0; g < G; ++g) {
+        const int64_t m = offsets[g + 1] - offsets[g];
+        if (m < 0 || offsets[g] < 0) return false;
+        rows += round_up(m, 128);
+    }
+    if (rows > kMaxRows) return false;
+    L->rows_pad_total = rows;
+    const size_t codes = (size_t)round_up(std::max<int64_t>(rows, 128) * (K / 2), 256);
+    const size_t scales = (size_t)round_up(std::max<int64_t>(rows, 128) * round_up(K / 32, 8), 256);
+    L->off_scales = codes;
+    L->off_tmaps = codes + scales;
+    L->off_desc = L->off_tmaps + (size_t)round_up(G * (int64_t)sizeof(CUtensorMap), 256);
+    L->total = L->off_desc + (size_t)round_up(G * (int64_t)sizeof(GemmGroup), 256);
+    return true;
+}
+
+}  // namespace
+
+size_t macaq_grouped_linear_workspace_bytes(const int64_t* offsets, int64_t G, int64_t K) {
+    GroupedLayout L;
+    return grouped_layout(offsets, G, K, &L) ? L.total : 0;
+}
+
+macaq_status macaq_grouped_linear_w4a4(const void* x_bf16, int64_t ldx, const int64_t* offsets, int64_t G,
+                                       const macaq_weight* weights, void* y, int64_t ldy, macaq_out_dtype out,
+                                       void* workspace, size_t ws_bytes, macaq_stream stream) {
+    if (!x_bf16 || !offsets || !weights || !y) return MACAQ_ERR_INVALID_ARG;
+    GroupedLayout GL;
+    if (G < 1 || !weights[0].codes) return MACAQ_ERR_INVALID_ARG;
+    const int64_t N = weights[0].N, K = weights[0].K;
+    if (offsets[0] != 0) return MACAQ_ERR_INVALID_ARG;
+    if (!grouped_layout(offsets, G, K, &GL)) return MACAQ_ERR_INVALID_ARG;
+    const int64_t M = offsets[G];
+    if (M < 1) return MACAQ_ERR_INVALID_ARG;
+    for (int64_t g = 0; g < G; ++g) {
+        macaq_status st = check_weight(&weights[g]);
+        if (st != MACAQ_OK) return st;
+        if (weights[g].N != N || weights[g].K != K || !weights[g].inv_s) return MACAQ_ERR_INVALID_ARG;
+        if (!aligned16(weights[g].inv_s)) return MACAQ_ERR_MISALIGNED;
+    }
+    macaq_status st = check_gemm_args(M, &weights[0], y, ldy, out);
+    if (st != MACAQ_OK) return st;
+    st = check_quant_args(x_bf16, M, K, ldx, weights[0].inv_s, weights[0].codes, weights[0].scales);
+    if (st != MACAQ_OK) return st;
+    if (!workspace || ws_bytes < GL.total) return MACAQ_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255) != 0) return MACAQ_ERR_MISALIGNED;
+    DeviceInfo* dev = nullptr;
+    st = device_info(&dev);
+    if (st != MACAQ_OK) return st;
+    cudaStream_t cs = (cudaStream_t)stream;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    uint8_t* a_codes = ws;
+    uint8_t* a_scales = ws + GL.off_scales;
+    const int64_t kb_pad = round_up(K / 32, 8);
+
+    // the GEMM's group tables, copied from pageable host memory before any kernel is
+    // enqueued (such a copy first waits for the stream, then is staged before return)
+    const int bn = N <= 128 ? 128 : 192;
+    const int64_t tiles_q = cdiv(N, bn);
+    std::vector<CUtensorMap> maps((size_t)G);
+    std::vector<GemmGroup> desc((size_t)G);
+    int64_t units = 0;
+    int64_t row_p = 0;
+    for (int64_t g = 0; g < G; ++g) {
+        const int64_t m = offsets[g + 1] - offsets[g];
+        if (!encode_codes_map(&maps[g], weights[g].codes, N, K, bn)) return MACAQ_ERR_CUDA;
+        desc[g].unit_begin = (int32_t)units;
+        desc[g].rows = (int32_t)m;
+        desc[g].row_p = (int32_t)row_p;
+        desc[g].row_y = (int32_t)offsets[g];
+        desc[g].sf_q = weights[g].scales;
+        desc[g].pad = 0;
+        units += cdiv(m, 128) * tiles_q;
+        row_p += round_up(m, 128);
+    }
+    if (units > INT32_MAX) return MACAQ_ERR_UNSUPPORTED_SHAPE;
+    if (cudaMemcpyAsync(ws + GL.off_tmaps, maps.data(), maps.size() * sizeof(CUtensorMap), cudaMemcpyHostToDevice,
+                        cs) != cudaSuccess ||
+        cudaMemcpyAsync(ws + GL.off_desc, desc.data(), desc.size() * sizeof(GemmGroup), cudaMemcpyHostToDevice,
+                        cs) != cudaSuccess)
+        return MACAQ_ERR_CUDA;
+    // every group's rows through the activation transform with its own inv_s
+    row_p = 0;
+    for (int64_t g = 0; g < G; ++g) {
+        const int64_t m = offsets[g + 1] - offsets[g];
+        if (m > 0) {
+            st = launch_quant(static_cast<const uint16_t*>(x_bf16) + offsets[g] * ldx, m, K, ldx, weights[g].inv_s,
+                              a_codes + row_p * (K / 2), a_scales + row_p * kb_pad, nullptr, nullptr, cs);
+            if (st != MACAQ_OK) return st;
+        }
+        row_p += round_up(m, 128);
+    }
+
+    // the GEMM: one launch over every group's units
+    CUtensorMap mp, mq, my;
+    std::memset(&mq, 0, sizeof(mq));
+    std::memset(&my, 0, sizeof(my));
+    if (!encode_codes_map(&mp, a_codes, std::max<int64_t>(GL.rows_pad_total, 1), K, 128)) return MACAQ_ERR_CUDA;
+    GemmParams gp{};
+    gp.sf_p = a_scales;
+    gp.sf_q = weights[0].scales;
+    gp.out = y;
+    gp.ldo = ldy;
+    gp.p_rows = (int32_t)GL.rows_pad_total;
+    gp.q_rows = (int32_t)N;
+    gp.k_tiles = (int32_t)cdiv(K, 256);
+    gp.kb4_pad = (int32_t)(kb_pad / 4);
+    gp.tiles_p = 1;
+    gp.tiles_q = (int32_t)tiles_q;
+    gp.splits = 1;
+    gp.k_tiles_per_split = gp.k_tiles;
+    gp.total_units = (int32_t)units;
+    gp.group_p = 1;
+    gp.out_bf16 = out == MACAQ_OUT_BF16 ? 1 : 0;
+    const int64_t esz = out == MACAQ_OUT_BF16 ? 2 : 4;
+    gp.vec_ok = (aligned16(y) && (ldy * esz) % 16 == 0) ? 1 : 0;
+    gp.err = dev->err_ptr;
+    gp.groups = (int32_t)G;
+    gp.g_desc = reinterpret_cast<const GemmGroup*>(ws + GL.off_desc);
+    gp.g_tmaps = reinterpret_cast<const CUtensorMap*>(ws + GL.off_tmaps);
+    if (units == 0) return MACAQ_OK;
+    const int grid = (int)std::min<int64_t>(units, dev->num_sms);
+    return bn == 128 ? launch_gemm_bn<128, 6>(mp, mq, my, gp, grid, cs) : launch_gemm_bn<192, 5>(mp, mq, my, gp, grid, cs);
 }
 
 size_t macaq_hessian_bytes(int64_t K) {

@@ -4,6 +4,7 @@ the ncu captures that back them.
     python -m mxfp4_w4a4_post_b200.timing list
     python -m mxfp4_w4a4_post_b200.timing {quant,gemm,linear,hessian,flip} WORKLOAD [--reps R]
                                           [--warmup W] [--fused] [--calib T] [--rounds R]
+    python -m mxfp4_w4a4_post_b200.timing moe [--experts G] [--tokens T] [--n N] [--k K]
 
 Inputs are the workload's seeded synthetic tensors (workloads.py), resident on the
 device. Before every timed call L2 is flushed by a 256 MiB write and a read of the same
@@ -14,6 +15,9 @@ printed, one line per measured call:
     linear   macaq_linear_w4a4 (fused = 0, or 1 with --fused)
     hessian  macaq_hessian_blocks on T calibration rows (the workload's activation model
              with another seed) and macaq_prepare_weight_hessian on the weight
+    moe      macaq_grouped_linear_w4a4 on T tokens routed over G experts (seeded skewed
+             counts, tokens sorted by expert), against the same work as G separate
+             macaq_linear_w4a4 calls
     flip     macaq_hessian_full on T calibration rows, then macaq_flip_refine of the
              prepared weight (each timed call starts again from the round-to-nearest
              codes, restored before the flush); also prints the moves per row
@@ -55,20 +59,82 @@ def _time(torch, fn, flush, reps, warmup):
     return total / reps
 
 
+def moe(a):
+    import ctypes
+    import torch
+    import mxfp4_w4a4_post_b200 as mq
+    dev = torch.device("cuda", torch.cuda.current_device())
+    G, T, N, K = a.experts, a.tokens, a.n, a.k
+    rng = np.random.default_rng(5)
+    p = 1.0 / np.arange(1, G + 1) ** 1.2
+    counts = np.bincount(rng.choice(G, T, p=p / p.sum()), minlength=G)
+    offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int64)
+    base = wl.with_shape(wl.tiny_layer(), M=T, N=N, K=K)
+    x = _bf16(torch, wl.draw_x(base), dev)
+    pws = []
+    for g in range(G):
+        Lg = wl.with_shape(base, M=1, seed=300 + g)
+        pws.append(mq.prepare_weight(_bf16(torch, wl.draw_W(Lg), dev), torch.from_numpy(wl.draw_s(Lg)).to(dev)))
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    y = torch.empty((T, N), dtype=torch.bfloat16, device=dev)
+    lib = mq.lib()
+    stream = ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+    offs = (ctypes.c_int64 * (G + 1))(*offsets.tolist())
+    wts = (mq.MacaqWeight * G)(*[w.c_struct() for w in pws])
+    gws = torch.empty(lib.macaq_grouped_linear_workspace_bytes(offs, G, K), dtype=torch.uint8, device=dev)
+    gargs = (x.data_ptr(), x.stride(0), offs, G, wts, y.data_ptr(), y.stride(0), mq.OUT_BF16, gws.data_ptr(),
+             gws.numel(), stream)
+
+    def grouped():
+        st = lib.macaq_grouped_linear_w4a4(*gargs)
+        if st != 0:
+            raise mq.MacaqError(st, "macaq_grouped_linear_w4a4")
+
+    lws = torch.empty(max(mq.linear_workspace_bytes(int(c), N, K, torch.bfloat16) for c in counts if c),
+                      dtype=torch.uint8, device=dev)
+    cws = [w.c_struct() for w in pws]
+    calls = []
+    for g in range(G):
+        if counts[g]:
+            calls.append((x[offsets[g]:].data_ptr(), int(counts[g]), x.stride(0), ctypes.byref(cws[g]),
+                          y[offsets[g]:].data_ptr(), y.stride(0), mq.OUT_BF16, 0, lws.data_ptr(), lws.numel(),
+                          stream))
+
+    def separate():
+        for args in calls:
+            st = lib.macaq_linear_w4a4(*args)
+            if st != 0:
+                raise mq.MacaqError(st, "macaq_linear_w4a4")
+
+    t_g = _time(torch, grouped, flush, a.reps, a.warmup)
+    t_s = _time(torch, separate, flush, a.reps, a.warmup)
+    flops = 2.0 * T * N * K
+    print(f"moe G={G} tokens={T} N={N} K={K} counts={counts.tolist()}")
+    print(f"grouped_linear_w4a4 {t_g * 1e6:.1f} us {flops / t_g / 1e12:.1f} TFLOP/s; "
+          f"{G} separate linear_w4a4 calls {t_s * 1e6:.1f} us {flops / t_s / 1e12:.1f} TFLOP/s")
+    return 1 if mq.device_error() != 0 else 0
+
+
 def main(argv=None):
     p = argparse.ArgumentParser()
-    p.add_argument("what", choices=["list", "quant", "gemm", "linear", "hessian", "flip"])
+    p.add_argument("what", choices=["list", "quant", "gemm", "linear", "hessian", "flip", "moe"])
     p.add_argument("workload", nargs="?")
     p.add_argument("--reps", type=int, default=20)
     p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--fused", action="store_true")
     p.add_argument("--calib", type=int, default=2048, help="calibration rows for `hessian` and `flip`")
     p.add_argument("--rounds", type=int, default=256, help="move cap per row for `flip`")
+    p.add_argument("--experts", type=int, default=8)
+    p.add_argument("--tokens", type=int, default=4096)
+    p.add_argument("--n", type=int, default=2048)
+    p.add_argument("--k", type=int, default=4096)
     a = p.parse_args(argv)
     ws = all_workloads()
     if a.what == "list":
         print("\n".join(ws))
         return 0
+    if a.what == "moe":
+        return moe(a)
     if a.workload not in ws:
         p.error(f"unknown workload {a.workload!r}; see `list`")
     import torch
