@@ -300,6 +300,25 @@ macaq_status macaq_linear_w4a4_noalloc(const void* x_bf16, int64_t M, int64_t ld
  * read fails). */
 macaq_status macaq_get_device_error(void);
 
+/* Self-test of the bounded device waits (failure detection; the pages have no
+ * counterpart). Launches on `stream` a 2-CTA kernel that runs the GEMM kernel's own
+ * wait routines against waits that cannot succeed, then synchronises `stream` and
+ * copies the outcome into result[0..9] (host memory, caller-owned):
+ *   [0] wait on an mbarrier nothing arrives at, limit limit_us: 1 completed, 0 gave up
+ *   [1] a second wait in the same CTA, normal 2 s limit: 0 if it left on the CTA's
+ *       abort flag
+ *   [2] a wait on a barrier the warp completes itself: 1
+ *   [3] the CTA's recorded error code (1: producer-wait timeout)
+ *   [4] [5] time spent in waits [0] and [1], ns, by the device clock
+ *   [6] wait on a global flag that holds another epoch, limit limit_us: 0 gave up
+ *   [7] that CTA's recorded error code (5: split-K flag timeout)
+ *   [8] time spent in wait [6], ns
+ *   [9] wait on a flag that already holds the epoch: 1
+ * limit_us must be in [1, 1000000] (else MACAQ_ERR_INVALID_ARG). A kernel that gives
+ * up returns normally, so the context stays usable; the device error word read by
+ * macaq_get_device_error is not touched. MACAQ_ERR_CUDA if the launch or copy fails. */
+macaq_status macaq_selftest_wait_timeout(uint32_t limit_us, int64_t* result, macaq_stream stream);
+
 /* Static, human-readable name of a status code. */
 const char* macaq_status_string(macaq_status status);
 

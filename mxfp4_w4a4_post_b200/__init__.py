@@ -66,6 +66,7 @@ def lib():
             "macaq_flip_refine": (I, [P, I64, I64, I64, P, P, P, P, I, P, P, SZ, P]),
             "macaq_grouped_linear_workspace_bytes": (SZ, [P, I64, I64]),
             "macaq_grouped_linear_w4a4": (I, [P, I64, P, I64, P, P, I64, I, P, SZ, P]),
+            "macaq_selftest_wait_timeout": (I, [ctypes.c_uint32, ctypes.POINTER(I64), P]),
             "macaq_get_device_error": (I, []),
             "macaq_status_string": (ctypes.c_char_p, [I]),
             "macaq_version": (I, []),
@@ -319,6 +320,20 @@ def linear(x, w, out_dtype=None, y=None, workspace=None, fused=False):
                                  _out_code(y.dtype), 1 if fused else 0, ws.data_ptr(), ws_bytes, _stream_ptr(dev))
     _check(st, "macaq_linear_w4a4")
     return y
+
+
+def selftest_wait_timeout(limit_us=2000, device=None):
+    """Run the bounded-wait self-test kernel on the current stream; returns the ten
+    result words of macaq_selftest_wait_timeout as a dict."""
+    torch = _torch()
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    res = (ctypes.c_int64 * 10)()
+    with torch.cuda.device(dev):
+        _check(lib().macaq_selftest_wait_timeout(limit_us, res, _stream_ptr(dev)), "macaq_selftest_wait_timeout")
+    r = list(res)
+    return {"bar_timeout_ok": r[0], "bar_abort_ok": r[1], "bar_done_ok": r[2], "bar_err": r[3],
+            "bar_timeout_ns": r[4], "bar_abort_ns": r[5], "flag_timeout_ok": r[6], "flag_err": r[7],
+            "flag_timeout_ns": r[8], "flag_done_ok": r[9]}
 
 
 def device_error():

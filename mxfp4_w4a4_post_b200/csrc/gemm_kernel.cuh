@@ -163,28 +163,31 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
     return t;
 }
 
-__device__ __noinline__ bool wait_or_abort_slow(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                                int* err, int code);
+// Longest a kernel waits on one barrier or flag before it gives up.
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
-// Wait for `parity` on `bar`, giving up after ~2 s (or as soon as another role of the
-// CTA has given up). On give-up record `code`, raise the CTA abort flag, return false.
-// mbarrier.try_wait suspends the thread in hardware until the phase completes or a
-// short hardware time limit passes, so the loop just polls again; the wall clock and
+__device__ __noinline__ bool wait_or_abort_slow(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                                int* err, int code, uint64_t limit_ns);
+
+// Wait for `parity` on `bar`, giving up after limit_ns (or as soon as another role of
+// the CTA has given up). On give-up record `code`, raise the CTA abort flag, return
+// false. mbarrier.try_wait suspends the thread in hardware until the phase completes or
+// a short hardware time limit passes, so the loop just polls again; the wall clock and
 // the abort flag are read every 16 polls.
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                              int* err, int code) {
+                                              int* err, int code, uint64_t limit_ns = kWaitLimitNs) {
     if (ptx::mbar_try_wait(bar, parity)) return true;
-    return wait_or_abort_slow(bar, parity, abort, err, code);
+    return wait_or_abort_slow(bar, parity, abort, err, code, limit_ns);
 }
 
 __device__ __noinline__ bool wait_or_abort_slow(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                                int* err, int code) {
+                                                int* err, int code, uint64_t limit_ns) {
     const uint64_t t0 = global_timer_ns();
     for (uint32_t it = 1;; ++it) {
         if (ptx::mbar_try_wait(bar, parity)) return true;
         if ((it & 15) == 0) {
             if (*abort) return false;
-            if (global_timer_ns() - t0 > 2000000000ull) {
+            if (global_timer_ns() - t0 > limit_ns) {
                 atomicExch(err, code);
                 *abort = 1;
                 return false;
@@ -199,8 +202,8 @@ __device__ __forceinline__ bool cta_aborted(volatile int* abort) { return __any_
 // wait_or_abort by every lane of a warp, with a warp-uniform result: false if any lane
 // gave up.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort, int* err,
-                                          int code) {
-    return __all_sync(0xffffffffu, wait_or_abort(bar, parity, abort, err, code));
+                                          int code, uint64_t limit_ns = kWaitLimitNs) {
+    return __all_sync(0xffffffffu, wait_or_abort(bar, parity, abort, err, code, limit_ns));
 }
 
 struct Unit {
@@ -354,13 +357,13 @@ __device__ __forceinline__ void st_release_u64(unsigned long long* f, unsigned l
 // Wait (bounded, ~2 s) until *flag == epoch. On give-up record kErrTimeoutSplit, raise
 // the CTA abort flag and return false. Polls sleep briefly: the flag lives in L2.
 __device__ __noinline__ bool wait_split_flag(const unsigned long long* flag, unsigned long long epoch,
-                                             volatile int* abort, int* err) {
+                                             volatile int* abort, int* err, uint64_t limit_ns = kWaitLimitNs) {
     const uint64_t t0 = global_timer_ns();
     for (uint32_t it = 0;; ++it) {
         if (ld_acquire_u64(flag) == epoch) return true;
         if ((it & 15) == 15) {
             if (*abort) return false;
-            if (global_timer_ns() - t0 > 2000000000ull) {
+            if (global_timer_ns() - t0 > limit_ns) {
                 atomicExch(err, kErrTimeoutSplit);
                 *abort = 1;
                 return false;

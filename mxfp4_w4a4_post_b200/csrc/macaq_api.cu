@@ -17,6 +17,7 @@
 #include "gemm_kernel.cuh"
 #include "hessian_kernel.cuh"
 #include "quant_kernel.cuh"
+#include "selftest_kernel.cuh"
 
 namespace macaq {
 
@@ -864,6 +865,38 @@ macaq_status macaq_flip_refine(const void* W_bf16, int64_t N, int64_t K, int64_t
     FlipRoundParams fr{wv, w_codes, w_scales, H, G, moves, N, K, kb_pad, max_rounds};
     if (launch_pdl(flip_rounds_kernel, dim3((unsigned)N), dim3(kFlipThreads), smem, cs, fr) != cudaSuccess)
         return MACAQ_ERR_CUDA;
+    return MACAQ_OK;
+}
+
+}  // extern "C"
+
+namespace {
+// Results and flags of macaq_selftest_wait_timeout (the device error word is not used).
+__device__ long long g_selftest_out[macaq::kSelftestWords];
+__device__ unsigned long long g_selftest_flags[2];
+}  // namespace
+
+extern "C" {
+
+macaq_status macaq_selftest_wait_timeout(uint32_t limit_us, int64_t* result, macaq_stream stream) {
+    if (!result || limit_us < 1 || limit_us > 1000000) return MACAQ_ERR_INVALID_ARG;
+    DeviceInfo* dev = nullptr;
+    const macaq_status st = device_info(&dev);
+    if (st != MACAQ_OK) return st;
+    void* out = nullptr;
+    void* flags = nullptr;
+    if (cudaGetSymbolAddress(&out, g_selftest_out) != cudaSuccess ||
+        cudaGetSymbolAddress(&flags, g_selftest_flags) != cudaSuccess)
+        return MACAQ_ERR_CUDA;
+    wait_selftest_kernel<<<2, 96, 0, stream>>>((uint64_t)limit_us * 1000u,
+                                               static_cast<unsigned long long*>(flags),
+                                               static_cast<long long*>(out));
+    if (cudaGetLastError() != cudaSuccess) return MACAQ_ERR_CUDA;
+    long long host[kSelftestWords];
+    if (cudaMemcpyAsync(host, out, sizeof host, cudaMemcpyDeviceToHost, stream) != cudaSuccess ||
+        cudaStreamSynchronize(stream) != cudaSuccess)
+        return MACAQ_ERR_CUDA;
+    for (int i = 0; i < kSelftestWords; ++i) result[i] = host[i];
     return MACAQ_OK;
 }
 
