@@ -147,6 +147,47 @@ macaq_status launch_quant(const void* x, int64_t rows, int64_t K, int64_t ld, co
                : MACAQ_ERR_CUDA;
 }
 
+// One launch of the grouped quantiser over every expert's padded rows (G > 0 experts
+// with rows, table in device memory). Grid as launch_quant's; each warp then takes a
+// contiguous range of rows_per_warp padded rows of its column chunk.
+macaq_status launch_quant_grouped(const void* x, int64_t ld, int64_t K, const QuantGroup* table, int G,
+                                  int64_t rows_pad, uint8_t* codes, uint8_t* scales, cudaStream_t stream) {
+    DeviceInfo* dev = nullptr;
+    macaq_status st = device_info(&dev);
+    if (st != MACAQ_OK) return st;
+    if (G < 1 || rows_pad < 128) return MACAQ_ERR_INVALID_ARG;
+    GroupedQuantParams p{};
+    p.x = static_cast<const uint16_t*>(x);
+    p.codes = codes;
+    p.scales = scales;
+    p.groups = table;
+    p.G = G;
+    p.K = K;
+    p.ld = ld;
+    p.rows_pad = rows_pad;
+    p.kb_pad = round_up(K / 32, 8);
+    p.chunks_per_row = cdiv(p.kb_pad, 32);
+    const int64_t warps_per_cta = kQuantThreads / 32;
+    const int64_t unit = std::max<int64_t>(1, std::lcm<int64_t>(warps_per_cta, p.chunks_per_row));
+    const int64_t want = std::min<int64_t>((int64_t)dev->num_sms * 2 * warps_per_cta, rows_pad * p.chunks_per_row);
+    const int64_t nwarps = std::max<int64_t>(unit, want / unit * unit);
+    p.rows_per_warp = (int32_t)cdiv(rows_pad, nwarps / p.chunks_per_row);
+    const int blocks = (int)(nwarps / warps_per_cta);
+    static std::atomic<uint64_t> smem_set{0};
+    int devid = 0;
+    cudaGetDevice(&devid);
+    if (!(smem_set.load() & (1ull << (devid & 63)))) {
+        if (cudaFuncSetAttribute(quant_grouped_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kQuantSmemBytes) != cudaSuccess)
+            return MACAQ_ERR_CUDA;
+        smem_set.fetch_or(1ull << (devid & 63));
+    }
+    return launch_pdl(quant_grouped_kernel, dim3(blocks), dim3(kQuantThreads), kQuantSmemBytes, stream, p) ==
+                   cudaSuccess
+               ? MACAQ_OK
+               : MACAQ_ERR_CUDA;
+}
+
 macaq_status check_quant_args(const void* x, int64_t rows, int64_t K, int64_t ld, const void* mult,
                               const void* codes, const void* scales) {
     if (!x || !mult || !codes || !scales) return MACAQ_ERR_INVALID_ARG;
@@ -619,7 +660,7 @@ namespace {
 // 128 after the previous group's, so every group owns whole scale slabs.
 struct GroupedLayout {
     int64_t rows_pad_total = 0;
-    size_t off_scales = 0, off_tmaps = 0, off_desc = 0, total = 0;
+    size_t off_scales = 0, off_tmaps = 0, off_desc = 0, off_qtab = 0, total = 0;
 };
 
 bool grouped_layout(const int64_t* offsets, int64_t G, int64_t K, GroupedLayout* L) {
@@ -637,7 +678,8 @@ bool grouped_layout(const int64_t* offsets, int64_t G, int64_t K, GroupedLayout*
     L->off_scales = codes;
     L->off_tmaps = codes + scales;
     L->off_desc = L->off_tmaps + (size_t)round_up(G * (int64_t)sizeof(CUtensorMap), 256);
-    L->total = L->off_desc + (size_t)round_up(G * (int64_t)sizeof(GemmGroup), 256);
+    L->off_qtab = L->off_desc + (size_t)round_up(G * (int64_t)sizeof(GemmGroup), 256);
+    L->total = L->off_qtab + (size_t)round_up(G * (int64_t)sizeof(QuantGroup), 256);
     return true;
 }
 
@@ -686,10 +728,12 @@ macaq_status macaq_grouped_linear_w4a4(const void* x_bf16, int64_t ldx, const in
     const int64_t tiles_q = cdiv(N, bn);
     std::vector<CUtensorMap> maps((size_t)G);
     std::vector<GemmGroup> desc((size_t)G);
+    std::vector<QuantGroup> qtab;
     int64_t units = 0;
     int64_t row_p = 0;
     for (int64_t g = 0; g < G; ++g) {
         const int64_t m = offsets[g + 1] - offsets[g];
+        if (m > 0) qtab.push_back(QuantGroup{offsets[g], (int32_t)m, (int32_t)row_p, weights[g].inv_s});
         if (!encode_codes_map(&maps[g], weights[g].codes, N, K, bn)) return MACAQ_ERR_CUDA;
         desc[g].unit_begin = (int32_t)units;
         desc[g].rows = (int32_t)m;
@@ -704,19 +748,14 @@ macaq_status macaq_grouped_linear_w4a4(const void* x_bf16, int64_t ldx, const in
     if (cudaMemcpyAsync(ws + GL.off_tmaps, maps.data(), maps.size() * sizeof(CUtensorMap), cudaMemcpyHostToDevice,
                         cs) != cudaSuccess ||
         cudaMemcpyAsync(ws + GL.off_desc, desc.data(), desc.size() * sizeof(GemmGroup), cudaMemcpyHostToDevice,
+                        cs) != cudaSuccess ||
+        cudaMemcpyAsync(ws + GL.off_qtab, qtab.data(), qtab.size() * sizeof(QuantGroup), cudaMemcpyHostToDevice,
                         cs) != cudaSuccess)
         return MACAQ_ERR_CUDA;
-    // every group's rows through the activation transform with its own inv_s
-    row_p = 0;
-    for (int64_t g = 0; g < G; ++g) {
-        const int64_t m = offsets[g + 1] - offsets[g];
-        if (m > 0) {
-            st = launch_quant(static_cast<const uint16_t*>(x_bf16) + offsets[g] * ldx, m, K, ldx, weights[g].inv_s,
-                              a_codes + row_p * (K / 2), a_scales + row_p * kb_pad, nullptr, nullptr, cs);
-            if (st != MACAQ_OK) return st;
-        }
-        row_p += round_up(m, 128);
-    }
+    // every expert's rows through the activation transform with its own inv_s: one launch
+    st = launch_quant_grouped(x_bf16, ldx, K, reinterpret_cast<const QuantGroup*>(ws + GL.off_qtab),
+                              (int)qtab.size(), GL.rows_pad_total, a_codes, a_scales, cs);
+    if (st != MACAQ_OK) return st;
 
     // the GEMM: one launch over every group's units
     CUtensorMap mp, mq, my;

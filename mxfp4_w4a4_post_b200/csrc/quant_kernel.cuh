@@ -304,4 +304,167 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_rows_kernel(QuantParam
     cp_async_wait<0>();
 }
 
+// ---------------------------------------------------------------------------------
+// Grouped activation transform (MoE experts): one launch for every expert's rows.
+//
+// Expert g's rows x_row .. x_row + rows - 1 of x go through the transform with its own
+// multipliers and land at padded rows row_p .. row_p + rows - 1 of one grouped output,
+// each expert on a 128-row boundary; rows row_p + rows .. up to the next boundary are
+// padding (scale byte 0, codes not written). Only experts with rows > 0 are listed,
+// in increasing row_p. A warp keeps one column chunk and walks a contiguous range of
+// padded rows, so it changes expert (and reloads its 32 multipliers) at most a few
+// times. Per block the arithmetic is the same encode_block as quant_rows_kernel.
+
+struct QuantGroup {
+    int64_t x_row;        // first row of the expert in x
+    int32_t rows;         // its row count (> 0)
+    int32_t row_p;        // its first padded row in the grouped output (multiple of 128)
+    const float* mult;    // its multipliers [K]
+};
+
+struct GroupedQuantParams {
+    const uint16_t* x;    // bf16 bits, row stride ld
+    uint8_t* codes;       // [rows_pad x K/2]
+    uint8_t* scales;      // atom layout, rows_pad x kb_pad bytes
+    const QuantGroup* groups;
+    int32_t G;
+    int32_t rows_per_warp;
+    int64_t K, ld;
+    int64_t rows_pad;     // sum over experts of round_up(rows, 128)
+    int64_t kb_pad;
+    int64_t chunks_per_row;
+};
+
+// Index of the expert whose padded rows contain r (largest g with row_p <= r).
+__device__ __forceinline__ int find_group(const QuantGroup* t, int G, int r) {
+    int lo = 0, hi = G - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (t[mid].row_p <= r) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+}
+
+__global__ void __launch_bounds__(kQuantThreads, 2) quant_grouped_kernel(GroupedQuantParams p) {
+    extern __shared__ __align__(16) uint8_t qsmem[];
+    const uint32_t lane = threadIdx.x & 31;
+    const int gw = (int)((blockIdx.x * kQuantThreads + threadIdx.x) >> 5);
+    const int cpr = (int)p.chunks_per_row;
+    const int chunk = gw % cpr;
+    const int r_begin = (gw / cpr) * p.rows_per_warp;
+    const int r_end = min(r_begin + p.rows_per_warp, (int)p.rows_pad);
+    const int b = chunk * 32 + lane;
+    const bool col_live = b < (int)(p.K >> 5);
+    const int G = p.G;
+    const QuantGroup* tab = p.groups;
+
+    const uint32_t swz16 = ((lane >> 1) & 3) << 4;
+    uint32_t off[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) off[j] = (uint32_t)(16 * j) ^ swz16;
+    const uint32_t slot0 = (uint32_t)__cvta_generic_to_shared(qsmem) + threadIdx.x * 64;
+    const uint32_t slot_end = slot0 + kQuantStages * kQuantStageBytes;
+    const uint8_t* xbase = reinterpret_cast<const uint8_t*>(p.x);
+
+    ptx::griddep_wait();
+    ptx::griddep_launch_dependents();
+    if (r_begin >= r_end) return;                        // warp-uniform
+
+    // copy side: the expert of the row being fetched
+    int irow = r_begin;
+    int ig = find_group(tab, G, r_begin);
+    int i_rowp = tab[ig].row_p, i_rows = tab[ig].rows;
+    int64_t i_xrow = tab[ig].x_row;
+    int i_next = ig + 1 < G ? tab[ig + 1].row_p : INT32_MAX;
+    uint32_t islot = slot0;
+    auto issue = [&]() {
+        if (irow >= i_next) {
+            ++ig;
+            i_rowp = tab[ig].row_p;
+            i_rows = tab[ig].rows;
+            i_xrow = tab[ig].x_row;
+            i_next = ig + 1 < G ? tab[ig + 1].row_p : INT32_MAX;
+        }
+        const int local = irow - i_rowp;
+        const bool v = col_live && irow < r_end && local < i_rows;
+        const uint8_t* src = v ? xbase + (i_xrow + local) * p.ld * 2 + (int64_t)b * 64 : xbase;
+        const uint32_t n = v ? 16u : 0u;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) cp_async_16(islot + off[j], src + 16 * j, n);
+        cp_async_commit();
+        ++irow;
+        islot += kQuantStageBytes;
+        if (islot == slot_end) islot = slot0;
+    };
+#pragma unroll
+    for (int s = 0; s < kQuantStages - 1; ++s) issue();
+
+    // compute side: the expert of the row being encoded, and its multipliers
+    int cg = find_group(tab, G, r_begin);
+    int c_rowp = tab[cg].row_p, c_rows = tab[cg].rows;
+    int c_next = cg + 1 < G ? tab[cg + 1].row_p : INT32_MAX;
+    uint64_t mult[16];
+    auto load_mult = [&]() {
+        if (col_live) {
+            const float4* mp = reinterpret_cast<const float4*>(tab[cg].mult + b * 32);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const float4 m = __ldg(mp + i);
+                mult[2 * i] = pk(m.x, m.y);
+                mult[2 * i + 1] = pk(m.z, m.w);
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) mult[i] = 0;
+        }
+    };
+    load_mult();
+
+    uint32_t rslot = slot0;
+    const int64_t half_k = p.K >> 1;
+    const int kb_pad = (int)p.kb_pad;
+    const int64_t kb4 = p.kb_pad >> 2;
+    for (int row = r_begin; row < r_end; ++row) {
+        issue();
+        if (row >= c_next) {
+            ++cg;
+            c_rowp = tab[cg].row_p;
+            c_rows = tab[cg].rows;
+            c_next = cg + 1 < G ? tab[cg + 1].row_p : INT32_MAX;
+            load_mult();
+        }
+        cp_async_wait<kQuantStages - 1>();
+
+        uint64_t T[16];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            uint32_t w[4];
+            asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
+                         : "r"(rslot + off[j]));
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                T[4 * j + q] = mul2(pk(__uint_as_float(w[q] << 16), __uint_as_float(w[q] & 0xFFFF0000u)),
+                                    mult[4 * j + q]);
+        }
+        rslot += kQuantStageBytes;
+        if (rslot == slot_end) rslot = slot0;
+
+        uint32_t packed[4];
+        const uint32_t sbyte = encode_block(T, packed);
+
+        if (col_live && row - c_rowp < c_rows)
+            *reinterpret_cast<uint4*>(p.codes + (int64_t)row * half_k + (int64_t)b * 16) =
+                make_uint4(packed[0], packed[1], packed[2], packed[3]);
+        const uint32_t s1 = __shfl_down_sync(0xffffffffu, sbyte, 1);
+        const uint32_t s2 = __shfl_down_sync(0xffffffffu, sbyte, 2);
+        const uint32_t s3 = __shfl_down_sync(0xffffffffu, sbyte, 3);
+        if ((lane & 3) == 0 && b < kb_pad) {
+            const int64_t o = ((int64_t)(row >> 7) * kb4 + (b >> 2)) * 512 + (row & 31) * 16 + ((row >> 5) & 3) * 4;
+            *reinterpret_cast<uint32_t*>(p.scales + o) = sbyte | (s1 << 8) | (s2 << 16) | (s3 << 24);
+        }
+    }
+    cp_async_wait<0>();
+}
+
 }  // namespace macaq
