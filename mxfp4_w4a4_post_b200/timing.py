@@ -5,6 +5,7 @@ the ncu captures that back them.
     python -m mxfp4_w4a4_post_b200.timing {quant,gemm,linear,hessian,flip} WORKLOAD [--reps R]
                                           [--warmup W] [--fused] [--calib T] [--rounds R]
     python -m mxfp4_w4a4_post_b200.timing moe [--experts G] [--tokens T] [--n N] [--k K]
+    python -m mxfp4_w4a4_post_b200.timing tp WORKLOAD [--world G]
 
 Inputs are the workload's seeded synthetic tensors (workloads.py), resident on the
 device. Before every timed call L2 is flushed by a 256 MiB write and a read of the same
@@ -18,6 +19,8 @@ printed, one line per measured call:
     moe      macaq_grouped_linear_w4a4 on T tokens routed over G experts (seeded skewed
              counts, tokens sorted by expert), against the same work as G separate
              macaq_linear_w4a4 calls
+    tp       one rank's macaq_linear_w4a4 under a column- and a row-parallel cut into G
+             pieces (the collective that follows needs several GPUs and is not timed)
     flip     macaq_hessian_full on T calibration rows, then macaq_flip_refine of the
              prepared weight (each timed call starts again from the round-to-nearest
              codes, restored before the flush); also prints the moves per row
@@ -115,9 +118,55 @@ def moe(a):
     return 1 if mq.device_error() != 0 else 0
 
 
+def tp(a, L):
+    """One rank's layer call under column- and row-parallel cuts of the workload's weight
+    into `--world` pieces (the rank with the largest piece), with the bytes its single
+    collective would move; the collective itself needs more than one GPU."""
+    import ctypes
+    import torch
+    import mxfp4_w4a4_post_b200 as mq
+    from .tensor_parallel import split_k, split_range
+    dev = torch.device("cuda", torch.cuda.current_device())
+    M, N, K, g = L.M, L.N, L.K, a.world
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    x = _bf16(torch, wl.draw_x(L), dev)
+    W, s = _bf16(torch, wl.draw_W(L), dev), torch.from_numpy(wl.draw_s(L)).to(dev)
+    lib = mq.lib()
+    stream = ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+    print(f"{L.name} M={M} N={N} K={K} world={g}")
+    for cut in ("column", "row"):
+        if cut == "column":
+            n0, n1 = split_range(N, g, 0)
+            pw = mq.prepare_weight(W[n0:n1], s)
+            xs, out, Nl, Kl = x, torch.bfloat16, n1 - n0, K
+            coll = f"all-gather {M * N * 2 / 1e6:.1f} MB bf16"
+        else:
+            k0, k1 = split_k(K, g, 0)
+            pw = mq.prepare_weight(W[:, k0:k1], s[k0:k1].contiguous())
+            xs, out, Nl, Kl = x[:, k0:k1], torch.float32, N, k1 - k0
+            coll = f"all-reduce {M * N * 4 / 1e6:.1f} MB fp32"
+        y = torch.empty((M, Nl), dtype=out, device=dev)
+        oc = mq.OUT_BF16 if out == torch.bfloat16 else mq.OUT_F32
+        ws = torch.empty(max(256, mq.linear_workspace_bytes(M, Nl, Kl, out)), dtype=torch.uint8, device=dev)
+        cw = pw.c_struct()
+        args = (xs.data_ptr(), M, xs.stride(0), ctypes.byref(cw), y.data_ptr(), y.stride(0), oc, 0,
+                ws.data_ptr(), ws.numel(), stream)
+
+        def run():
+            st = lib.macaq_linear_w4a4(*args)
+            if st != 0:
+                raise mq.MacaqError(st, "macaq_linear_w4a4")
+
+        t = _time(torch, run, flush, a.reps, a.warmup)
+        flops = 2.0 * M * Nl * Kl
+        print(f"{cut}-parallel rank 0 of {g}: linear_w4a4 {M}x{Nl}x{Kl} {t * 1e6:.1f} us "
+              f"{flops / t / 1e12:.1f} TFLOP/s; then {coll}")
+    return 1 if mq.device_error() != 0 else 0
+
+
 def main(argv=None):
     p = argparse.ArgumentParser()
-    p.add_argument("what", choices=["list", "quant", "gemm", "linear", "hessian", "flip", "moe"])
+    p.add_argument("what", choices=["list", "quant", "gemm", "linear", "hessian", "flip", "moe", "tp"])
     p.add_argument("workload", nargs="?")
     p.add_argument("--reps", type=int, default=20)
     p.add_argument("--warmup", type=int, default=3)
@@ -128,6 +177,7 @@ def main(argv=None):
     p.add_argument("--tokens", type=int, default=4096)
     p.add_argument("--n", type=int, default=2048)
     p.add_argument("--k", type=int, default=4096)
+    p.add_argument("--world", type=int, default=8, help="tensor-parallel pieces for `tp`")
     a = p.parse_args(argv)
     ws = all_workloads()
     if a.what == "list":
@@ -137,9 +187,11 @@ def main(argv=None):
         return moe(a)
     if a.workload not in ws:
         p.error(f"unknown workload {a.workload!r}; see `list`")
+    L = ws[a.workload]
+    if a.what == "tp":
+        return tp(a, L)
     import torch
     import mxfp4_w4a4_post_b200 as mq
-    L = ws[a.workload]
     dev = torch.device("cuda", torch.cuda.current_device())
     M, N, K = L.M, L.N, L.K
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
