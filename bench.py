@@ -77,6 +77,9 @@ def parse_args(argv=None):
     p.add_argument("--workload", default=DEFAULT_WORKLOAD)
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--oracle-table", action="store_true",
+                   help="time the oracle on the host cores per config (single-threaded and OpenMP) "
+                        "and print one JSON line per config and mode; uses no GPU")
     p.add_argument("--sample-rows", type=int, default=None,
                    help="oracle sample size in rows of x (default: 128 for the CPU baseline of the GPU arm; "
                         "for --impl reference, as many rows per step, up to 16, as keep the run within ~150 s)")
@@ -458,9 +461,83 @@ def run_reference(args):
     return result
 
 
+def oracle_configs():
+    """(label, workloads, GEMM rows per workload: None = all rows) of the oracle table."""
+    from mxfp4_w4a4_post_b200 import workloads as wl
+    return [
+        ("C1", [wl.tiny_layer()], None),
+        ("C2", [wl.llama3_8b_gate_up_prefill()], 256),
+        ("C3", [wl.qwen3_32b_up_decode(b) for b in (1, 8, 16, 64)], None),
+        ("C4", [wl.qwen3_32b_down_prefill()], 256),
+        ("C5", wl.qwen3_32b_layer_decode(256), None),
+    ]
+
+
+def oracle_table(args):
+    """The oracle on the host cores, per config, single-threaded and with OpenMP over
+    rows: full quantisation of x and preparation of W, and the fp64 GEMM over all rows
+    (C1, C3, C5) or over 256 seeded sampled rows of x (C2, C4; the single-threaded run
+    of C5 also samples, 64 rows per linear). One JSON line per config and mode; GEMM
+    throughput in MAC/s with the full-size time extrapolated from it."""
+    import oracle
+    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+    rows_out = []
+    for label, layers, gemm_rows in oracle_configs():
+        inputs = []
+        for L in layers:
+            x, W, s = wl_draw(L)
+            inputs.append((L, x, W, s))
+        for omp in (False, True):
+            oracle.set_openmp(omp)
+            t_q = t_g = 0.0
+            elems = macs = macs_full = 0
+            sampled = False
+            for L, x, W, s in inputs:
+                t0 = time.perf_counter()
+                wc, ws, inv = oracle.prepare_weight(W, s)
+                ac, as_ = oracle.quant_rows(x, inv)
+                t_q += time.perf_counter() - t0
+                elems += L.M * L.K + L.N * L.K
+                r = gemm_rows
+                if r is None and not omp and label == "C5":
+                    r = 64
+                if r is not None and r < L.M:
+                    sampled = True
+                    idx = np.sort(np.random.default_rng(0).choice(L.M, r, replace=False)).astype(np.int64)
+                else:
+                    idx = None
+                t0 = time.perf_counter()
+                oracle.gemm_fp64(ac, as_, wc, ws, L.K, rows=idx)
+                t_g += time.perf_counter() - t0
+                n = L.M if idx is None else len(idx)
+                macs += n * L.N * L.K
+                macs_full += L.M * L.N * L.K
+            mac_s = macs / t_g
+            line = {
+                "oracle_table": label, "mode": "openmp" if omp else "single-thread",
+                "threads": cores if omp else 1, "host_cores": cores,
+                "workloads": [L.name for L, *_ in inputs],
+                "quantise_s": t_q, "quantise_elems": elems, "quantise_melem_per_s": elems / t_q / 1e6,
+                "gemm_s": t_g, "gemm_macs": macs, "gemm_mac_per_s": mac_s,
+                "gemm_rows": "sampled" if sampled else "all",
+                "gemm_full_s_extrapolated" if sampled else "gemm_full_s": macs_full / mac_s,
+            }
+            print(json.dumps(line), flush=True)
+            rows_out.append(line)
+    oracle.set_openmp(False)
+    return rows_out
+
+
+def wl_draw(L):
+    from mxfp4_w4a4_post_b200 import workloads as wl
+    return wl.draw_x(L), wl.draw_W(L), wl.draw_s(L)
+
+
 def main(argv=None):
     args = parse_args(argv)
-    if args.impl == "reference":
+    if args.oracle_table:
+        oracle_table(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)

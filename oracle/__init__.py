@@ -14,13 +14,22 @@ import numpy as np
 
 from . import build_oracle
 
-_lib = None
+_libs = {}
+_openmp = False
+
+
+def set_openmp(flag):
+    """Route every call below to the OpenMP build of the oracle (row loops on all host
+    cores, same results) or back to the single-threaded one (the default). Used only to
+    time the oracle."""
+    global _openmp
+    _openmp = bool(flag)
 
 
 def lib():
-    global _lib
-    if _lib is None:
-        path = build_oracle.build()
+    key = "omp" if _openmp else "serial"
+    if key not in _libs:
+        path = build_oracle.build_omp() if _openmp else build_oracle.build()
         L = ctypes.CDLL(path)
         P = ctypes.c_void_p
         I64 = ctypes.c_int64
@@ -78,8 +87,8 @@ def lib():
         L.oracle_flip_refine_row.restype = ctypes.c_int
         L.oracle_flip_refine.argtypes = [P, I64, I64, I64, P, P, P, P, ctypes.c_int, P]
         L.oracle_flip_refine.restype = None
-        _lib = L
-    return _lib
+        _libs[key] = L
+    return _libs[key]
 
 
 def _p(a):
@@ -320,9 +329,10 @@ class use_library:
         self.path = path
 
     def __enter__(self):
-        global _lib
-        lib()  # make sure the default build exists and its signatures are known
-        self._saved = _lib
+        global _openmp
+        self._saved_mode = _openmp
+        _openmp = False
+        self._saved = lib()  # the default build, whose signatures are known
         L = ctypes.CDLL(self.path)
         for name in dir(self._saved):
             if name.startswith("oracle_"):
@@ -330,10 +340,11 @@ class use_library:
                 f = getattr(L, name)
                 f.argtypes = f_src.argtypes
                 f.restype = f_src.restype
-        _lib = L
+        _libs["serial"] = L
         return L
 
     def __exit__(self, *exc):
-        global _lib
-        _lib = self._saved
+        global _openmp
+        _libs["serial"] = self._saved
+        _openmp = self._saved_mode
         return False

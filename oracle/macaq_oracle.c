@@ -6,6 +6,11 @@
  *
  * Only tests/, __graft_entry__.smoke() and bench.py's CPU-baseline leg may use this.
  *
+ * Rows are independent in quant_rows, dequant_rows and gemm_fp64; their row loops
+ * carry OpenMP pragmas so that a second build (-fopenmp) can time the oracle on all
+ * host cores. The default build ignores the pragmas; either way every row is computed
+ * by the same scalar code in the same order, so the results are identical.
+ *
  * Sources, by page and section:
  *  - Layer identity y = xW^T rewritten with an online per-channel scale and block
  *    Hadamard on the activation, inverse folded into the weight: zicq.com English
@@ -164,6 +169,7 @@ static void quant_block(const float v[32], uint8_t* codes16, uint8_t* scale) {
 void oracle_quant_rows(const uint16_t* x, int64_t rows, int64_t K, int64_t ld,
                        const float* mult, uint8_t* codes, uint8_t* scales) {
     int64_t Kb = K / 32;
+#pragma omp parallel for schedule(static)
     for (int64_t r = 0; r < rows; ++r) {
         for (int64_t b = 0; b < Kb; ++b) {
             float v[32];
@@ -224,6 +230,7 @@ void oracle_unswizzle_scales(const uint8_t* atom, int64_t rows, int64_t K, uint8
 void oracle_dequant_rows(const uint8_t* codes, const uint8_t* scales, int64_t rows, int64_t K,
                          double* out) {
     int64_t Kb = K / 32;
+#pragma omp parallel for schedule(static)
     for (int64_t r = 0; r < rows; ++r) {
         for (int64_t k = 0; k < K; ++k) {
             uint8_t byte = codes[r * (K / 2) + k / 2];
@@ -239,26 +246,28 @@ void oracle_gemm_fp64(const uint8_t* a_codes, const uint8_t* a_scales, int64_t M
                       const int64_t* rows, int64_t n_rows, double* y) {
     (void)M;
     double* wdec = (double*)malloc(sizeof(double) * (size_t)(N * K));
-    double* adec = (double*)malloc(sizeof(double) * (size_t)K);
-    if (!wdec || !adec) {
-        free(wdec);
-        free(adec);
-        return;
-    }
+    if (!wdec) return;
     oracle_dequant_rows(w_codes, w_scales, N, K, wdec);
     int64_t count = rows ? n_rows : M;
-    for (int64_t i = 0; i < count; ++i) {
-        int64_t m = rows ? rows[i] : i;
-        oracle_dequant_rows(a_codes + m * (K / 2), a_scales + m * (K / 32), 1, K, adec);
-        for (int64_t n = 0; n < N; ++n) {
-            double acc = 0.0;
-            const double* wr = wdec + n * K;
-            for (int64_t k = 0; k < K; ++k) acc += adec[k] * wr[k];
-            y[i * N + n] = acc;
+#pragma omp parallel
+    {
+        /* one decoded activation row per thread (one in all without OpenMP) */
+        double* adec = (double*)malloc(sizeof(double) * (size_t)K);
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t i = 0; i < count; ++i) {
+            if (!adec) continue;
+            int64_t m = rows ? rows[i] : i;
+            oracle_dequant_rows(a_codes + m * (K / 2), a_scales + m * (K / 32), 1, K, adec);
+            for (int64_t n = 0; n < N; ++n) {
+                double acc = 0.0;
+                const double* wr = wdec + n * K;
+                for (int64_t k = 0; k < K; ++k) acc += adec[k] * wr[k];
+                y[i * N + n] = acc;
+            }
         }
+        free(adec);
     }
     free(wdec);
-    free(adec);
 }
 
 /* ------------------------------------------------ exact algebra (fp64) ----- */
