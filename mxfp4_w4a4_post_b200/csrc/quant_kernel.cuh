@@ -174,7 +174,12 @@ __device__ __forceinline__ uint32_t encode_block(uint64_t (&T)[16], uint32_t (&p
 }
 
 constexpr int kQuantThreads = 256;
-constexpr int kQuantStages = 4;
+// Two stages: one row in flight while the current one is encoded. Deeper prefetch
+// puts more rows in the first burst of requests that all warps issue at once, and a
+// warp's first row then arrives later (every warp waits on its oldest copy, which the
+// memory system does not serve first); one row ahead already keeps HBM busy in the
+// steady state with 16 warps per SM.
+constexpr int kQuantStages = 2;
 constexpr uint32_t kQuantStageBytes = kQuantThreads * 64;
 constexpr int kQuantSmemBytes = kQuantStages * kQuantStageBytes;
 
