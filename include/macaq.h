@@ -163,15 +163,17 @@ macaq_status macaq_linear_w4a4(const void* x_bf16, int64_t M, int64_t ldx, const
  * MACaQ targets MoE models and a grouped matmul kernel, openai-hub.com article): the
  * tokens arrive sorted by expert; expert g owns rows offsets[g] .. offsets[g+1] - 1 of x
  * and y and its own prepared weight weights[g] (own s, so its own online transform).
- * Each group goes through the activation transform with weights[g].inv_s, then one GEMM
- * launch covers every group's tiles (prefill orientation, 128- or 192-wide weight tiles).
+ * One quantiser launch puts every group's rows through the activation transform with
+ * its own weights[g].inv_s, then one GEMM launch covers every group's tiles (prefill
+ * orientation, 128- or 192-wide weight tiles).
  *   offsets   host [G + 1], offsets[0] == 0, non-decreasing (empty groups allowed)
  *   weights   host [G], all with the same N and K
  *   x_bf16    device bf16 [offsets[G] x K], row stride ldx; y device [offsets[G] x N]
  *   workspace >= macaq_grouped_linear_workspace_bytes(offsets, G, K), 256-byte aligned:
- *             activation codes and scales with every group padded to 128 rows, and the
- *             per-group tables of the GEMM (copied from host memory on `stream`; the
- *             call waits for the stream's earlier work before that copy)
+ *             activation codes and scales with every group padded to 128 rows, the
+ *             per-group tables of the GEMM and the quantiser's table of non-empty groups
+ *             (copied from pageable host memory on `stream`: such a copy waits for the
+ *             stream's earlier work)
  * G <= 4096. */
 size_t macaq_grouped_linear_workspace_bytes(const int64_t* offsets, int64_t G, int64_t K);
 macaq_status macaq_grouped_linear_w4a4(const void* x_bf16, int64_t ldx, const int64_t* offsets, int64_t G,
