@@ -157,6 +157,31 @@ macaq_status macaq_linear_w4a4(const void* x_bf16, int64_t M, int64_t ldx, const
                                void* y, int64_t ldy, macaq_out_dtype out, int fused,
                                void* workspace, size_t ws_bytes, macaq_stream stream);
 
+/* ------------------------------- gathered output (column-parallel layers) ----- */
+
+/* macaq_linear_w4a4 for one rank of a column-parallel layer (the pages have no
+ * tensor parallelism; the cut follows from the layer being row-wise in W', whose
+ * quantisation is row by row): the GEMM's epilogue writes this rank's y columns
+ * straight into each of n_dest full-width outputs (every rank's y, when the caller maps
+ * the other GPUs' buffers into this process), so no separate all-gather is needed.
+ *   dest      host [n_dest] device addresses: dest[d] is the address of row 0, column
+ *             n0 of destination d (n0 = this rank's first output column); each
+ *             destination has row stride ldy elements (ldy >= w->N) and room for M rows
+ *             of w->N columns from there; aligned to the element size. Memory of another
+ *             GPU must be accessible from this device (peer access or an IPC mapping).
+ *   n_dest    1 .. 64
+ *   workspace >= macaq_linear_gather_workspace_bytes(M, N, K, out), 256-byte aligned:
+ *             macaq_linear_w4a4's workspace, then the destination table (copied from
+ *             host memory on `stream`: the copy waits for the stream's earlier work)
+ * Every destination receives the same values that macaq_linear_w4a4 (fused = 0) would
+ * write to y, except that K is never split. Completion of the writes into another
+ * GPU's memory is ordered for that GPU only by the caller (for example a barrier on
+ * both streams after the call). */
+size_t macaq_linear_gather_workspace_bytes(int64_t M, int64_t N, int64_t K, macaq_out_dtype out);
+macaq_status macaq_linear_w4a4_gather(const void* x_bf16, int64_t M, int64_t ldx, const macaq_weight* w,
+                                      const uint64_t* dest, int n_dest, int64_t ldy, macaq_out_dtype out,
+                                      void* workspace, size_t ws_bytes, macaq_stream stream);
+
 /* --------------------------------------------- grouped layer (MoE experts) ----- */
 
 /* The layer for the routed experts of a mixture-of-experts block (the pages' remark that

@@ -66,6 +66,8 @@ def lib():
             "macaq_flip_refine": (I, [P, I64, I64, I64, P, P, P, P, I, P, P, SZ, P]),
             "macaq_grouped_linear_workspace_bytes": (SZ, [P, I64, I64]),
             "macaq_grouped_linear_w4a4": (I, [P, I64, P, I64, P, P, I64, I, P, SZ, P]),
+            "macaq_linear_gather_workspace_bytes": (SZ, [I64, I64, I64, I]),
+            "macaq_linear_w4a4_gather": (I, [P, I64, I64, ctypes.POINTER(MacaqWeight), P, I, I64, I, P, SZ, P]),
             "macaq_selftest_wait_timeout": (I, [ctypes.c_uint32, ctypes.POINTER(I64), P]),
             "macaq_get_device_error": (I, []),
             "macaq_status_string": (ctypes.c_char_p, [I]),
@@ -320,6 +322,32 @@ def linear(x, w, out_dtype=None, y=None, workspace=None, fused=False):
                                  _out_code(y.dtype), 1 if fused else 0, ws.data_ptr(), ws_bytes, _stream_ptr(dev))
     _check(st, "macaq_linear_w4a4")
     return y
+
+
+def linear_gather(x, w, dests, workspace=None):
+    """The layer for one rank of a column-parallel cut, written into several outputs:
+    dests are CUDA tensors [M, w.N] of one dtype (bf16 or fp32), each a column slice of a
+    full-width y (unit column stride, one common row stride), all reachable from x's
+    device. Every one receives this rank's columns of y."""
+    torch = _torch()
+    _require(x, torch.bfloat16, "x")
+    M, K = x.shape
+    if K != w.K:
+        raise ValueError(f"x has K={K}, weight has K={w.K}")
+    if not dests:
+        raise ValueError("no destinations")
+    dt, ld = dests[0].dtype, dests[0].stride(0)
+    for d in dests:
+        if tuple(d.shape) != (M, w.N) or d.dtype != dt or d.stride(0) != ld or d.stride(1) != 1:
+            raise ValueError("destinations must be [M, N] slices with one dtype and row stride")
+    addrs = (ctypes.c_uint64 * len(dests))(*[d.data_ptr() for d in dests])
+    need = lib().macaq_linear_gather_workspace_bytes(M, w.N, K, _out_code(dt))
+    ws, ws_bytes = _workspace(need, x.device, workspace)
+    cw = w.c_struct()
+    st = lib().macaq_linear_w4a4_gather(x.data_ptr(), M, x.stride(0), ctypes.byref(cw), addrs, len(dests), ld,
+                                        _out_code(dt), ws.data_ptr(), ws_bytes, _stream_ptr(x.device))
+    _check(st, "macaq_linear_w4a4_gather")
+    return dests
 
 
 def selftest_wait_timeout(limit_us=2000, device=None):

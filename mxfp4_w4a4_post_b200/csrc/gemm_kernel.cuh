@@ -97,6 +97,12 @@ struct GemmParams {
     int32_t groups;
     const GemmGroup* g_desc;         // [groups]
     const CUtensorMap* g_tmaps;      // [groups], 64-byte aligned
+    // Gathered output (column-parallel layers; the kernel's GATHER instantiation): every
+    // output element goes to each of dest[0 .. n_dest - 1] (device addresses of the
+    // destinations' first column for this weight, the same row stride ldo) instead of to
+    // out, with direct stores (no TMA store, no split K).
+    int32_t n_dest;
+    const unsigned long long* dest;  // [n_dest], device memory
 };
 
 enum : int {
@@ -264,27 +270,27 @@ __device__ __forceinline__ Unit decode_unit(const GemmParams& p, int u, const CU
 // Writes one chunk of output row `prow` (a P row; the output column of it when
 // transposed) if `valid`.
 template <int CW>
-__device__ __forceinline__ void store_chunk(const GemmParams& p, int prow, bool valid, int q_base,
+__device__ __forceinline__ void store_chunk(const GemmParams& p, void* out, int prow, bool valid, int q_base,
                                             const uint32_t (&r)[CW]) {
     if (!valid) return;
     if (p.transpose_out) {
         // out[q, prow]: for each column the 32 lanes of the warp write consecutive prow
         if (p.atomic) {
-            float* o = reinterpret_cast<float*>(p.out);
+            float* o = reinterpret_cast<float*>(out);
 #pragma unroll
             for (int j = 0; j < CW; ++j) {
                 const int q = q_base + j;
                 if (q < p.q_rows) atomicAdd(o + (int64_t)q * p.ldo + prow, __uint_as_float(r[j]));
             }
         } else if (p.out_bf16) {
-            __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(p.out);
+            __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(out);
 #pragma unroll
             for (int j = 0; j < CW; ++j) {
                 const int q = q_base + j;
                 if (q < p.q_rows) o[(int64_t)q * p.ldo + prow] = __float2bfloat16_rn(__uint_as_float(r[j]));
             }
         } else {
-            float* o = reinterpret_cast<float*>(p.out);
+            float* o = reinterpret_cast<float*>(out);
 #pragma unroll
             for (int j = 0; j < CW; ++j) {
                 const int q = q_base + j;
@@ -295,7 +301,7 @@ __device__ __forceinline__ void store_chunk(const GemmParams& p, int prow, bool 
     }
     const bool full = q_base + CW <= p.q_rows && p.vec_ok;
     if (p.atomic) {
-        float* o = reinterpret_cast<float*>(p.out) + (int64_t)prow * p.ldo + q_base;
+        float* o = reinterpret_cast<float*>(out) + (int64_t)prow * p.ldo + q_base;
         if (full) {
 #pragma unroll
             for (int j = 0; j < CW; j += 4)
@@ -308,7 +314,7 @@ __device__ __forceinline__ void store_chunk(const GemmParams& p, int prow, bool 
                 if (q_base + j < p.q_rows) atomicAdd(o + j, __uint_as_float(r[j]));
         }
     } else if (p.out_bf16) {
-        __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(p.out) + (int64_t)prow * p.ldo + q_base;
+        __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(out) + (int64_t)prow * p.ldo + q_base;
         if (full) {
 #pragma unroll
             for (int j = 0; j < CW; j += 8) {
@@ -329,7 +335,7 @@ __device__ __forceinline__ void store_chunk(const GemmParams& p, int prow, bool 
                 if (q_base + j < p.q_rows) o[j] = __float2bfloat16_rn(__uint_as_float(r[j]));
         }
     } else {
-        float* o = reinterpret_cast<float*>(p.out) + (int64_t)prow * p.ldo + q_base;
+        float* o = reinterpret_cast<float*>(out) + (int64_t)prow * p.ldo + q_base;
         if (full) {
 #pragma unroll
             for (int j = 0; j < CW; j += 4)
@@ -433,7 +439,9 @@ __device__ __forceinline__ void fused_quant_share(const GemmParams& p, int et) {
 constexpr int kSfWarpSets = 2;                                // scale-writer sets
 constexpr int kGemmThreads = 32 * (6 + 4 * kSfWarpSets);
 
-template <int BN, int STAGES>
+// GATHER: the output goes to p.dest[0 .. p.n_dest - 1] (a separate instantiation, so
+// that the ordinary kernels keep their registers).
+template <int BN, int STAGES, bool GATHER = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_mxf4_kernel(const __grid_constant__ CUtensorMap tmap_p, const __grid_constant__ CUtensorMap tmap_q,
                      const __grid_constant__ CUtensorMap tmap_y, const GemmParams p) {
@@ -717,6 +725,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             }
             // write chunk c of y from registers: staged TMA store or direct stores
             auto emit = [&](int c, uint32_t (&r)[CW]) {
+                if constexpr (GATHER) {
+                    for (int d = 0; d < p.n_dest; ++d)
+                        store_chunk<CW>(p, reinterpret_cast<void*>(p.dest[d]), prow, row_ok, t.tq * BN + c * CW, r);
+                    return;
+                }
                 if constexpr (S::kStagingBytes > 0) {
                     if (via_tma) {
                         // Stage this warp's box of 32 rows x 64 bytes in shared memory in the
@@ -759,7 +772,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         return;
                     }
                 }
-                store_chunk<CW>(p, prow, row_ok, t.tq * BN + c * CW, r);
+                store_chunk<CW>(p, p.out, prow, row_ok, t.tq * BN + c * CW, r);
             };
 #pragma unroll 1
             for (int c = 0; c < NCH; ++c) {

@@ -83,6 +83,7 @@ inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 // Limits that keep every index inside 32 bits where the kernels use int.
 constexpr int64_t kMaxRows = (int64_t)1 << 30;
 constexpr int64_t kMaxK = (int64_t)1 << 24;
+constexpr int kMaxGatherDest = 64;                 // destinations of a gathered output
 constexpr int64_t kMaxFlipK = 8192;     // Flip-Refinement keeps a row's gradient in shared memory
 
 // --------------------------------------------------------------------- quant ---
@@ -332,7 +333,7 @@ bool encode_out_map(CUtensorMap* map, void* y, int64_t M, int64_t N, int64_t ldy
     return r == CUDA_SUCCESS;
 }
 
-template <int BN, int STAGES>
+template <int BN, int STAGES, bool GATHER = false>
 macaq_status launch_gemm_bn(const CUtensorMap& mp, const CUtensorMap& mq, const CUtensorMap& my,
                             const GemmParams& gp, int grid, cudaStream_t stream) {
     using L = GemmSmem<BN, STAGES>;
@@ -342,12 +343,12 @@ macaq_status launch_gemm_bn(const CUtensorMap& mp, const CUtensorMap& mq, const 
     cudaGetDevice(&dev);
     const uint64_t bit = 1ull << (dev & 63);
     if (!(configured_mask.load() & bit)) {
-        if (cudaFuncSetAttribute(gemm_mxf4_kernel<BN, STAGES>,
+        if (cudaFuncSetAttribute(gemm_mxf4_kernel<BN, STAGES, GATHER>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc) != cudaSuccess)
             return MACAQ_ERR_CUDA;
         configured_mask.fetch_or(bit);
     }
-    return launch_pdl(gemm_mxf4_kernel<BN, STAGES>, dim3(grid), dim3(kGemmThreads), L::kAlloc, stream, mp, mq, my,
+    return launch_pdl(gemm_mxf4_kernel<BN, STAGES, GATHER>, dim3(grid), dim3(kGemmThreads), L::kAlloc, stream, mp, mq, my,
                       gp) ==
                    cudaSuccess
                ? MACAQ_OK
@@ -407,14 +408,30 @@ constexpr size_t kFusedFlagBytes = 8192;                 // up to 1024 CTAs
 // transform as its own kernel, which uses every thread of the GPU for it.
 constexpr int64_t kFusedMaxRows = 128;
 
+// Output written to several destinations (the gathered output of a column-parallel
+// layer): a device table of destination addresses, and whether all of them allow
+// 16-byte vector stores.
+struct GatherOut {
+    const unsigned long long* dest;
+    int n;
+    bool vec_ok;
+};
+
 macaq_status run_gemm(const uint8_t* a_codes, const uint8_t* a_scales, int64_t M,
                       const macaq_weight* w, void* y, int64_t ldy, macaq_out_dtype out,
-                      void* workspace, size_t ws_bytes, cudaStream_t stream, const FusedAct* fa = nullptr) {
+                      void* workspace, size_t ws_bytes, cudaStream_t stream, const FusedAct* fa = nullptr,
+                      const GatherOut* go = nullptr) {
     DeviceInfo* dev = nullptr;
     macaq_status st = device_info(&dev);
     if (st != MACAQ_OK) return st;
     const int64_t N = w->N, K = w->K;
-    const GemmPlan g = plan_gemm(M, N, K, dev->num_sms);
+    GemmPlan g = plan_gemm(M, N, K, dev->num_sms);
+    if (go && g.splits > 1) {
+        // a gathered output is written by the GEMM's own epilogue: no split K
+        g.splits = 1;
+        g.kps = g.k_tiles;
+        g.grid = (int)std::min<int64_t>((int64_t)g.tiles_p * g.tiles_q, dev->num_sms);
+    }
     const size_t need = gemm_workspace(M, N, K, dev->num_sms);
     if (need > 0 && (workspace == nullptr || ws_bytes < need)) return MACAQ_ERR_WORKSPACE;
     if (need > 0 && (reinterpret_cast<uintptr_t>(workspace) & 255) != 0) return MACAQ_ERR_MISALIGNED;
@@ -464,6 +481,12 @@ macaq_status run_gemm(const uint8_t* a_codes, const uint8_t* a_scales, int64_t M
         gp.vec_ok = y_vec;
         // wide row-major tiles store through TMA (an aligned output is all it needs)
         gp.tma_store = (!g.swap && g.bn >= 128 && gp.vec_ok) ? 1 : 0;
+        if (go) {
+            gp.n_dest = go->n;
+            gp.dest = go->dest;
+            gp.vec_ok = go->vec_ok ? 1 : 0;
+            gp.tma_store = 0;
+        }
     }
     int grid = g.grid;
     if (fa) {
@@ -487,6 +510,16 @@ macaq_status run_gemm(const uint8_t* a_codes, const uint8_t* a_scales, int64_t M
     std::memset(&my, 0, sizeof(my));
     if (gp.tma_store && !encode_out_map(&my, y, M, N, ldy, out == MACAQ_OUT_BF16)) return MACAQ_ERR_CUDA;
 
+    if (go) {
+        switch (g.bn) {
+            case 16: st = launch_gemm_bn<16, 8, true>(mp, mq, my, gp, grid, stream); break;
+            case 32: st = launch_gemm_bn<32, 8, true>(mp, mq, my, gp, grid, stream); break;
+            case 64: st = launch_gemm_bn<64, 8, true>(mp, mq, my, gp, grid, stream); break;
+            case 128: st = launch_gemm_bn<128, 6, true>(mp, mq, my, gp, grid, stream); break;
+            default: st = launch_gemm_bn<192, 5, true>(mp, mq, my, gp, grid, stream); break;
+        }
+        return st;
+    }
     switch (g.bn) {
         case 16: st = launch_gemm_bn<16, 8>(mp, mq, my, gp, grid, stream); break;
         case 32: st = launch_gemm_bn<32, 8>(mp, mq, my, gp, grid, stream); break;
@@ -495,7 +528,8 @@ macaq_status run_gemm(const uint8_t* a_codes, const uint8_t* a_scales, int64_t M
         default: st = launch_gemm_bn<192, 5>(mp, mq, my, gp, grid, stream); break;
     }
     if (st != MACAQ_OK || g.splits == 1) return st;
-    // split K (planned only for M <= 65535): one grid row per output row
+    // split K (planned only for M <= 65535, never with a gathered output): one grid row
+    // per output row
     const dim3 fgrid((unsigned)cdiv(cdiv(N, 4), 256), (unsigned)M);
     if (launch_pdl(finalize_kernel, fgrid, dim3(256), 0, stream, static_cast<const float*>(workspace), acc_ld(N),
                    (int)N, y, ldy, out == MACAQ_OUT_BF16 ? 1 : 0, y_vec) != cudaSuccess)
@@ -611,6 +645,44 @@ macaq_status macaq_linear_w4a4(const void* x_bf16, int64_t M, int64_t ldx, const
     st = launch_quant(x_bf16, M, w->K, ldx, w->inv_s, a_codes, a_scales, nullptr, nullptr, (cudaStream_t)stream);
     if (st != MACAQ_OK) return st;
     return run_gemm(a_codes, a_scales, M, w, y, ldy, out, ws + off_gemm, ws_bytes - off_gemm, (cudaStream_t)stream);
+}
+
+size_t macaq_linear_gather_workspace_bytes(int64_t M, int64_t N, int64_t K, macaq_out_dtype out) {
+    const size_t lin = macaq_linear_workspace_bytes(M, N, K, out);
+    return lin == 0 ? 0 : lin + (size_t)round_up(kMaxGatherDest * 8, 256);
+}
+
+macaq_status macaq_linear_w4a4_gather(const void* x_bf16, int64_t M, int64_t ldx, const macaq_weight* w,
+                                      const uint64_t* dest, int n_dest, int64_t ldy, macaq_out_dtype out,
+                                      void* workspace, size_t ws_bytes, macaq_stream stream) {
+    if (!dest || n_dest < 1 || n_dest > kMaxGatherDest) return MACAQ_ERR_INVALID_ARG;
+    const uintptr_t esz = out == MACAQ_OUT_BF16 ? 2 : 4;
+    bool vec = (ldy * (int64_t)esz) % 16 == 0;
+    for (int d = 0; d < n_dest; ++d) {
+        macaq_status st = check_gemm_args(M, w, reinterpret_cast<const void*>(dest[d]), ldy, out);
+        if (st != MACAQ_OK) return st;
+        vec = vec && (dest[d] & 15) == 0;
+    }
+    if (!w->inv_s) return MACAQ_ERR_INVALID_ARG;
+    macaq_status st = check_quant_args(x_bf16, M, w->K, ldx, w->inv_s, w->codes, w->scales);
+    if (st != MACAQ_OK) return st;
+    size_t off_scales, off_flags, off_gemm;
+    const size_t lin = linear_ws_parts(M, w->N, w->K, out, &off_scales, &off_flags, &off_gemm);
+    const size_t need = macaq_linear_gather_workspace_bytes(M, w->N, w->K, out);
+    if (!workspace || ws_bytes < need) return MACAQ_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255) != 0) return MACAQ_ERR_MISALIGNED;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    // the destination table goes after the layer's own workspace (a copy from pageable
+    // host memory waits for the stream's earlier work)
+    unsigned long long* table = reinterpret_cast<unsigned long long*>(ws + lin);
+    if (cudaMemcpyAsync(table, dest, (size_t)n_dest * 8, cudaMemcpyHostToDevice, (cudaStream_t)stream) !=
+        cudaSuccess)
+        return MACAQ_ERR_CUDA;
+    st = launch_quant(x_bf16, M, w->K, ldx, w->inv_s, ws, ws + off_scales, nullptr, nullptr, (cudaStream_t)stream);
+    if (st != MACAQ_OK) return st;
+    const GatherOut go{table, n_dest, vec};
+    return run_gemm(ws, ws + off_scales, M, w, nullptr, ldy, out, ws + off_gemm, lin - off_gemm,
+                    (cudaStream_t)stream, nullptr, &go);
 }
 
 }  // extern "C"

@@ -14,8 +14,14 @@ Two shardings of y = x W^T, W [N, K]:
 
 All arithmetic runs in the library's kernels through the package's binding; this module
 cuts the weight, picks each rank's slice of x and issues the one collective. The
-per-rank operations are an object with `prepare(W, s)` and `linear(x, w, out_dtype)`;
-the default is the CUDA binding.
+per-rank operations are an object with `prepare(W, s)`, `linear(x, w, out_dtype)` and
+`linear_gather(x, w, dests)`; the default is the CUDA binding.
+
+The column cut can also skip the collective: `ColumnParallelW4A4.forward_into` hands
+the GEMM every rank's full-width y (as this process sees it: its own buffer and the
+other GPUs' buffers mapped into it), and the GEMM's epilogue writes this rank's columns
+into all of them (`macaq_linear_w4a4_gather`). The caller orders the writes with the
+readers (for example a barrier on every rank's stream afterwards).
 """
 from dataclasses import dataclass
 
@@ -55,6 +61,10 @@ class CudaOps:
         import mxfp4_w4a4_post_b200 as mq
         return mq.linear(x, w, out_dtype=out_dtype)
 
+    def linear_gather(self, x, w, dests):
+        import mxfp4_w4a4_post_b200 as mq
+        return mq.linear_gather(x, w, dests)
+
 
 def _dist():
     import torch.distributed as dist
@@ -83,6 +93,10 @@ class ColumnParallelW4A4:
     weight: object          # the ops' prepared weight of W[n0:n1], or None for an empty shard
     group: object = None
     ops: object = None
+
+    def __post_init__(self):
+        if self.ops is None:
+            self.ops = CudaOps()
 
     @classmethod
     def from_full(cls, W, s, group=None, ops=None):
@@ -115,6 +129,15 @@ class ColumnParallelW4A4:
         _dist().all_gather(parts, buf.contiguous(), group=self.group)
         return torch.cat([p[:, :hi - lo] for p, (lo, hi) in zip(parts, widths)], dim=1)
 
+    def forward_into(self, x, ys):
+        """x [M, K] (replicated); ys: full-width outputs [M, N] (one dtype, unit column
+        stride, one common row stride), typically every rank's y as mapped into this
+        process. Writes this rank's columns n0 .. n1 - 1 of y into each of them with one
+        layer call and no collective; returns ys."""
+        if self.weight is not None:
+            self.ops.linear_gather(x, self.weight, [y[:, self.n0:self.n1] for y in ys])
+        return ys
+
 
 @dataclass
 class RowParallelW4A4:
@@ -126,6 +149,10 @@ class RowParallelW4A4:
     weight: object          # the ops' prepared weight of W[:, k0:k1] with s[k0:k1], or None
     group: object = None
     ops: object = None
+
+    def __post_init__(self):
+        if self.ops is None:
+            self.ops = CudaOps()
 
     @classmethod
     def from_full(cls, W, s, group=None, ops=None):

@@ -88,3 +88,13 @@ def test_validation_rejects_bad_arguments(L):
     assert L.macaq_selftest_wait_timeout(0, res, None) == 1
     assert L.macaq_selftest_wait_timeout(1000001, res, None) == 1
     assert L.macaq_selftest_wait_timeout(100, None, None) == 1
+    # gathered output: no destinations, too many, a misaligned one
+    d_ok = (ctypes.c_uint64 * 2)(0x2000, 0x3000)
+    d_mis = (ctypes.c_uint64 * 1)(0x2002)
+    d_many = (ctypes.c_uint64 * 65)(*([0x2000] * 65))
+    assert L.macaq_linear_w4a4_gather(a, 4, 256, ctypes.byref(w), None, 1, 128, 0, a, 1 << 20, None) == 1
+    assert L.macaq_linear_w4a4_gather(a, 4, 256, ctypes.byref(w), d_ok, 0, 128, 0, a, 1 << 20, None) == 1
+    assert L.macaq_linear_w4a4_gather(a, 4, 256, ctypes.byref(w), d_many, 65, 128, 0, a, 1 << 20, None) == 1
+    assert L.macaq_linear_w4a4_gather(a, 4, 256, ctypes.byref(w), d_mis, 1, 128, 0, a, 1 << 20, None) == 2
+    assert L.macaq_linear_w4a4_gather(a, 4, 256, ctypes.byref(w), d_ok, 2, 64, 0, a, 1 << 20, None) == 1  # ldy < N
+    assert L.macaq_linear_gather_workspace_bytes(4, 128, 256, 0) == L.macaq_linear_workspace_bytes(4, 128, 256, 0) + 512

@@ -62,6 +62,12 @@ class OracleOps:
         y = oracle.gemm_fp64(ac, as_, codes, scales, xn.shape[1])
         return _torch().from_numpy(y).to(out_dtype)
 
+    def linear_gather(self, x, w, dests):
+        y = self.linear(x, w, dests[0].dtype)
+        for d in dests:
+            d.copy_(y)
+        return dests
+
 
 def _torch():
     import torch
@@ -135,3 +141,26 @@ def test_two_rank_column_and_row_parallel(shape):
             assert wrow is None
     # both ranks hold the same joined result
     assert np.array_equal(res[0][3], res[1][3]) and np.array_equal(res[0][5], res[1][5])
+
+
+def test_gathered_column_cut_host_logic():
+    """forward_into: each rank's shard writes its columns into every full-width output;
+    two shards emulated in one process, three outputs, joined without a collective."""
+    import torch
+    import oracle
+    from mxfp4_w4a4_post_b200 import workloads as wl
+    from mxfp4_w4a4_post_b200.tensor_parallel import ColumnParallelW4A4
+    M, N, K = 6, 70, 96
+    L = wl.with_shape(wl.tiny_layer(), M=M, N=N, K=K)
+    x, W, s = _bf16(wl.draw_x(L)), _bf16(wl.draw_W(L)), torch.from_numpy(wl.draw_s(L))
+    ops = OracleOps()
+    ys = [torch.full((M, N), float("nan")) for _ in range(3)]
+    for rank in range(2):
+        n0, n1 = split_range(N, 2, rank)
+        shard = ColumnParallelW4A4(N, K, n0, n1, ops.prepare(W[n0:n1], s), None, ops)
+        shard.forward_into(x, ys)
+    wc, ws, winv = oracle.prepare_weight(wl.draw_W(L), wl.draw_s(L))
+    ac, as_ = oracle.quant_rows(wl.draw_x(L), winv)
+    ref = oracle.gemm_fp64(ac, as_, wc, ws, K).astype(np.float32)
+    for y in ys:
+        assert np.array_equal(y.numpy(), ref)

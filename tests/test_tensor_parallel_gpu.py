@@ -10,7 +10,7 @@ import numpy as np
 import pytest
 
 import oracle
-from helpers import assert_gemm_close, bf16_dev, f32_dev, host
+from helpers import assert_bf16_matches_f32, assert_gemm_close, bf16_dev, f32_dev, host
 from mxfp4_w4a4_post_b200 import workloads as wl
 from mxfp4_w4a4_post_b200.tensor_parallel import split_k, split_range
 
@@ -104,4 +104,59 @@ def test_module_with_nccl_one_rank(mq):
         torch.cuda.synchronize()
     finally:
         dist.destroy_process_group()
+    assert mq.device_error() == 0
+
+
+# (M, N, K, shards): prefill tiles, decode (swapped) tiles, and a shape for which the
+# ordinary layer splits K (the gathered output never does)
+GATHER_CASES = [(200, 520, 1024, 2), (5, 300, 512, 3), (16, 256, 16384, 2)]
+
+
+@pytest.mark.parametrize("M,N,K,shards", GATHER_CASES)
+@pytest.mark.parametrize("dt", ["f32", "bf16"])
+def test_gathered_column_cut(mq, M, N, K, shards, dt):
+    """Every shard writes its columns straight into two full-width outputs (local
+    buffers standing in for two ranks' y; no rank waits on another): both equal the
+    oracle's unsharded layer, and their pad columns and the guard bytes around them
+    are untouched."""
+    import torch
+    from mxfp4_w4a4_post_b200.tensor_parallel import ColumnParallelW4A4
+    dtype = torch.float32 if dt == "f32" else torch.bfloat16
+    L, x, W, s = layer(M, N, K)
+    xd, Wd, sd = bf16_dev(x), bf16_dev(W), f32_dev(s)
+    ld, guard = N + 8, 4096
+    esz = 4 if dt == "f32" else 2
+    raws = [torch.full((2 * guard + M * ld * esz,), 0xA5, dtype=torch.uint8, device="cuda") for _ in range(2)]
+    ys = [r[guard:guard + M * ld * esz].view(dtype).view(M, ld)[:, :N] for r in raws]
+    shard_out = []
+    for r in range(shards):
+        n0, n1 = split_range(N, shards, r)
+        w = mq.prepare_weight(Wd[n0:n1], sd)
+        ColumnParallelW4A4(N, K, n0, n1, w).forward_into(xd, ys)
+        shard_out.append((n0, n1, w))
+    torch.cuda.synchronize()
+    for raw in raws:
+        b = host(raw)
+        assert (b[:guard] == 0xA5).all() and (b[-guard:] == 0xA5).all(), "guard bytes changed"
+        full = b[guard:-guard].view(np.uint16 if esz == 2 else np.uint32).reshape(M, ld)
+        assert (full[:, N:].view(np.uint8) == 0xA5).all(), "pad columns changed"
+    y0, y1 = host(ys[0].float()), host(ys[1].float())
+    assert np.array_equal(y0, y1)
+    wc, ws, winv = oracle.prepare_weight(W, s)
+    ac, as_ = oracle.quant_rows(x, winv)
+    ref = oracle.gemm_fp64(ac, as_, wc, ws, K)
+    if dt == "f32":
+        assert_gemm_close(y0, ref, f"gathered column cut {M}x{N}x{K}")
+    # each shard's columns equal the ordinary layer's output for that shard whenever
+    # that one does not split K (same tiles, same MMAs, another store path)
+    for n0, n1, w in shard_out:
+        y_lin = mq.linear(xd, w, out_dtype=dtype)
+        if mq.gemm_workspace_bytes(M, n1 - n0, K, dtype) == 0:
+            assert torch.equal(ys[0][:, n0:n1], y_lin), (n0, n1)
+        else:
+            y32 = mq.linear(xd, w, out_dtype=torch.float32)
+            if dt == "f32":
+                assert_gemm_close(host(ys[0][:, n0:n1]), host(y32).astype(np.float64), "split shard")
+            else:
+                assert_bf16_matches_f32(ys[0][:, n0:n1], y32, "split shard")
     assert mq.device_error() == 0
