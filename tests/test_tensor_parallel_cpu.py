@@ -1,4 +1,4 @@
-"""Host logic of the tensor-parallel layers on CPU: two gloo ranks cut the weight
+"""Host logic of the tensor-parallel layers on CPU: two or three gloo ranks cut the weight
 (columns, or K on MX-block boundaries), run each rank's share with the oracle as the
 per-rank operations, and join the results with the module's own all-gather /
 all-reduce. The joined y must equal the oracle's unsharded layer (exactly for the
@@ -102,11 +102,11 @@ def _worker(rank, world, port, shape, q):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("shape", [(5, 70, 160), (3, 1, 32), (130, 64, 96)])
-def test_two_rank_column_and_row_parallel(shape):
+@pytest.mark.parametrize("world,shape", [(2, (5, 70, 160)), (2, (3, 1, 32)), (2, (130, 64, 96)),
+                                         (3, (7, 70, 160)), (3, (4, 2, 64))])
+def test_multi_rank_column_and_row_parallel(world, shape):
     import oracle
     from mxfp4_w4a4_post_b200 import workloads as wl
-    world = 2
     port = _free_port()
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
@@ -139,8 +139,9 @@ def test_two_rank_column_and_row_parallel(shape):
             assert np.array_equal(inv.view(np.uint32), winv[k0:k1].view(np.uint32))
         else:
             assert wrow is None
-    # both ranks hold the same joined result
-    assert np.array_equal(res[0][3], res[1][3]) and np.array_equal(res[0][5], res[1][5])
+    # every rank holds the same joined result
+    for r in res[1:]:
+        assert np.array_equal(res[0][3], r[3]) and np.array_equal(res[0][5], r[5])
 
 
 def test_gathered_column_cut_host_logic():
