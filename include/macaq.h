@@ -15,10 +15,15 @@
  *
  * Conventions shared by every entry point:
  *  - Pointers marked "device" are CUDA device pointers of the current device; the
- *    caller allocates and owns every buffer. The library allocates no memory and keeps
- *    no state apart from one device-side error word per device.
+ *    caller allocates and owns every buffer. The library allocates no memory. Its only
+ *    state is static: one device-side error word per device, the scratch array of
+ *    macaq_linear_w4a4_noalloc, the self-test's result words, and per-device host
+ *    facts (SM count, symbol addresses) looked up on first use.
  *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default stream).
- *    A returned MACAQ_OK means the work was validated and enqueued.
+ *    A returned MACAQ_OK means the work was validated and enqueued. Exceptions, each
+ *    stated at its declaration: macaq_grouped_linear_w4a4 and macaq_linear_w4a4_gather
+ *    copy small tables from host memory, which first waits for the stream's earlier
+ *    work; macaq_selftest_wait_timeout and macaq_get_device_error synchronise.
  *  - Arguments are validated on the host before any launch; a failed check returns an
  *    error code and enqueues nothing. Nothing throws or aborts across the ABI.
  *  - Only devices of compute capability 10.0 (B200, sm_100a) are supported.
