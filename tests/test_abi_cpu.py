@@ -98,3 +98,23 @@ def test_validation_rejects_bad_arguments(L):
     assert L.macaq_linear_w4a4_gather(a, 4, 256, ctypes.byref(w), d_mis, 1, 128, 0, a, 1 << 20, None) == 2
     assert L.macaq_linear_w4a4_gather(a, 4, 256, ctypes.byref(w), d_ok, 2, 64, 0, a, 1 << 20, None) == 1  # ldy < N
     assert L.macaq_linear_gather_workspace_bytes(4, 128, 256, 0) == L.macaq_linear_workspace_bytes(4, 128, 256, 0) + 512
+
+
+def test_no_usable_device_is_a_status_not_a_crash(L):
+    """Valid arguments on a machine without a usable CUDA device (the nearest this host
+    comes to a wrong architecture): every launching entry point returns MACAQ_ERR_CUDA
+    after validation, and nothing aborts."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a CUDA device is present")
+    a = ctypes.c_void_p(0x1000)
+    w = mq.MacaqWeight(0x1000, 0x1000, 0x1000, 128, 256)
+    d = (ctypes.c_uint64 * 1)(0x2000)
+    res = (ctypes.c_int64 * 10)()
+    assert L.macaq_quant_act(a, 4, 64, 64, a, a, a, None) == 5
+    assert L.macaq_prepare_weight(a, 4, 64, 64, a, a, a, a, None) == 5
+    assert L.macaq_gemm_mxfp4(a, a, 4, ctypes.byref(w), a, 128, 0, None, 0, None) == 5
+    assert L.macaq_linear_w4a4(a, 4, 256, ctypes.byref(w), a, 128, 0, 0, a, 1 << 24, None) == 5
+    assert L.macaq_linear_w4a4_gather(a, 4, 256, ctypes.byref(w), d, 1, 128, 0, a, 1 << 24, None) == 5
+    assert L.macaq_selftest_wait_timeout(100, res, None) == 5
+    assert L.macaq_get_device_error() == 5
