@@ -9,6 +9,13 @@ input lines and no dirty lines (whose write-back would be charged to the first k
 L2; each step is timed with CUDA events on the launching stream.
 
   python bench.py [--gpus N --steps K --warmup W] [--impl reference] [--workload NAME]
+  python bench.py --oracle-table
+
+The `e2e` leg times the same steps from pinned host memory: every step uploads its x,
+W and s and reads back its whole y, consecutive steps pipelined over copy-in, compute
+and copy-out streams. `--impl reference` times the oracle on the host cores on a
+bounded row sample; `--oracle-table` times the oracle per config, single-threaded and
+with OpenMP, and uses no GPU.
 
 Under torchrun (N > 1) every rank runs its own replica of the workload (token rows
 are independent, no data-path collective): weak scaling, value = all ranks' FLOPs /
