@@ -90,3 +90,37 @@ def random_mxfp4(rng, rows, K, scale_lo=117, scale_hi=137):
     codes = rng.integers(0, 256, size=(rows, K // 2)).astype(np.uint8)
     scales = rng.integers(scale_lo, scale_hi + 1, size=(rows, K // 32)).astype(np.uint8)
     return codes, scales
+
+
+def tile_covering_rows(M, n_rows=256, seed=0):
+    """Seeded output rows for a GEMM parity check that touch every 128-row M tile and, in
+    each, every 32-row group of the scale atom (rows r with (r // 32) % 4 = 0..3): the
+    same number of random rows from each 32-row group (at least one, enough for
+    n_rows in all), plus rows 0 and M - 1, topped up to min(M, n_rows) rows when short
+    groups hold fewer. Sorted, unique."""
+    rng = np.random.default_rng(seed)
+    groups = [(g0, min(g0 + 32, M)) for g0 in range(0, M, 32)]
+    per = max(1, -(-n_rows // len(groups)))
+    rows = [0, M - 1]
+    for g0, g1 in groups:
+        k = min(per, g1 - g0)
+        rows.extend((g0 + rng.choice(g1 - g0, k, replace=False)).tolist())
+    rows = np.unique(np.asarray(rows, dtype=np.int64))
+    short = min(M, n_rows) - rows.size
+    if short > 0:          # short groups at the end: top up from the rows not taken
+        rest = np.setdiff1d(np.arange(M, dtype=np.int64), rows)
+        rows = np.unique(np.concatenate([rows, rng.choice(rest, short, replace=False)]))
+    return rows
+
+
+class oracle_on_all_cores:
+    """Run the oracle's OpenMP build (bit-identical to the serial one, checked by
+    test_oracle_openmp) inside the block, to keep large parity references to seconds."""
+
+    def __enter__(self):
+        oracle.set_openmp(True)
+        return self
+
+    def __exit__(self, *exc):
+        oracle.set_openmp(False)
+        return False

@@ -2,13 +2,14 @@
 the C ABI on the seeded workloads, from the tiny layer to the full-size prefill,
 decode and decoder-layer shapes. Codes and scales are compared in full, bit for bit;
 GEMM outputs on all rows (small shapes) or on sampled rows (large shapes) against
-the oracle's fp64 sum of decoded products."""
+the oracle's fp64 sum of decoded products. The sampled rows cover every 128-row M
+tile of the launch and, in each, all four 32-row groups of the scale atom."""
 import numpy as np
 import pytest
 
 import oracle
 from helpers import (assert_bf16_matches_f32, assert_codes_equal, assert_gemm_close, assert_scales_equal,
-                     bf16_dev, f32_dev, host)
+                     bf16_dev, f32_dev, host, oracle_on_all_cores, tile_covering_rows)
 from mxfp4_w4a4_post_b200 import workloads as wl
 
 pytestmark = pytest.mark.gpu
@@ -34,18 +35,20 @@ def run_layer(mq, layer, sample_rows=None, check_bf16=True):
     del Wd
 
     # weight preparation and activation quantisation: bit-exact in full
-    rwc, rws, rinv = oracle.prepare_weight(W, s)
+    with oracle_on_all_cores():
+        rwc, rws, rinv = oracle.prepare_weight(W, s)
+        rac, ras = oracle.quant_rows(x, rinv)
     assert np.array_equal(host(pw.inv_s).view(np.uint32), rinv.view(np.uint32)), "inv_s"
     assert_codes_equal(host(pw.codes), rwc, f"{layer.name} W codes")
     assert_scales_equal(host(pw.scales), rws, K, f"{layer.name} W scales")
-    rac, ras = oracle.quant_rows(x, rinv)
     assert_codes_equal(host(a_codes), rac, f"{layer.name} x codes")
     assert_scales_equal(host(a_scales), ras, K, f"{layer.name} x scales")
 
-    # the GEMM output against the oracle's fp64 reference
-    rows = np.arange(M) if sample_rows is None or M <= sample_rows else \
-        np.unique(np.concatenate([np.random.default_rng(0).choice(M, sample_rows, replace=False), [0, M - 1]]))
-    ref = oracle.gemm_fp64(rac, ras, rwc, rws, K, rows=rows)
+    # the GEMM output against the oracle's fp64 reference: every row, or seeded rows
+    # that reach every M tile and every 32-row group of the scale atom
+    rows = np.arange(M) if sample_rows is None or M <= sample_rows else tile_covering_rows(M, sample_rows)
+    with oracle_on_all_cores():
+        ref = oracle.gemm_fp64(rac, ras, rwc, rws, K, rows=rows)
     fro, mx = assert_gemm_close(host(y32)[rows], ref, layer.name)
     if check_bf16:
         y16 = mq.linear(xd, pw, out_dtype=torch.bfloat16)
@@ -97,16 +100,16 @@ def test_qwen3_32b_up_decode_t3_variant(mq):
 
 
 def test_llama3_8b_gate_up_prefill(mq):
-    run_layer(mq, wl.llama3_8b_gate_up_prefill(), sample_rows=24)
+    run_layer(mq, wl.llama3_8b_gate_up_prefill(), sample_rows=256)
 
 
 def test_qwen3_32b_down_prefill(mq):
-    run_layer(mq, wl.qwen3_32b_down_prefill(), sample_rows=12, check_bf16=False)
+    run_layer(mq, wl.qwen3_32b_down_prefill(), sample_rows=256, check_bf16=False)
 
 
 @pytest.mark.parametrize("idx", range(7))
 def test_qwen3_32b_decoder_layer_b256(mq, idx):
-    run_layer(mq, wl.qwen3_32b_layer_decode(256)[idx], sample_rows=32)
+    run_layer(mq, wl.qwen3_32b_layer_decode(256)[idx])
 
 
 def test_ragged_layer(mq):
