@@ -20,10 +20,14 @@
  *    macaq_linear_w4a4_noalloc, the self-test's result words, and per-device host
  *    facts (SM count, symbol addresses) looked up on first use.
  *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default stream).
- *    A returned MACAQ_OK means the work was validated and enqueued. Exceptions, each
- *    stated at its declaration: macaq_grouped_linear_w4a4 and macaq_linear_w4a4_gather
- *    copy small tables from host memory, which first waits for the stream's earlier
- *    work; macaq_selftest_wait_timeout and macaq_get_device_error synchronise.
+ *    A returned MACAQ_OK means the work was validated and enqueued. Host arrays passed
+ *    in (offsets, weight descriptors, destination addresses) are read before the call
+ *    returns and may be reused at once: per-call tables reach the device inside kernel
+ *    parameters, never through a copy that waits for the stream. Exceptions:
+ *    macaq_selftest_wait_timeout and macaq_get_device_error synchronise.
+ *  - The library looks up, once per device, the device addresses of its static arrays
+ *    (the error word, the no-allocation scratch) and keeps them for the life of the
+ *    process: do not keep using it on a device after cudaDeviceReset.
  *  - Arguments are validated on the host before any launch; a failed check returns an
  *    error code and enqueues nothing. Nothing throws or aborts across the ABI.
  *  - Only devices of compute capability 10.0 (B200, sm_100a) are supported.
@@ -89,12 +93,14 @@ size_t macaq_codes_bytes(int64_t rows, int64_t K);
 size_t macaq_scales_bytes(int64_t rows, int64_t K);
 
 /* Device workspace macaq_gemm_mxfp4 needs for an M x N x K product with output
- * `out`: when the library splits K, one fp32 sum per output tile, an arrival count per
- * tile and a flag per CTA (the kernel clears what it needs itself); 0 otherwise. */
+ * `out`: when the library runs the product on a stream-K schedule (shapes with few
+ * output tiles per SM: the K tiles of all output tiles are dealt out evenly over the
+ * CTAs, so a tile may be shared by several), two fp32 partial tiles per CTA and an
+ * arrival counter per output tile; 0 otherwise. Its contents need no clearing. */
 size_t macaq_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, macaq_out_dtype out);
 
-/* Device workspace macaq_linear_w4a4 needs: the activation codes and scales, per-CTA
- * flags of the fused transform, and the GEMM workspace, each 256-byte aligned. */
+/* Device workspace macaq_linear_w4a4 needs: the activation codes and scales, then the
+ * GEMM workspace, each 256-byte aligned. */
 size_t macaq_linear_workspace_bytes(int64_t M, int64_t N, int64_t K, macaq_out_dtype out);
 
 /* ------------------------------------------------------------ compute --------- */
@@ -140,8 +146,11 @@ macaq_status macaq_quant_act(const void* x_bf16, int64_t M, int64_t K, int64_t l
  *            enables vector stores)
  *   workspace device, >= macaq_gemm_workspace_bytes(M, N, K, out), 256-byte aligned
  *            (may be NULL when that size is 0). Contents are scratch and need no
- *            clearing (each call tags its split-K flags with a value unique to the
- *            call); two calls that may run at the same time must not share it.
+ *            clearing: a stream-K product's CTAs never wait for one another; the last
+ *            contributor to a shared output tile adds the partial tiles, in the order
+ *            of their K ranges, and writes it, and each call tags its arrival counters
+ *            with a value unique to the call. Two calls that may run at the same time
+ *            must not share it.
  * M >= 1. Also the entry point for externally refined weight codes/scales. */
 macaq_status macaq_gemm_mxfp4(const uint8_t* a_codes, const uint8_t* a_scales, int64_t M,
                               const macaq_weight* w, void* y, int64_t ldy, macaq_out_dtype out,
@@ -150,9 +159,13 @@ macaq_status macaq_gemm_mxfp4(const uint8_t* a_codes, const uint8_t* a_scales, i
 /* The whole online layer: the activation transform of macaq_quant_act into the
  * workspace, then the GEMM of macaq_gemm_mxfp4.
  *   fused     0: two launches (macaq_quant_act's kernel, then the GEMM).
- *             1: for M <= 128 (decode) one launch: the GEMM kernel quantises the
- *             activations itself (each CTA a share, while its first weight tiles load)
- *             with the same bit-exact transform and encoding; for M > 128 as 0.
+ *             1: for M <= 32 (decode) one launch: the GEMM kernel makes the MXFP4
+ *             activations itself, K tile by K tile, in the shared memory its tensor-core
+ *             MMAs read them from (the per-channel multiplier, block Hadamard, E8M0
+ *             exponent and E2M1 encoding of macaq_quant_act, bit for bit), while the
+ *             weight tiles stream in; y is bit-identical to fused = 0. The activation
+ *             part of the workspace is then not written. For M > 32 as 0 (there every
+ *             CTA would repeat the transform of too many activation rows).
  *             Other values return MACAQ_ERR_INVALID_ARG.
  *   workspace device, >= macaq_linear_workspace_bytes(M, N, K, out), 256-byte aligned;
  *             it starts with the activation codes (macaq_codes_bytes(M, K) bytes) and,
@@ -175,11 +188,12 @@ macaq_status macaq_linear_w4a4(const void* x_bf16, int64_t M, int64_t ldx, const
  *             of w->N columns from there; aligned to the element size. Memory of another
  *             GPU must be accessible from this device (peer access or an IPC mapping).
  *   n_dest    1 .. 64
- *   workspace >= macaq_linear_gather_workspace_bytes(M, N, K, out), 256-byte aligned:
- *             macaq_linear_w4a4's workspace, then the destination table (copied from
- *             host memory on `stream`: the copy waits for the stream's earlier work)
+ *   workspace >= macaq_linear_gather_workspace_bytes(M, N, K, out) (the same size as
+ *             macaq_linear_w4a4's), 256-byte aligned. The destination addresses travel in
+ *             the GEMM kernel's parameters.
  * Every destination receives the same values that macaq_linear_w4a4 (fused = 0) would
- * write to y, except that K is never split. Completion of the writes into another
+ * write to y, except that no output tile is shared between CTAs (no stream-K
+ * schedule), so sums may round differently. Completion of the writes into another
  * GPU's memory is ordered for that GPU only by the caller (for example a barrier on
  * both streams after the call). */
 size_t macaq_linear_gather_workspace_bytes(int64_t M, int64_t N, int64_t K, macaq_out_dtype out);
@@ -202,13 +216,38 @@ macaq_status macaq_linear_w4a4_gather(const void* x_bf16, int64_t M, int64_t ldx
  *   workspace >= macaq_grouped_linear_workspace_bytes(offsets, G, K), 256-byte aligned:
  *             activation codes and scales with every group padded to 128 rows, the
  *             per-group tables of the GEMM and the quantiser's table of non-empty groups
- *             (copied from pageable host memory on `stream`: such a copy waits for the
- *             stream's earlier work)
+ *             (built on the host and written by small kernels that carry them in their
+ *             parameters, 16 KB per launch, ahead of the two compute launches)
  * G <= 4096. */
 size_t macaq_grouped_linear_workspace_bytes(const int64_t* offsets, int64_t G, int64_t K);
 macaq_status macaq_grouped_linear_w4a4(const void* x_bf16, int64_t ldx, const int64_t* offsets, int64_t G,
                                        const macaq_weight* weights, void* y, int64_t ldy, macaq_out_dtype out,
                                        void* workspace, size_t ws_bytes, macaq_stream stream);
+
+/* ----------------------------------- layers that share one input (one launch each) --- */
+
+/* Several MACaQ layers that read the same activation x: the q, k and v projections of
+ * an attention block, or the gate and up projections of an MLP (the pages apply the
+ * per-channel scale and block Hadamard to each linear layer's input separately; each
+ * weight carries its own s, so x goes through each weight's own online transform). One
+ * quantiser launch transforms x once per weight, with weights[g].inv_s, and one GEMM
+ * launch covers every weight's output tiles (prefill orientation, 128- or 192-wide
+ * weight tiles); y[g] = the layer of weights[g] applied to x, exactly what
+ * macaq_linear_w4a4 gives up to the order of fp32 sums.
+ *   x_bf16    device bf16 [M x K], row stride ldx (ldx >= K, ldx % 8 == 0), 16-byte
+ *             aligned
+ *   weights   host [G], all with the same K (N may differ)
+ *   y         host [G] device pointers: y[g] is [M x weights[g].N], fp32 or bf16 per
+ *             `out`, row stride ldy[g] (host [G]), aligned to the element size
+ *   workspace >= macaq_multi_linear_workspace_bytes(M, K, G), 256-byte aligned: the
+ *             activation codes and scales of every weight's transform (each padded to
+ *             128 rows), then the GEMM's tables (written by small kernels that carry
+ *             them in their parameters)
+ * 1 <= G <= 4096. */
+size_t macaq_multi_linear_workspace_bytes(int64_t M, int64_t K, int64_t G);
+macaq_status macaq_multi_linear_w4a4(const void* x_bf16, int64_t M, int64_t ldx, const macaq_weight* weights,
+                                     int64_t G, void* const* y, const int64_t* ldy, macaq_out_dtype out,
+                                     void* workspace, size_t ws_bytes, macaq_stream stream);
 
 /* ------------------------------------------ Hessian exponent search (offline) --- */
 
@@ -304,7 +343,7 @@ macaq_status macaq_flip_refine(const void* W_bf16, int64_t N, int64_t K, int64_t
  * libraries none of it, and latency-critical loops where allocating or freeing would
  * stall the device (cudaFree synchronises it) or could fail under memory pressure in the
  * middle of serving. This entry point takes no workspace: the activation codes, scales
- * and split-K partial sums live in one file-scope static device array of
+ * and stream-K partial tiles live in one file-scope static device array of
  * MACAQ_NOALLOC_SCRATCH_BYTES. The caller still passes x, the prepared weight and y,
  * with the same meaning, layout and alignment rules as macaq_linear_w4a4 (fused = 0).
  *
@@ -315,7 +354,7 @@ macaq_status macaq_flip_refine(const void* W_bf16, int64_t N, int64_t K, int64_t
  *   with that device current); make that first call before any stream capture.
  * - Every call on a device shares the one array, and the array keeps the last call's
  *   contents. Nothing in it needs to start at zero: every call overwrites what it reads
- *   and tags its split-K flags with a value unique to the call. Calls whose executions
+ *   and tags its stream-K counters with a value unique to the call. Calls whose executions
  *   overlap on the GPU (other streams, or no ordering between them) race on the array
  *   and give undefined results: order them on one stream.
  * - Allocates nothing: no cudaMalloc, cudaFree or allocating library routine. */
@@ -342,10 +381,12 @@ macaq_status macaq_get_device_error(void);
  *   [2] a wait on a barrier the warp completes itself: 1
  *   [3] the CTA's recorded error code (1: producer-wait timeout)
  *   [4] [5] time spent in waits [0] and [1], ns, by the device clock
- *   [6] wait on a global flag that holds another epoch, limit limit_us: 0 gave up
- *   [7] that CTA's recorded error code (5: split-K flag timeout)
- *   [8] time spent in wait [6], ns
- *   [9] wait on a flag that already holds the epoch: 1
+ *   [6] a group of three warps, one of whose waits (limit limit_us) cannot succeed,
+ *       agreeing at its named barrier whether to go on, as the kernel's warp groups
+ *       do: 0 (all leave together, none is held at the barrier)
+ *   [7] that CTA's recorded error code (5: a warp group's wait timed out)
+ *   [8] time spent in the wait that gave up, ns
+ *   [9] another member's own wait (on a barrier that completes): 1
  * limit_us must be in [1, 1000000] (else MACAQ_ERR_INVALID_ARG). A kernel that gives
  * up returns normally, so the context stays usable; the device error word read by
  * macaq_get_device_error is not touched. MACAQ_ERR_CUDA if the launch or copy fails. */

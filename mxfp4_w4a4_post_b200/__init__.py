@@ -66,6 +66,8 @@ def lib():
             "macaq_flip_refine": (I, [P, I64, I64, I64, P, P, P, P, I, P, P, SZ, P]),
             "macaq_grouped_linear_workspace_bytes": (SZ, [P, I64, I64]),
             "macaq_grouped_linear_w4a4": (I, [P, I64, P, I64, P, P, I64, I, P, SZ, P]),
+            "macaq_multi_linear_workspace_bytes": (SZ, [I64, I64, I64]),
+            "macaq_multi_linear_w4a4": (I, [P, I64, I64, P, I64, P, P, I, P, SZ, P]),
             "macaq_linear_gather_workspace_bytes": (SZ, [I64, I64, I64, I]),
             "macaq_linear_w4a4_gather": (I, [P, I64, I64, ctypes.POINTER(MacaqWeight), P, I, I64, I, P, SZ, P]),
             "macaq_selftest_wait_timeout": (I, [ctypes.c_uint32, ctypes.POINTER(I64), P]),
@@ -258,6 +260,33 @@ def grouped_linear(x, offsets, weights, out_dtype=None, y=None, workspace=None):
     return y
 
 
+def multi_linear(x, weights, out_dtype=None, ys=None, workspace=None):
+    """Several layers that share the input x (q/k/v, gate/up): returns [y_g] with
+    y_g = linear(x, weights[g]), from one quantiser launch and one GEMM launch."""
+    torch = _torch()
+    _require(x, torch.bfloat16, "x")
+    M, K = x.shape
+    G = len(weights)
+    if G == 0 or any(w.K != K for w in weights):
+        raise ValueError("weights must be non-empty and share x's K")
+    out_dtype = out_dtype or torch.bfloat16
+    dev = x.device
+    if ys is None:
+        ys = [torch.empty((M, w.N), dtype=out_dtype, device=dev) for w in weights]
+    for y, w in zip(ys, weights):
+        if tuple(y.shape) != (M, w.N) or y.dtype != ys[0].dtype or y.stride(1) != 1:
+            raise ValueError("outputs must be [M, N_g] with one dtype and unit column stride")
+    ws_structs = (MacaqWeight * G)(*[w.c_struct() for w in weights])
+    yp = (ctypes.c_void_p * G)(*[y.data_ptr() for y in ys])
+    lds = (ctypes.c_int64 * G)(*[y.stride(0) for y in ys])
+    need = lib().macaq_multi_linear_workspace_bytes(M, K, G)
+    ws, ws_bytes = _workspace(need, dev, workspace)
+    st = lib().macaq_multi_linear_w4a4(x.data_ptr(), M, x.stride(0), ws_structs, G, yp, lds, _out_code(ys[0].dtype),
+                                       ws.data_ptr(), ws_bytes, _stream_ptr(dev))
+    _check(st, "macaq_multi_linear_w4a4")
+    return ys
+
+
 def quant_act(x, inv_s, codes=None, scales=None):
     """x: bf16 [M, K]; inv_s: fp32 [K]. Returns (codes uint8 [M, K/2], scales uint8)."""
     torch = _torch()
@@ -360,8 +389,8 @@ def selftest_wait_timeout(limit_us=2000, device=None):
         _check(lib().macaq_selftest_wait_timeout(limit_us, res, _stream_ptr(dev)), "macaq_selftest_wait_timeout")
     r = list(res)
     return {"bar_timeout_ok": r[0], "bar_abort_ok": r[1], "bar_done_ok": r[2], "bar_err": r[3],
-            "bar_timeout_ns": r[4], "bar_abort_ns": r[5], "flag_timeout_ok": r[6], "flag_err": r[7],
-            "flag_timeout_ns": r[8], "flag_done_ok": r[9]}
+            "bar_timeout_ns": r[4], "bar_abort_ns": r[5], "set_agreed_ok": r[6], "set_err": r[7],
+            "set_timeout_ns": r[8], "set_member_ok": r[9]}
 
 
 def device_error():

@@ -45,64 +45,80 @@
 
 namespace macaq {
 
+// One group of a grouped GEMM: its P rows, its own weight (tensor map alongside, scale
+// atoms sf_q) with q_rows rows, and its own output (row row_y of out, row stride ldo).
 struct GemmGroup {
     int32_t unit_begin, rows, row_p, row_y;
+    int32_t q_rows, tiles_q;
     const uint8_t* sf_q;
-    int64_t pad;
+    void* out;
+    int64_t ldo;
 };
+
+// Largest number of destinations of a gathered output.
+constexpr int kMaxGatherDest = 64;
 
 struct GemmParams {
     const uint8_t* sf_p;     // scale atoms of P
     const uint8_t* sf_q;     // scale atoms of Q
-    void* out;               // y, or the fp32 split-K accumulator when atomic
+    void* out;               // y
     int64_t ldo;             // leading dimension of out, elements
     int32_t p_rows, q_rows;  // logical rows of P and Q
     int32_t k_tiles;         // ceil(K / 256)
     int32_t kb4_pad;         // scale atoms per 128-row slab along K
     int32_t tiles_p, tiles_q;
-    int32_t splits, k_tiles_per_split;
-    int32_t total_units;     // tiles_p * tiles_q * splits
+    int32_t total_units;     // tiles (grouped: every group's tiles)
     int32_t group_p;         // raster group height (in P tiles)
-    int32_t out_bf16;        // 1: bf16 output, 0: fp32 (ignored when atomic)
-    int32_t atomic;          // 1: split K, fp32 vector reductions into out
+    int32_t out_bf16;        // 1: bf16 output, 0: fp32
     int32_t transpose_out;   // 1: out[q * ldo + p], 0: out[p * ldo + q]
     int32_t vec_ok;          // 1: out and ldo allow 16-byte vector stores
     int32_t tma_store;       // 1: epilogue stages 32 x 32 output boxes in shared memory and
                              //    writes them with TMA stores (row-major tiles, vec_ok)
     int* err;                // device error word
-    // Split K (atomic): the accumulator `out` starts at zero without a separate memset.
-    // First thing, the epilogue warps of every CTA zero their slice of it and set their
-    // CTA's flag to `epoch` (a value unique to the call, so flags left by earlier calls
-    // never match); before its first reduction a CTA waits until every flag is set.
-    int64_t zero_vec4;               // 16-byte words of the accumulator
-    unsigned long long* cta_flags;   // [gridDim.x]
-    unsigned long long epoch;
-    // Fused activation transform (decode, Q = activations): first thing, the epilogue
-    // warps of every CTA quantise their share of the activation blocks into the Q codes
-    // and scales (the transform and encoding of macaq_quant_act) and then set the CTA's
-    // flag as above; the producer issues the Q side of its copies only once every flag
-    // is set (the weight side of its first fills goes ahead meanwhile).
-    int32_t fused;
-    const uint16_t* fx;              // bf16 activations [f_rows x f_K], row stride fx_ld
+    // Schedule (ungrouped). Tiles [0, sk_tile0) are whole units dealt round robin: CTA c
+    // takes tiles c, c + G, .. (G = gridDim.x). The K tiles of tiles [sk_tile0,
+    // total_units), tile after tile, form one sequence of sk_iters iterations that is
+    // split evenly over the CTAs (stream-K): CTA c takes iterations [c I / G, (c + 1) I / G)
+    // of it (G = sk_ctas, I = sk_iters), before its whole tiles, so a CTA's share of the
+    // grid's work differs from another's by at most one K tile. A tile whose K tiles fall to several CTAs is
+    // finished by the last of them to arrive: each writes its fp32 partial tile into its
+    // own slot of sk_partials (two per CTA: the first and the last tile of its stream-K
+    // range), counts itself in on the tile's counter, and the one that completes the count
+    // adds the partials in the order of their K ranges and writes y. No CTA ever waits for
+    // another, and as the stream-K tiles come first, a finisher's epilogue runs while its
+    // MMAs go on with its whole tiles. A counter holds the call's tag in its upper 48
+    // bits, so counts left by earlier calls (or whatever the workspace held) read as zero.
+    int32_t sk_tile0;                // first stream-K tile (total_units: none)
+    int32_t sk_ctas;                 // CTAs 0 .. sk_ctas - 1 share the stream-K iterations
+                                     // (at most sk_iters: every share is non-empty)
+    int64_t sk_iters;                // (total_units - sk_tile0) * k_tiles
+    float* sk_partials;              // [G][2][128 x BN] fp32
+    unsigned long long* sk_counters; // [total_units]
+    unsigned long long sk_tag;       // 48-bit tag unique to the call
+    // Fused activation transform (the kernel's FUSED instantiation; decode, Q =
+    // activations, one Q tile): the scale-factor warps transform the bf16 activation K
+    // tile themselves (per-channel multiplier, block Hadamard, E8M0 exponent, E2M1 codes)
+    // and write the codes into the stage's Q buffer and the scales into its Q scale
+    // chunk, in the layouts the TMA would have written; only the weight side is copied.
+    const uint16_t* fx;              // bf16 activations [q_rows x f_K], row stride fx_ld
     int64_t fx_ld;
     const float* f_mult;             // inv_s [f_K]
-    uint8_t* f_codes;                // [f_rows x f_K/2]
-    uint8_t* f_scales;               // atom layout, 128-row slabs x f_kb_pad blocks
-    int32_t f_rows, f_K, f_kb_pad;
-    // Grouped GEMM (groups > 0; prefill orientation, no split K): group g multiplies the
-    // g_rows[g] activation rows starting at P row g_row_p[g] (a multiple of 128: groups
-    // sit in whole scale slabs) by its own weight (tensor map g_tmaps[g], scale atoms
-    // g_sf_q[g]) and writes y rows g_row_y[g] ..; its units are g_unit_begin[g] ..
-    // g_unit_begin[g + 1] - 1, P tiles fastest.
+    int32_t f_K;
+    // Grouped GEMM (groups > 0; prefill orientation, every tile whole): group g multiplies
+    // its rows activation rows starting at P row row_p (a multiple of 128: groups sit in
+    // whole scale slabs) by its own weight (tensor map g_tmaps[g], q_rows rows, scale atoms
+    // sf_q) and writes rows row_y .. of its own output; its units are unit_begin ..
+    // unit_begin + ceil(rows / 128) * tiles_q - 1, P tiles fastest.
     int32_t groups;
     const GemmGroup* g_desc;         // [groups]
     const CUtensorMap* g_tmaps;      // [groups], 64-byte aligned
     // Gathered output (column-parallel layers; the kernel's GATHER instantiation): every
     // output element goes to each of dest[0 .. n_dest - 1] (device addresses of the
     // destinations' first column for this weight, the same row stride ldo) instead of to
-    // out, with direct stores (no TMA store, no split K).
+    // out, with direct stores (no TMA store, no stream-K schedule). The addresses travel
+    // in the kernel's parameters.
     int32_t n_dest;
-    const unsigned long long* dest;  // [n_dest], device memory
+    unsigned long long dest[kMaxGatherDest];
 };
 
 enum : int {
@@ -110,7 +126,7 @@ enum : int {
     kErrTimeoutMma = 2,
     kErrTimeoutEpilogue = 3,
     kErrSfOffset = 4,
-    kErrTimeoutSplit = 5
+    kErrTimeoutSet = 5
 };
 
 template <int BN, int STAGES>
@@ -141,26 +157,34 @@ struct GemmShape {
     static_assert(kTmemNeed <= 512, "tensor memory budget");
     static constexpr int kTmemCols = kTmemNeed <= 32 ? 32 : kTmemNeed <= 64 ? 64
                                    : kTmemNeed <= 128 ? 128 : kTmemNeed <= 256 ? 256 : 512;
-    static constexpr int kChunkCols = BN <= 32 ? 16 : 32;   // epilogue TMEM load width
+    static constexpr int kChunkCols = BN <= 64 ? 16 : 32;   // epilogue TMEM load width
     // Output staging for TMA stores (wide tiles only): one box of 32 rows x 64 bytes
     // (32 bf16 or 16 fp32 columns) per epilogue warp.
     static constexpr int kStageBoxBytes = 32 * 64;
     static constexpr int kStagingBytes = BN >= 128 ? 4 * kStageBoxBytes : 0;
 };
 
-template <int BN, int STAGES>
+template <int BN, int STAGES, bool FUSED = false>
 struct GemmSmem {
     using S = GemmShape<BN, STAGES>;
+    // the fused variant keeps its Q operand for every K tile in one persistent region
+    // after the fixed layout instead of in the stage ring
+    static constexpr int kQRing = FUSED ? 0 : 1;
     static constexpr int kOffP = 0;
     static constexpr int kOffQ = kOffP + STAGES * S::kPTileBytes;
-    static constexpr int kOffSfP = kOffQ + STAGES * S::kQTileBytes;
+    static constexpr int kOffSfP = kOffQ + kQRing * STAGES * S::kQTileBytes;
     static constexpr int kOffSfQ = kOffSfP + STAGES * S::kSfChunkBytes;
-    static constexpr int kOffStaging = kOffSfQ + STAGES * S::kQChunks * S::kSfChunkBytes;   // 1 KB aligned
+    static constexpr int kOffStaging = kOffSfQ + kQRing * STAGES * S::kQChunks * S::kSfChunkBytes;   // 1 KB aligned
     static constexpr int kOffBar = kOffStaging + S::kStagingBytes;
     static constexpr int kNumBars = 3 * STAGES + 4 + 1;
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;
     static constexpr int kBytes = kOffMisc + 16;
+    // fused: Q codes of K tile kt at kOffPersist + kt * BN * 128 (128-byte swizzle, as the
+    // copies of the plain kernel lay them out), then its scale atoms (1 KB per K tile)
+    static constexpr int kOffPersist = (kBytes + 1023) / 1024 * 1024;
+    static constexpr int kPersistPerKt = S::kQTileBytes + S::kSfChunkBytes;
     static constexpr int kAlloc = kBytes + 1024;            // slack to align the base to 1 KB
+    static constexpr int alloc(int k_tiles) { return FUSED ? kOffPersist + k_tiles * kPersistPerKt + 1024 : kAlloc; }
 };
 
 __device__ __forceinline__ uint64_t global_timer_ns() {
@@ -212,16 +236,77 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
     return __all_sync(0xffffffffu, wait_or_abort(bar, parity, abort, err, code, limit_ns));
 }
 
+// Named barrier `id` over `nthreads` threads (whole warps) that also returns, to every
+// thread, whether `v` held in all of them.
+__device__ __forceinline__ bool bar_and(int id, int nthreads, bool v) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.and.pred q, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)v), "r"(id), "r"(nthreads)
+        : "memory");
+    return r != 0;
+}
+
 struct Unit {
-    int tile, split, tp, tq, kt_begin, kt_end;
+    int tile, tp, tq, kt_begin, kt_end;
     int p_row0;                    // first P row of the tile in the P tensor map
     int out_row0;                  // output row of the tile's P row 0
     int rows;                      // valid P rows from p_row0 on (the tile's group)
+    int q_rows;                    // rows of the tile's Q operand (its group's)
     const CUtensorMap* tmap_q;     // Q tensor map of the tile
     const uint8_t* sf_q;           // Q scale atoms of the tile
+    void* out;                     // the tile's output and its row stride
+    int64_t ldo;
 };
 
-__device__ __forceinline__ Unit decode_unit(const GemmParams& p, int u, const CUtensorMap* tmap_q) {
+// The units a CTA works through, in order: its stream-K tiles sk_first .. sk_first +
+// n_sk - 1 (the tiles that hold iterations [i0, i1) of the stream-K sequence, each
+// clipped to the K tiles in that range), then its whole tiles blockIdx.x, blockIdx.x + G,
+// .. below sk_tile0 (grouped GEMM: every tile is whole).
+struct Sched {
+    int n_sk, sk_first, n_units;
+    int64_t i0, i1;
+    __device__ __forceinline__ int unit(int j) const {
+        return j < n_sk ? sk_first + j : (int)blockIdx.x + (j - n_sk) * (int)gridDim.x;
+    }
+};
+
+__device__ __forceinline__ int64_t sk_start(const GemmParams& p, int c) {
+    return (int64_t)c * p.sk_iters / p.sk_ctas;
+}
+
+__device__ __forceinline__ Sched cta_sched(const GemmParams& p) {
+    Sched s;
+    const int whole = p.groups > 0 ? p.total_units : p.sk_tile0;
+    s.i0 = 0;
+    s.i1 = 0;
+    s.n_sk = 0;
+    s.sk_first = 0;
+    if (p.groups == 0 && p.sk_iters > 0 && (int)blockIdx.x < p.sk_ctas) {
+        s.i0 = sk_start(p, blockIdx.x);
+        s.i1 = sk_start(p, blockIdx.x + 1);
+        if (s.i1 > s.i0) {
+            s.sk_first = p.sk_tile0 + (int)(s.i0 / p.k_tiles);
+            s.n_sk = p.sk_tile0 + (int)((s.i1 - 1) / p.k_tiles) + 1 - s.sk_first;
+        }
+    }
+    const int n_whole = (int)blockIdx.x < whole ? (whole - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+    s.n_units = s.n_sk + n_whole;
+    return s;
+}
+
+// The CTA whose stream-K range holds iteration j: the largest c with c I / G <= j (every
+// range is non-empty, as G <= I, so the CTAs from the holder of a tile's first K tile to
+// the holder of its last are exactly its contributors).
+__device__ __forceinline__ int sk_cta_of(const GemmParams& p, int64_t j) {
+    return (int)(((j + 1) * p.sk_ctas - 1) / p.sk_iters);
+}
+
+__device__ __forceinline__ Unit decode_unit(const GemmParams& p, int u, const CUtensorMap* tmap_q, const Sched& sc) {
     if (p.groups > 0) {
         // the group whose units contain u: binary search over the unit offsets
         int lo = 0, hi = p.groups - 1;
@@ -234,7 +319,6 @@ __device__ __forceinline__ Unit decode_unit(const GemmParams& p, int u, const CU
         const int lu = u - gd.unit_begin;
         Unit x;
         x.tile = u;
-        x.split = 0;
         x.tp = lu % tiles_p;
         x.tq = lu / tiles_p;
         x.kt_begin = 0;
@@ -242,79 +326,84 @@ __device__ __forceinline__ Unit decode_unit(const GemmParams& p, int u, const CU
         x.p_row0 = gd.row_p + x.tp * 128;
         x.out_row0 = gd.row_y + x.tp * 128;
         x.rows = gd.rows - x.tp * 128;
+        x.q_rows = gd.q_rows;
         x.tmap_q = p.g_tmaps + lo;
         x.sf_q = gd.sf_q;
+        x.out = gd.out;
+        x.ldo = gd.ldo;
         return x;
     }
-    const int tile = u / p.splits;
-    const int split = u - tile * p.splits;
+    const int tile = u;
     const int per_group = p.group_p * p.tiles_q;
     const int g = tile / per_group;
     const int r = tile - g * per_group;
     const int gp = min(p.group_p, p.tiles_p - g * p.group_p);
     Unit x;
     x.tile = tile;
-    x.split = split;
     x.tp = g * p.group_p + r % gp;
     x.tq = r / gp;
-    x.kt_begin = split * p.k_tiles_per_split;
-    x.kt_end = min(p.k_tiles, x.kt_begin + p.k_tiles_per_split);
+    x.kt_begin = 0;
+    x.kt_end = p.k_tiles;
+    if (tile >= p.sk_tile0) {
+        // a stream-K tile: the K tiles of it in this CTA's range
+        const int64_t t0 = (int64_t)(tile - p.sk_tile0) * p.k_tiles;
+        x.kt_begin = (int)(max(sc.i0, t0) - t0);
+        x.kt_end = (int)(min(sc.i1, t0 + p.k_tiles) - t0);
+    }
     x.p_row0 = x.tp * 128;
     x.out_row0 = x.tp * 128;
     x.rows = p.p_rows - x.tp * 128;
+    x.q_rows = p.q_rows;
     x.tmap_q = tmap_q;
     x.sf_q = p.sf_q;
+    x.out = p.out;
+    x.ldo = p.ldo;
     return x;
 }
 
+// Stream-K: count this CTA in on a tile's counter; returns the count including this
+// arrival (1 for the first arrival of the call). Lock-free: the compare-and-swap loop
+// only retries when another contributor of the same tile arrived in between.
+__device__ __forceinline__ uint32_t sk_arrive(unsigned long long* ctr, unsigned long long tag) {
+    unsigned long long cur = *reinterpret_cast<volatile unsigned long long*>(ctr);
+    for (;;) {
+        const uint32_t n = (cur >> 16) == tag ? (uint32_t)(cur & 0xFFFFu) : 0u;
+        const unsigned long long next = (tag << 16) | (unsigned long long)(n + 1);
+        const unsigned long long prev = atomicCAS(ctr, cur, next);
+        if (prev == cur) return n + 1;
+        cur = prev;
+    }
+}
+
 // Writes one chunk of output row `prow` (a P row; the output column of it when
-// transposed) if `valid`.
+// transposed) if `valid`, into `out` with row stride ldo and q_rows columns (rows when
+// transposed).
 template <int CW>
-__device__ __forceinline__ void store_chunk(const GemmParams& p, void* out, int prow, bool valid, int q_base,
-                                            const uint32_t (&r)[CW]) {
+__device__ __forceinline__ void store_chunk(const GemmParams& p, void* out, int64_t ldo, int q_rows, int prow,
+                                            bool valid, int q_base, const uint32_t (&r)[CW]) {
     if (!valid) return;
     if (p.transpose_out) {
         // out[q, prow]: for each column the 32 lanes of the warp write consecutive prow
-        if (p.atomic) {
-            float* o = reinterpret_cast<float*>(out);
-#pragma unroll
-            for (int j = 0; j < CW; ++j) {
-                const int q = q_base + j;
-                if (q < p.q_rows) atomicAdd(o + (int64_t)q * p.ldo + prow, __uint_as_float(r[j]));
-            }
-        } else if (p.out_bf16) {
+        if (p.out_bf16) {
             __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(out);
 #pragma unroll
             for (int j = 0; j < CW; ++j) {
                 const int q = q_base + j;
-                if (q < p.q_rows) o[(int64_t)q * p.ldo + prow] = __float2bfloat16_rn(__uint_as_float(r[j]));
+                if (q < q_rows) o[(int64_t)q * ldo + prow] = __float2bfloat16_rn(__uint_as_float(r[j]));
             }
         } else {
             float* o = reinterpret_cast<float*>(out);
 #pragma unroll
             for (int j = 0; j < CW; ++j) {
                 const int q = q_base + j;
-                if (q < p.q_rows) o[(int64_t)q * p.ldo + prow] = __uint_as_float(r[j]);
+                if (q < q_rows) o[(int64_t)q * ldo + prow] = __uint_as_float(r[j]);
             }
         }
         return;
     }
-    const bool full = q_base + CW <= p.q_rows && p.vec_ok;
-    if (p.atomic) {
-        float* o = reinterpret_cast<float*>(out) + (int64_t)prow * p.ldo + q_base;
-        if (full) {
-#pragma unroll
-            for (int j = 0; j < CW; j += 4)
-                atomicAdd(reinterpret_cast<float4*>(o + j),
-                          make_float4(__uint_as_float(r[j]), __uint_as_float(r[j + 1]),
-                                      __uint_as_float(r[j + 2]), __uint_as_float(r[j + 3])));
-        } else {
-#pragma unroll
-            for (int j = 0; j < CW; ++j)
-                if (q_base + j < p.q_rows) atomicAdd(o + j, __uint_as_float(r[j]));
-        }
-    } else if (p.out_bf16) {
-        __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(out) + (int64_t)prow * p.ldo + q_base;
+    const bool full = q_base + CW <= q_rows && p.vec_ok;
+    if (p.out_bf16) {
+        __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(out) + (int64_t)prow * ldo + q_base;
         if (full) {
 #pragma unroll
             for (int j = 0; j < CW; j += 8) {
@@ -332,10 +421,10 @@ __device__ __forceinline__ void store_chunk(const GemmParams& p, void* out, int 
         } else {
 #pragma unroll
             for (int j = 0; j < CW; ++j)
-                if (q_base + j < p.q_rows) o[j] = __float2bfloat16_rn(__uint_as_float(r[j]));
+                if (q_base + j < q_rows) o[j] = __float2bfloat16_rn(__uint_as_float(r[j]));
         }
     } else {
-        float* o = reinterpret_cast<float*>(out) + (int64_t)prow * p.ldo + q_base;
+        float* o = reinterpret_cast<float*>(out) + (int64_t)prow * ldo + q_base;
         if (full) {
 #pragma unroll
             for (int j = 0; j < CW; j += 4)
@@ -345,37 +434,8 @@ __device__ __forceinline__ void store_chunk(const GemmParams& p, void* out, int 
         } else {
 #pragma unroll
             for (int j = 0; j < CW; ++j)
-                if (q_base + j < p.q_rows) o[j] = __uint_as_float(r[j]);
+                if (q_base + j < q_rows) o[j] = __uint_as_float(r[j]);
         }
-    }
-}
-
-// Split-K zeroing protocol (gpu scope): a CTA zeroes its slice, fences, and one thread
-// releases its flag; the epilogue lanes acquire every CTA's flag before reducing.
-__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long* f) {
-    unsigned long long v;
-    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(f) : "memory");
-    return v;
-}
-__device__ __forceinline__ void st_release_u64(unsigned long long* f, unsigned long long v) {
-    asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(f), "l"(v) : "memory");
-}
-// Wait (bounded, ~2 s) until *flag == epoch. On give-up record kErrTimeoutSplit, raise
-// the CTA abort flag and return false. Polls sleep briefly: the flag lives in L2.
-__device__ __noinline__ bool wait_split_flag(const unsigned long long* flag, unsigned long long epoch,
-                                             volatile int* abort, int* err, uint64_t limit_ns = kWaitLimitNs) {
-    const uint64_t t0 = global_timer_ns();
-    for (uint32_t it = 0;; ++it) {
-        if (ld_acquire_u64(flag) == epoch) return true;
-        if ((it & 15) == 15) {
-            if (*abort) return false;
-            if (global_timer_ns() - t0 > limit_ns) {
-                atomicExch(err, kErrTimeoutSplit);
-                *abort = 1;
-                return false;
-            }
-        }
-        __nanosleep(128);
     }
 }
 
@@ -398,55 +458,106 @@ __device__ __forceinline__ void tmem_load_chunk<16>(uint32_t taddr, uint32_t (&r
         : "r"(taddr));
 }
 
-// This CTA's share of the fused activation transform: one 32-element block per thread
-// and step over the 128-row slab(s) x f_kb_pad blocks of the Q operand. Blocks of real
-// rows and columns get codes and their scale byte; padding blocks get scale byte 0.
-__device__ __forceinline__ void fused_quant_share(const GemmParams& p, int et) {
-    const int kb = p.f_K >> 5;
-    const int64_t rows_pad = ((int64_t)p.f_rows + 127) / 128 * 128;
-    const int64_t total = rows_pad * p.f_kb_pad;
-    const int64_t per = (total + gridDim.x - 1) / gridDim.x;
-    const int64_t b0 = (int64_t)blockIdx.x * per, b1 = min(total, b0 + per);
-    for (int64_t i = b0 + et; i < b1; i += 128) {
-        const int row = (int)(i / p.f_kb_pad);
-        const int b = (int)(i - (int64_t)row * p.f_kb_pad);
-        uint32_t sbyte = 0;
-        if (row < p.f_rows && b < kb) {
-            const uint4* xs = reinterpret_cast<const uint4*>(p.fx + (int64_t)row * p.fx_ld + (int64_t)b * 32);
-            const float4* ms = reinterpret_cast<const float4*>(p.f_mult + (int64_t)b * 32);
-            uint64_t T[16];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const uint4 v = __ldg(xs + j);
-                const float4 m0 = __ldg(ms + 2 * j), m1 = __ldg(ms + 2 * j + 1);
-                const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-                const uint64_t mm[4] = {pk(m0.x, m0.y), pk(m0.z, m0.w), pk(m1.x, m1.y), pk(m1.z, m1.w)};
-#pragma unroll
-                for (int q = 0; q < 4; ++q)
-                    T[4 * j + q] = mul2(pk(__uint_as_float(w[q] << 16), __uint_as_float(w[q] & 0xFFFF0000u)), mm[q]);
-            }
-            uint32_t packed[4];
-            sbyte = encode_block(T, packed);
-            *reinterpret_cast<uint4*>(p.f_codes + (int64_t)row * (p.f_K >> 1) + (int64_t)b * 16) =
-                make_uint4(packed[0], packed[1], packed[2], packed[3]);
-        }
-        const int64_t o = ((int64_t)(row >> 7) * (p.f_kb_pad >> 2) + (b >> 2)) * 512 + (row & 31) * 16 +
-                          ((row >> 5) & 3) * 4 + (b & 3);
-        p.f_scales[o] = (uint8_t)sbyte;
-    }
-}
-
 constexpr int kSfWarpSets = 2;                                // scale-writer sets
+constexpr int kPrefetchAhead = 4;                             // K tiles of L2 prefetch beyond the copies
 constexpr int kGemmThreads = 32 * (6 + 4 * kSfWarpSets);
 
-// GATHER: the output goes to p.dest[0 .. p.n_dest - 1] (a separate instantiation, so
-// that the ordinary kernels keep their registers).
-template <int BN, int STAGES, bool GATHER = false>
+// Kernel variants, each its own instantiation so that the ordinary kernels keep their
+// registers: kVarGather writes the output to p.dest[0 .. p.n_dest - 1]; kVarFused makes
+// the Q operand (the activations) from bf16 inside the kernel.
+enum : int { kVarPlain = 0, kVarGather = 1, kVarFused = 2 };
+
+// The fused variant's Q operand, made once per CTA before its main loop by warps 2-13
+// (the epilogue and scale-factor warps; the producer starts streaming the weight tiles
+// meanwhile and the MMA warp waits for its first scale slot): the MXFP4 form of the
+// activation's q_rows (<= BN) rows for every K tile, with the quantiser's own block
+// routine, written where the copies of the plain kernel would have put each K tile:
+// codes at kOffPersist + kt * BN * 128 in the 128-byte swizzle (16-byte piece j of row r
+// at j ^ (r % 8)), scales in a 1 KB atom chunk per K tile after them. Rows past the last
+// activation row get zero codes, blocks past K zero codes and scale byte 0 (what the
+// zero-filled copies give). Item i = (K tile, row, block) goes to thread i % 384 of the
+// warps, so four consecutive lanes hold the four blocks of one scale word.
+constexpr int kFusedThreads = 32 * (4 + 4 * kSfWarpSets);
+
+template <int BN, int STAGES>
+__device__ __forceinline__ void fused_transform(const GemmParams& p, uint8_t* smem) {
+    using S = GemmShape<BN, STAGES>;
+    using L = GemmSmem<BN, STAGES, true>;
+    const int tt = (int)threadIdx.x - 64;              // 0 .. kFusedThreads - 1
+    const int rows = p.q_rows;
+    const int kb = p.f_K >> 5;
+    const uint32_t qp = ptx::smem_u32(smem + L::kOffPersist);
+    const uint32_t sp = qp + p.k_tiles * S::kQTileBytes;
+    const int zero_items = (BN - rows) * 8;            // 16-byte pieces of rows past the last
+    for (int i = tt; i < p.k_tiles * zero_items; i += kFusedThreads) {
+        const int kt = i / zero_items, rem = i - kt * zero_items;
+        ptx::sts128(qp + kt * S::kQTileBytes + (rows + rem / 8) * 128 + (rem % 8) * 16, 0u, 0u, 0u, 0u);
+    }
+    for (int i = tt; i < p.k_tiles * S::kSfChunkBytes / 16; i += kFusedThreads) ptx::sts128(sp + 16 * i, 0u, 0u, 0u, 0u);
+    asm volatile("bar.sync 2, %0;" ::"n"(kFusedThreads) : "memory");   // zeros before scale words
+    const int total = p.k_tiles * rows * 8;
+    for (int base = 0; base < total; base += kFusedThreads) {
+        const int i = base + tt;
+        const bool live = i < total;
+        int kt = 0, r = 0, j = 0;
+        if (live) {
+            kt = i / (rows * 8);
+            const int rem = i - kt * rows * 8;
+            r = rem >> 3;
+            j = rem & 7;
+        }
+        const int b = kt * 8 + j;
+        uint32_t sbyte = 0;
+        if (live) {
+            uint32_t packed[4] = {0u, 0u, 0u, 0u};
+            if (b < kb) {
+                const uint4* xs = reinterpret_cast<const uint4*>(p.fx + (int64_t)r * p.fx_ld + (int64_t)b * 32);
+                const float4* ms = reinterpret_cast<const float4*>(p.f_mult + (int64_t)b * 32);
+                uint4 xv[4];
+                float4 mv[8];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) xv[c] = __ldg(xs + c);
+#pragma unroll
+                for (int c = 0; c < 8; ++c) mv[c] = __ldg(ms + c);
+                uint64_t T[16];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const uint32_t w[4] = {xv[c].x, xv[c].y, xv[c].z, xv[c].w};
+                    const uint64_t mm[4] = {pk(mv[2 * c].x, mv[2 * c].y), pk(mv[2 * c].z, mv[2 * c].w),
+                                            pk(mv[2 * c + 1].x, mv[2 * c + 1].y), pk(mv[2 * c + 1].z, mv[2 * c + 1].w)};
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        T[4 * c + q] =
+                            mul2(pk(__uint_as_float(w[q] << 16), __uint_as_float(w[q] & 0xFFFF0000u)), mm[q]);
+                }
+                sbyte = encode_block(T, packed);
+            }
+            ptx::sts128(qp + kt * S::kQTileBytes + r * 128 + ((j ^ (r & 7)) << 4), packed[0], packed[1], packed[2],
+                        packed[3]);
+        }
+        const uint32_t s1 = __shfl_down_sync(0xffffffffu, sbyte, 1);
+        const uint32_t s2 = __shfl_down_sync(0xffffffffu, sbyte, 2);
+        const uint32_t s3 = __shfl_down_sync(0xffffffffu, sbyte, 3);
+        if (live && (j & 3) == 0)
+            ptx::sts32(sp + kt * S::kSfChunkBytes + 512 * (j >> 2) + (r & 31) * 16 + ((r >> 5) & 3) * 4,
+                       sbyte | (s1 << 8) | (s2 << 16) | (s3 << 24));
+    }
+    // the MMAs read the codes through the async proxy; the scale-factor warps read the
+    // scale words after this barrier
+    ptx::fence_proxy_async_smem();
+    asm volatile("bar.sync 2, %0;" ::"n"(kFusedThreads) : "memory");
+}
+
+template <int BN, int STAGES, int VAR = kVarPlain>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_mxf4_kernel(const __grid_constant__ CUtensorMap tmap_p, const __grid_constant__ CUtensorMap tmap_q,
                      const __grid_constant__ CUtensorMap tmap_y, const GemmParams p) {
+    constexpr bool GATHER = VAR == kVarGather;
+    constexpr bool FUSED = VAR == kVarFused;
+    // The fused variant covers Q tiles of at most 32 rows (one 128-row scale slab).
+    static_assert(!FUSED || BN <= 32, "fused transform tile");
     using S = GemmShape<BN, STAGES>;
-    using L = GemmSmem<BN, STAGES>;
+    using L = GemmSmem<BN, STAGES, FUSED>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -489,9 +600,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    const Sched sc = cta_sched(p);
     // Set-up above overlaps the previous kernel's tail; operands are read only after it.
     ptx::griddep_wait();
     ptx::griddep_launch_dependents();
+    if constexpr (FUSED) {
+        if (warp >= 2) fused_transform<BN, STAGES>(p, smem);
+    }
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer ---
@@ -501,7 +616,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         int stage = 0;
         uint32_t phase = 0;
         uint32_t issued_mask = 0, issued_phase = 0;
-        const int q_slabs = (p.q_rows + 127) / 128;
         // Q side of one fill: codes tile and scale chunks
         auto issue_q = [&](const Unit& t, int st, int kt, int q0, int slab0, int nchunks) {
             ptx::tma_load_2d(smem + L::kOffQ + st * S::kQTileBytes, t.tmap_q, &full[st], kt * S::kBKBytes, q0);
@@ -510,15 +624,29 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                                t.sf_q + ((int64_t)(slab0 + c) * p.kb4_pad + 2 * kt) * 512, S::kSfChunkBytes,
                                &full[st]);
         };
-        bool q_ready = !p.fused;
-        int deferred = 0;                   // fills of the first unit still without their Q side
-        for (int u = blockIdx.x; u < p.total_units; u += gridDim.x) {
+        // L2 prefetch of the K tile kPrefetchAhead positions further along this CTA's
+        // schedule, so that the copy of it later finds its lines in L2
+        auto prefetch = [&](const Unit& t, int kt) {
+            const int q0 = t.tq * BN;
+            ptx::tma_prefetch_2d(&tmap_p, kt * S::kBKBytes, t.p_row0);
+            ptx::bulk_prefetch_l2(p.sf_p + ((int64_t)(t.p_row0 >> 7) * p.kb4_pad + 2 * kt) * 512, S::kSfChunkBytes);
+            if constexpr (!FUSED) {
+                ptx::tma_prefetch_2d(t.tmap_q, kt * S::kBKBytes, q0);
+                ptx::bulk_prefetch_l2(t.sf_q + ((int64_t)(q0 / 128) * p.kb4_pad + 2 * kt) * 512, S::kSfChunkBytes);
+            }
+        };
+        for (int uj = 0; uj < sc.n_units; ++uj) {
+            const int u = sc.unit(uj);
             if (cta_aborted(abort)) break;
-            const Unit t = decode_unit(p, u, &tmap_q);
+            const Unit t = decode_unit(p, u, &tmap_q, sc);
+            const bool has_next = uj + 1 < sc.n_units;
+            const Unit tn = has_next ? decode_unit(p, sc.unit(uj + 1), &tmap_q, sc) : t;
             const int q0 = t.tq * BN;
             const int slab0 = q0 / 128;
-            const int nchunks = min(S::kQChunks, q_slabs - slab0);
-            const uint32_t bytes = S::kPTileBytes + S::kQTileBytes + S::kSfChunkBytes * (1 + nchunks);
+            const int nchunks = min(S::kQChunks, (t.q_rows + 127) / 128 - slab0);   // scale slabs of the Q rows
+            // the fused variant copies only the weight side; its Q side is made in place
+            const uint32_t bytes = FUSED ? S::kPTileBytes + S::kSfChunkBytes
+                                         : S::kPTileBytes + S::kQTileBytes + S::kSfChunkBytes * (1 + nchunks);
             bool ok = true;
             for (int kt = t.kt_begin; kt < t.kt_end; ++kt) {
                 if (!warp_wait(&empty[stage], phase ^ 1, abort, p.err, kErrTimeoutProducer)) { ok = false; break; }
@@ -529,25 +657,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     ptx::bulk_load(smem + L::kOffSfP + stage * S::kSfChunkBytes,
                                    p.sf_p + ((int64_t)(t.p_row0 >> 7) * p.kb4_pad + 2 * kt) * 512,
                                    S::kSfChunkBytes, &full[stage]);
-                    if (q_ready) issue_q(t, stage, kt, q0, slab0, nchunks);
+                    if constexpr (!FUSED) issue_q(t, stage, kt, q0, slab0, nchunks);
+                    const int pk = kt + kPrefetchAhead;
+                    if (pk < t.kt_end)
+                        prefetch(t, pk);
+                    else if (has_next && tn.kt_begin + (pk - t.kt_end) < tn.kt_end)
+                        prefetch(tn, tn.kt_begin + (pk - t.kt_end));
                 }
                 __syncwarp();
                 issued_mask |= 1u << stage;
                 issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
                 if (++stage == STAGES) { stage = 0; phase ^= 1; }
-                if (!q_ready && (++deferred == STAGES || kt + 1 == t.kt_end)) {
-                    // every CTA's share of the quantised activations is in memory: give
-                    // the deferred fills (stages 0.. of the first unit) their Q side
-                    bool fl = true;
-                    for (int i = lane; i < (int)gridDim.x && fl; i += 32)
-                        fl = wait_split_flag(p.cta_flags + i, p.epoch, abort, p.err);
-                    if (!__all_sync(0xffffffffu, fl)) { ok = false; break; }
-                    ptx::fence_proxy_async_global();
-                    if (leader)
-                        for (int d = 0; d < deferred; ++d) issue_q(t, d, t.kt_begin + d, q0, slab0, nchunks);
-                    __syncwarp();
-                    q_ready = true;
-                }
             }
             if (!ok) break;
         }
@@ -575,9 +695,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         int acc = 0;
         uint32_t acc_phase = 0;
         bool issued = false;
-        for (int u = blockIdx.x; u < p.total_units; u += gridDim.x) {
+        for (int uj = 0; uj < sc.n_units; ++uj) {
+            const int u = sc.unit(uj);
             if (cta_aborted(abort)) break;
-            const Unit t = decode_unit(p, u, &tmap_q);
+            const Unit t = decode_unit(p, u, &tmap_q, sc);
             const uint32_t q_off = (uint32_t)((t.tq * BN) % 128) / 32;
             if ((q_off & 1) != 0 || q_off * 32 + (BN < 32 ? 32 : BN) > 128 * S::kQChunks) {
                 // never planned: a scale-factor column offset the MMA is not given
@@ -597,7 +718,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 ptx::tc_fence_after();
                 const uint32_t sf_base = tmem + S::kSfBase + stage * S::kSfCols;
                 const uint64_t adesc = ptx::smem_desc_sw128(ptx::smem_u32(smem + L::kOffP + stage * S::kPTileBytes));
-                const uint64_t bdesc = ptx::smem_desc_sw128(ptx::smem_u32(smem + L::kOffQ + stage * S::kQTileBytes));
+                const uint64_t bdesc = ptx::smem_desc_sw128(ptx::smem_u32(
+                    FUSED ? smem + L::kOffPersist + kt * S::kQTileBytes : smem + L::kOffQ + stage * S::kQTileBytes));
                 if (leader) {
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk) {
@@ -646,8 +768,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         int stage = 0;
         uint32_t phase = 0;
         uint32_t kt_count = 0;
-        for (int u = blockIdx.x; u < p.total_units && !*abort; u += gridDim.x) {
-            const Unit t = decode_unit(p, u, &tmap_q);
+        for (int uj = 0; uj < sc.n_units && !*abort; ++uj) {
+            const int u = sc.unit(uj);
+            const Unit t = decode_unit(p, u, &tmap_q, sc);
             bool ok = true;
             for (int kt = t.kt_begin; kt < t.kt_end; ++kt, ++kt_count) {
                 // Every set waits for every fill, in order, even those it does not
@@ -665,7 +788,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 const uint32_t col = lane_base + S::kSfBase + stage * S::kSfCols;
                 const uint32_t sfp_s = ptx::smem_u32(smem + L::kOffSfP + stage * S::kSfChunkBytes) + lane * 16;
                 const uint32_t sfq_s =
-                    ptx::smem_u32(smem + L::kOffSfQ + stage * S::kQChunks * S::kSfChunkBytes) + lane * 16;
+                    ptx::smem_u32(FUSED ? smem + L::kOffPersist + p.k_tiles * S::kQTileBytes + kt * S::kSfChunkBytes
+                                        : smem + L::kOffSfQ + stage * S::kQChunks * S::kSfChunkBytes) +
+                    lane * 16;
 #pragma unroll
                 for (int a = 0; a < 2; ++a) {
                     ptx::tmem_st_32x32b_x1(col + 4 * a + quad, ptx::lds32(sfp_s + 512 * a + 4 * quad));
@@ -692,42 +817,27 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         constexpr int NCH = BN / CW;
         const bool via_tma = S::kStagingBytes > 0 && p.tma_store;
         const uint32_t staging = ptx::smem_u32(smem + L::kOffStaging) + quad * S::kStageBoxBytes;
-        bool zeroed = false;
-        if (p.atomic || p.fused) {
-            const int et = threadIdx.x - 64;                     // 0..127 over warps 2-5
-            if (p.atomic) {
-                // zero this CTA's slice of the split-K accumulator
-                const int64_t per = (p.zero_vec4 + gridDim.x - 1) / gridDim.x;
-                const int64_t b0 = (int64_t)blockIdx.x * per, b1 = min(p.zero_vec4, b0 + per);
-                float4* z = reinterpret_cast<float4*>(p.out);
-                for (int64_t i = b0 + et; i < b1; i += 128) z[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-            }
-            if (p.fused) fused_quant_share(p, et);
-            ptx::fence_proxy_async_global();
-            __threadfence();
-            asm volatile("bar.sync 1, 128;" ::: "memory");
-            if (et == 0) st_release_u64(p.cta_flags + blockIdx.x, p.epoch);
-        }
-        for (int u = blockIdx.x; u < p.total_units && !*abort; u += gridDim.x) {
-            const Unit t = decode_unit(p, u, &tmap_q);
-            if (!wait_or_abort(&acc_full[acc], acc_phase, abort, p.err, kErrTimeoutEpilogue)) break;
+        volatile int* sk_last = reinterpret_cast<volatile int*>(smem + L::kOffMisc + 8);
+        constexpr bool kSkWidth = BN <= 64 && !GATHER;
+        // The four epilogue warps leave the loop together: a stream-K tile synchronises
+        // them on a named barrier, which a warp that had left alone would hold forever.
+        for (int uj = 0; uj < sc.n_units; ++uj) {
+            const int u = sc.unit(uj);
+            const Unit t = decode_unit(p, u, &tmap_q, sc);
+            if (!bar_and(1, 128, wait_or_abort(&acc_full[acc], acc_phase, abort, p.err, kErrTimeoutEpilogue))) break;
             ptx::tc_fence_after();
             const int prow = t.out_row0 + quad * 32 + lane;      // output row (transposed: column)
             const bool row_ok = quad * 32 + lane < t.rows;
             const uint32_t taddr = tmem + acc * S::kAccStride + ((uint32_t)(quad * 32) << 16);
-            if (p.atomic && !zeroed) {
-                // once per kernel: every CTA has zeroed its slice of the accumulator
-                bool ok = true;
-                for (int i = lane; i < (int)gridDim.x && ok; i += 32)
-                    ok = wait_split_flag(p.cta_flags + i, p.epoch, abort, p.err);
-                if (!__all_sync(0xffffffffu, ok)) break;
-                zeroed = true;
-            }
+            // stream-K (planned for decode tiles of width <= 64 only): this CTA holds only
+            // part of the tile's K range
+            const bool partial = kSkWidth && (t.kt_begin > 0 || t.kt_end < p.k_tiles);
             // write chunk c of y from registers: staged TMA store or direct stores
             auto emit = [&](int c, uint32_t (&r)[CW]) {
                 if constexpr (GATHER) {
                     for (int d = 0; d < p.n_dest; ++d)
-                        store_chunk<CW>(p, reinterpret_cast<void*>(p.dest[d]), prow, row_ok, t.tq * BN + c * CW, r);
+                        store_chunk<CW>(p, reinterpret_cast<void*>(p.dest[d]), p.ldo, p.q_rows, prow, row_ok,
+                                        t.tq * BN + c * CW, r);
                     return;
                 }
                 if constexpr (S::kStagingBytes > 0) {
@@ -772,8 +882,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         return;
                     }
                 }
-                store_chunk<CW>(p, p.out, prow, row_ok, t.tq * BN + c * CW, r);
+                store_chunk<CW>(p, t.out, t.ldo, t.q_rows, prow, row_ok, t.tq * BN + c * CW, r);
             };
+            // this thread's row of the CTA's partial-tile slot (the first or the last tile of
+            // its stream-K range)
+            const int64_t slot_row = ((int64_t)blockIdx.x * 2 + (u == sc.sk_first ? 0 : 1)) * (128 * BN) +
+                                     (int64_t)(quad * 32 + lane) * BN;
 #pragma unroll 1
             for (int c = 0; c < NCH; ++c) {
                 uint32_t r[CW];
@@ -796,7 +910,65 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     __syncwarp();
                     if (lane == 0) ptx::mbar_arrive(&acc_empty[acc]);
                 }
-                emit(c, r);
+                if (!partial) {
+                    emit(c, r);
+                } else {
+                    float4* dst = reinterpret_cast<float4*>(p.sk_partials + slot_row + c * CW);
+#pragma unroll
+                    for (int j = 0; j < CW; j += 4)
+                        dst[j / 4] = make_float4(__uint_as_float(r[j]), __uint_as_float(r[j + 1]),
+                                                 __uint_as_float(r[j + 2]), __uint_as_float(r[j + 3]));
+                }
+            }
+            if constexpr (kSkWidth) if (partial) {
+                // Count the CTA in once all four warps' rows are written; the arrival that
+                // completes the count finishes the tile.
+                const int64_t t0 = (int64_t)(u - p.sk_tile0) * p.k_tiles;
+                const int c_lo = sk_cta_of(p, t0), c_hi = sk_cta_of(p, t0 + p.k_tiles - 1);
+                __threadfence();
+                asm volatile("bar.sync 1, 128;" ::: "memory");
+                if (threadIdx.x == 64)
+                    *sk_last = sk_arrive(p.sk_counters + u, p.sk_tag) == (uint32_t)(c_hi - c_lo + 1) ? 1 : 0;
+                asm volatile("bar.sync 1, 128;" ::: "memory");
+                if (*sk_last) {
+                    __threadfence();
+                    // y = the contributors' partial tiles added in the order of their K
+                    // ranges, 16 columns at a time; the loads of two contributors are issued
+                    // together (decode tiles: transposed direct stores)
+                    const int64_t row_off = (int64_t)(quad * 32 + lane) * BN;
+#pragma unroll 1
+                    for (int c16 = 0; c16 < BN / 16; ++c16) {
+                        uint32_t r[16];
+#pragma unroll 1
+                        for (int k0 = c_lo; k0 <= c_hi; k0 += 2) {
+                            float4 v[2][4];
+#pragma unroll
+                            for (int g = 0; g < 2; ++g) {
+                                const int k = k0 + g;
+                                if (k <= c_hi) {
+                                    const int slot = u == p.sk_tile0 + (int)(sk_start(p, k) / p.k_tiles) ? 0 : 1;
+                                    const float4* src = reinterpret_cast<const float4*>(
+                                        p.sk_partials + ((int64_t)k * 2 + slot) * (128 * BN) + row_off + c16 * 16);
+#pragma unroll
+                                    for (int j = 0; j < 4; ++j) v[g][j] = __ldcg(src + j);
+                                }
+                            }
+#pragma unroll
+                            for (int g = 0; g < 2; ++g) {
+                                if (k0 + g > c_hi) break;
+#pragma unroll
+                                for (int j = 0; j < 4; ++j) {
+                                    const float f[4] = {v[g][j].x, v[g][j].y, v[g][j].z, v[g][j].w};
+#pragma unroll
+                                    for (int e = 0; e < 4; ++e)
+                                        r[4 * j + e] = k0 + g == c_lo ? __float_as_uint(f[e])
+                                                                      : __float_as_uint(__fadd_rn(__uint_as_float(r[4 * j + e]), f[e]));
+                                }
+                            }
+                        }
+                        store_chunk<16>(p, t.out, t.ldo, t.q_rows, prow, row_ok, t.tq * BN + c16 * 16, r);
+                    }
+                }
             }
             if (S::kNumAcc == 2) {
                 acc ^= 1;

@@ -83,7 +83,6 @@ inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 // Limits that keep every index inside 32 bits where the kernels use int.
 constexpr int64_t kMaxRows = (int64_t)1 << 30;
 constexpr int64_t kMaxK = (int64_t)1 << 24;
-constexpr int kMaxGatherDest = 64;                 // destinations of a gathered output
 constexpr int64_t kMaxFlipK = 8192;     // Flip-Refinement keeps a row's gradient in shared memory
 
 // --------------------------------------------------------------------- quant ---
@@ -205,22 +204,25 @@ struct GemmPlan {
     bool swap;        // P = weight, Q = activations, output written transposed
     int bn;
     int tiles_p, tiles_q, k_tiles;
-    int splits, kps;
+    int sk_tile0;     // tiles below are whole units dealt round robin; the rest stream-K
+    int64_t sk_iters; // K tiles of the stream-K tiles
+    int sk_ctas;      // CTAs that share them (<= sk_iters)
     int group_p;
     int grid;
+    bool sk() const { return sk_iters > 0; }
 };
 
 // Estimated SM cycles per 256-wide K tile of a 128 x bn tile: the four MMAs take about
 // 2.4 bn cycles at the measured tensor rate, and a K tile costs ~400 cycles of copies,
 // barriers and issue however narrow it is.
 inline double ktile_cycles(int bn) { return std::max(400.0, 2.42 * bn); }
-// Extra cost of splitting K: zeroing the accumulator and the finalize kernel that
-// converts it (~4 us), plus the fp32 reductions of every unit's 128 x bn tile, which
-// L2 absorbs at an estimated 800 bytes per cycle.
-constexpr double kSplitCycles = 8000.0;
-constexpr double kReduceBytesPerCycle = 800.0;
 
-GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, int num_sms) {
+// Stream-K (decode orientation): a CTA takes at least this many K tiles, and a tile is
+// shared by at most this many CTAs (its finisher reads every contributor's partial).
+constexpr int64_t kSkMinIters = 3;
+constexpr int64_t kSkMaxContributors = 8;
+
+GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, int num_sms, bool allow_sk = true) {
     GemmPlan best{};
     double best_cost = 0.0;
     const int k_tiles = (int)cdiv(K, 256);
@@ -245,66 +247,72 @@ GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, int num_sms) {
         g.tiles_p = (int)cdiv(swap ? N : M, 128);
         g.tiles_q = (int)cdiv(swap ? M : N, g.bn);
         const int64_t tiles = (int64_t)g.tiles_p * g.tiles_q;
-        // time = rounds of units over the SMs x K tiles per unit x cycles per K tile,
-        // plus the cost of splitting; K tiles per unit stay >= 2
-        const int max_splits = std::max(1, k_tiles / 2);
-        for (int s = 1; s <= max_splits; ++s) {
-            const int kps = (int)cdiv(k_tiles, s);
-            const int splits = (int)cdiv(k_tiles, kps);
-            if (splits != s) continue;
-            if (splits > 1 && M > 65535) break;        // the finalize grid has one row per block row
-            const int64_t units = tiles * splits;
-            const double cost =
-                (double)cdiv(units, num_sms) * kps * ktile_cycles(g.bn) +
-                (splits > 1 ? kSplitCycles + (double)units * 128 * g.bn * 4 / kReduceBytesPerCycle : 0.0);
-            if (best.bn == 0 || cost < best_cost * 0.98) {
-                best = g;
-                best.splits = splits;
-                best.kps = kps;
-                best_cost = cost;
-            }
+        // time = rounds of tiles over the SMs x K tiles per tile x cycles per K tile
+        const double cost = (double)cdiv(tiles, num_sms) * k_tiles * ktile_cycles(g.bn);
+        g.sk_tile0 = (int)tiles;
+        g.sk_iters = 0;
+        g.grid = (int)std::min<int64_t>(tiles, num_sms);
+        if (best.bn == 0 || cost < best_cost * 0.98) {
+            best = g;
+            best_cost = cost;
+        }
+    }
+    // Decode: a weight-streaming product whose last round of tiles would leave SMs idle.
+    // Every CTA takes an even share of that round's K tiles first (stream-K), then its
+    // whole tiles; with fewer tiles than SMs, every tile is shared.
+    const int64_t tiles = (int64_t)best.tiles_p * best.tiles_q;
+    if (allow_sk && best.swap && best.bn <= 64 && tiles % num_sms != 0 && best.k_tiles >= 2) {
+        const int64_t whole_rounds = tiles / num_sms;
+        const int64_t rest = tiles - whole_rounds * num_sms;
+        int64_t grid = num_sms;
+        if (whole_rounds == 0)
+            grid = std::max<int64_t>(1, std::min<int64_t>({(int64_t)num_sms, tiles * best.k_tiles / kSkMinIters,
+                                                           tiles * kSkMaxContributors}));
+        if (grid > 1 && (whole_rounds > 0 || grid > tiles)) {
+            best.sk_tile0 = (int)(whole_rounds * num_sms);
+            best.sk_iters = rest * best.k_tiles;
+            best.grid = (int)grid;
+            best.sk_ctas = (int)std::min<int64_t>(grid, best.sk_iters);
         }
     }
     best.group_p = std::min(best.tiles_p, 16);
-    best.grid = (int)std::min<int64_t>((int64_t)best.tiles_p * best.tiles_q * best.splits, num_sms);
     return best;
 }
 
-// Row stride (elements) of the fp32 split-K accumulator: a multiple of 4 so that the
-// epilogue's 16-byte vector reductions stay aligned.
-inline int64_t acc_ld(int64_t N) { return round_up(N, 4); }
-
-// Split-K workspace: the fp32 accumulator (M x acc_ld(N)), then one 8-byte flag per CTA.
-struct SplitWorkspace {
-    size_t acc_bytes, flag_bytes;
+// Stream-K workspace: two fp32 partial tiles per CTA (128 x bn each), then one 8-byte
+// counter per tile.
+struct SkWorkspace {
+    size_t partial_bytes, counter_bytes;
 };
-SplitWorkspace split_workspace(const GemmPlan& g, int64_t M, int64_t N) {
-    SplitWorkspace w{0, 0};
-    if (g.splits > 1) {
-        w.acc_bytes = (size_t)round_up(M * acc_ld(N) * 4, 256);
-        w.flag_bytes = (size_t)round_up((int64_t)g.grid * 8, 256);
+SkWorkspace sk_workspace(const GemmPlan& g) {
+    SkWorkspace w{0, 0};
+    if (g.sk()) {
+        w.partial_bytes = (size_t)round_up((int64_t)g.grid * 2 * 128 * g.bn * 4, 256);
+        w.counter_bytes = (size_t)round_up((int64_t)g.tiles_p * g.tiles_q * 8, 256);
     }
     return w;
 }
 
 size_t gemm_workspace(int64_t M, int64_t N, int64_t K, int num_sms) {
-    const SplitWorkspace w = split_workspace(plan_gemm(M, N, K, num_sms), M, N);
-    return w.acc_bytes + w.flag_bytes;
+    const SkWorkspace w = sk_workspace(plan_gemm(M, N, K, num_sms));
+    return w.partial_bytes + w.counter_bytes;
 }
 
-// Split-K flags are set to a value unique to each call, so a flag left by an earlier
-// call (or whatever the workspace held) is never taken for a fresh one: 32 bits of a
-// per-process salt from the clock, then a call counter.
-unsigned long long next_epoch() {
+// Stream-K counters carry a 48-bit tag unique to each call, so a count left by an
+// earlier call (or whatever the workspace held) is never taken for a fresh one: a
+// per-process salt from the clock and a call counter, mixed.
+unsigned long long next_sk_tag() {
     static std::atomic<unsigned long long> counter{0};
     static const unsigned long long salt = [] {
         unsigned long long t = (unsigned long long)std::chrono::steady_clock::now().time_since_epoch().count();
         t ^= t >> 33;
         t *= 0xff51afd7ed558ccdull;
         t ^= t >> 33;
-        return (t | 1ull) << 32;
+        return t;
     }();
-    return salt + counter.fetch_add(1) + 1;
+    unsigned long long v = salt + 0x9e3779b97f4a7c15ull * (counter.fetch_add(1) + 1);
+    v ^= v >> 29;
+    return v & 0xFFFFFFFFFFFFull;
 }
 
 bool encode_codes_map(CUtensorMap* map, const uint8_t* codes, int64_t rows, int64_t K, int box_rows) {
@@ -333,57 +341,37 @@ bool encode_out_map(CUtensorMap* map, void* y, int64_t M, int64_t N, int64_t ldy
     return r == CUDA_SUCCESS;
 }
 
-template <int BN, int STAGES, bool GATHER = false>
+// Largest dynamic shared memory of a CTA on sm_100.
+constexpr int kMaxSmem = 232448;
+
+template <int BN, int STAGES, int VAR = kVarPlain>
 macaq_status launch_gemm_bn(const CUtensorMap& mp, const CUtensorMap& mq, const CUtensorMap& my,
                             const GemmParams& gp, int grid, cudaStream_t stream) {
-    using L = GemmSmem<BN, STAGES>;
-    static_assert(L::kAlloc <= 232448, "shared memory budget");
+    using L = GemmSmem<BN, STAGES, VAR == kVarFused>;
+    static_assert(L::kAlloc <= kMaxSmem, "shared memory budget");
+    const int smem = L::alloc(gp.k_tiles);
+    if (smem > kMaxSmem) return MACAQ_ERR_UNSUPPORTED_SHAPE;
     static std::atomic<uint64_t> configured_mask{0};
     int dev = 0;
     cudaGetDevice(&dev);
     const uint64_t bit = 1ull << (dev & 63);
     if (!(configured_mask.load() & bit)) {
-        if (cudaFuncSetAttribute(gemm_mxf4_kernel<BN, STAGES, GATHER>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc) != cudaSuccess)
+        if (cudaFuncSetAttribute(gemm_mxf4_kernel<BN, STAGES, VAR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 VAR == kVarFused ? kMaxSmem : L::kAlloc) != cudaSuccess)
             return MACAQ_ERR_CUDA;
         configured_mask.fetch_or(bit);
     }
-    return launch_pdl(gemm_mxf4_kernel<BN, STAGES, GATHER>, dim3(grid), dim3(kGemmThreads), L::kAlloc, stream, mp, mq, my,
-                      gp) ==
-                   cudaSuccess
+    return launch_pdl(gemm_mxf4_kernel<BN, STAGES, VAR>, dim3(grid), dim3(kGemmThreads), (size_t)smem, stream, mp, mq,
+                      my, gp) == cudaSuccess
                ? MACAQ_OK
                : MACAQ_ERR_CUDA;
 }
 
-// Split K: converts the fp32 accumulator (row stride lda, a multiple of 4) into y, four
-// columns per thread; blockIdx.y is the row (split-K products have few rows).
-__global__ void finalize_kernel(const float* __restrict__ acc, int64_t lda, int N, void* y, int64_t ldy, int bf16,
-                                int vec) {
-    ptx::griddep_wait();
-    ptx::griddep_launch_dependents();
-    const int n = (blockIdx.x * blockDim.x + threadIdx.x) * 4;
-    if (n >= N) return;
-    const int64_t m = blockIdx.y;
-    const float4 v = *reinterpret_cast<const float4*>(acc + m * lda + n);
-    const float f[4] = {v.x, v.y, v.z, v.w};
-    if (bf16) {
-        __nv_bfloat16* o = static_cast<__nv_bfloat16*>(y) + m * ldy + n;
-        if (vec && n + 4 <= N) {
-            __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y), hi = __floats2bfloat162_rn(v.z, v.w);
-            uint2 w;
-            w.x = *reinterpret_cast<uint32_t*>(&lo);
-            w.y = *reinterpret_cast<uint32_t*>(&hi);
-            *reinterpret_cast<uint2*>(o) = w;
-        } else {
-            for (int j = 0; j < 4 && n + j < N; ++j) o[j] = __float2bfloat16_rn(f[j]);
-        }
-    } else {
-        float* o = static_cast<float*>(y) + m * ldy + n;
-        if (vec && n + 4 <= N)
-            *reinterpret_cast<float4*>(o) = v;
-        else
-            for (int j = 0; j < 4 && n + j < N; ++j) o[j] = f[j];
-    }
+// Whether the fused variant's persistent Q operand (every K tile of a bn-row tile) fits
+// in shared memory beside its weight ring.
+bool fused_fits(int bn, int k_tiles) {
+    return bn == 16 ? GemmSmem<16, 8, true>::alloc(k_tiles) <= kMaxSmem
+                    : GemmSmem<32, 6, true>::alloc(k_tiles) <= kMaxSmem;
 }
 
 macaq_status check_weight(const macaq_weight* w) {
@@ -394,25 +382,22 @@ macaq_status check_weight(const macaq_weight* w) {
     return MACAQ_OK;
 }
 
-// Activation transform fused into the GEMM kernel: the kernel quantises x (with w's
-// inv_s) into a_codes / a_scales itself before it loads them; `flags` holds one 8-byte
-// flag per CTA.
+// Activation transform fused into the GEMM kernel (decode): every CTA makes the MXFP4
+// form of the whole activation (at most 32 rows) in shared memory before its main loop.
 struct FusedAct {
     const void* x;
     int64_t ldx;
-    unsigned long long* flags;
 };
-constexpr size_t kFusedFlagBytes = 8192;                 // up to 1024 CTAs
-// Largest M the fused transform takes (decode): every CTA then quantises a small share,
-// one 128-row slab of blocks in all, while the weight tiles stream in. Larger M runs the
-// transform as its own kernel, which uses every thread of the GPU for it.
-constexpr int64_t kFusedMaxRows = 128;
+// Largest M the fused transform takes: the activation's MXFP4 form for every K tile
+// stays in shared memory beside the weight ring (one 16- or 32-row tile); larger M, or a
+// K whose tiles do not fit, runs the transform as its own kernel.
+constexpr int64_t kFusedMaxRows = 32;
 
 // Output written to several destinations (the gathered output of a column-parallel
 // layer): a device table of destination addresses, and whether all of them allow
 // 16-byte vector stores.
 struct GatherOut {
-    const unsigned long long* dest;
+    const uint64_t* dest;          // host array, copied into the kernel's parameters
     int n;
     bool vec_ok;
 };
@@ -426,12 +411,7 @@ macaq_status run_gemm(const uint8_t* a_codes, const uint8_t* a_scales, int64_t M
     if (st != MACAQ_OK) return st;
     const int64_t N = w->N, K = w->K;
     GemmPlan g = plan_gemm(M, N, K, dev->num_sms);
-    if (go && g.splits > 1) {
-        // a gathered output is written by the GEMM's own epilogue: no split K
-        g.splits = 1;
-        g.kps = g.k_tiles;
-        g.grid = (int)std::min<int64_t>((int64_t)g.tiles_p * g.tiles_q, dev->num_sms);
-    }
+    if (go && g.sk()) g = plan_gemm(M, N, K, dev->num_sms, false);   // a gathered output: one CTA per tile
     const size_t need = gemm_workspace(M, N, K, dev->num_sms);
     if (need > 0 && (workspace == nullptr || ws_bytes < need)) return MACAQ_ERR_WORKSPACE;
     if (need > 0 && (reinterpret_cast<uintptr_t>(workspace) & 255) != 0) return MACAQ_ERR_MISALIGNED;
@@ -453,58 +433,40 @@ macaq_status run_gemm(const uint8_t* a_codes, const uint8_t* a_scales, int64_t M
     gp.kb4_pad = (int32_t)(round_up(K / 32, 8) / 4);
     gp.tiles_p = g.tiles_p;
     gp.tiles_q = g.tiles_q;
-    gp.splits = g.splits;
-    gp.k_tiles_per_split = g.kps;
-    gp.total_units = g.tiles_p * g.tiles_q * g.splits;
+    gp.total_units = g.tiles_p * g.tiles_q;
     gp.group_p = g.group_p;
     gp.transpose_out = g.swap ? 1 : 0;
     gp.err = dev->err_ptr;
     const int64_t esz = out == MACAQ_OUT_BF16 ? 2 : 4;
-    const int y_vec = (aligned16(y) && (ldy * esz) % 16 == 0) ? 1 : 0;
-    if (g.splits > 1) {
-        // fp32 reductions into the workspace accumulator, zeroed by the kernel itself
-        const SplitWorkspace sw = split_workspace(g, M, N);
-        gp.out = workspace;
-        gp.ldo = acc_ld(N);
-        gp.atomic = 1;
-        gp.out_bf16 = 0;
-        gp.vec_ok = 1;
+    gp.out = y;
+    gp.ldo = ldy;
+    gp.out_bf16 = out == MACAQ_OUT_BF16 ? 1 : 0;
+    gp.vec_ok = (aligned16(y) && (ldy * esz) % 16 == 0) ? 1 : 0;
+    // wide row-major tiles store through TMA (an aligned output is all it needs)
+    gp.tma_store = (!g.swap && g.bn >= 128 && gp.vec_ok) ? 1 : 0;
+    if (go) {
+        gp.n_dest = go->n;
+        for (int d = 0; d < go->n; ++d) gp.dest[d] = go->dest[d];
+        gp.vec_ok = go->vec_ok ? 1 : 0;
         gp.tma_store = 0;
-        gp.zero_vec4 = M * acc_ld(N) * 4 / 16;
-        gp.cta_flags = reinterpret_cast<unsigned long long*>(static_cast<uint8_t*>(workspace) + sw.acc_bytes);
-        gp.epoch = next_epoch();
-    } else {
-        gp.out = y;
-        gp.ldo = ldy;
-        gp.atomic = 0;
-        gp.out_bf16 = out == MACAQ_OUT_BF16 ? 1 : 0;
-        gp.vec_ok = y_vec;
-        // wide row-major tiles store through TMA (an aligned output is all it needs)
-        gp.tma_store = (!g.swap && g.bn >= 128 && gp.vec_ok) ? 1 : 0;
-        if (go) {
-            gp.n_dest = go->n;
-            gp.dest = go->dest;
-            gp.vec_ok = go->vec_ok ? 1 : 0;
-            gp.tma_store = 0;
-        }
     }
-    int grid = g.grid;
+    gp.sk_tile0 = g.sk_tile0;
+    gp.sk_iters = g.sk_iters;
+    gp.sk_ctas = g.sk_ctas;
+    if (g.sk()) {
+        const SkWorkspace sw = sk_workspace(g);
+        gp.sk_partials = static_cast<float*>(workspace);
+        gp.sk_counters = reinterpret_cast<unsigned long long*>(static_cast<uint8_t*>(workspace) + sw.partial_bytes);
+        gp.sk_tag = next_sk_tag();
+    }
+    const int grid = g.grid;
     if (fa) {
-        // one CTA per SM however few tiles there are: CTAs without a unit still take
-        // their share of the activation transform
-        grid = dev->num_sms;
-        if ((size_t)grid * 8 > kFusedFlagBytes) return MACAQ_ERR_UNSUPPORTED_SHAPE;
-        gp.fused = 1;
+        // decode orientation only, one activation tile held whole in shared memory
+        if (!g.swap || g.tiles_q != 1 || g.bn > 32 || !fused_fits(g.bn, g.k_tiles)) return MACAQ_ERR_UNSUPPORTED_SHAPE;
         gp.fx = static_cast<const uint16_t*>(fa->x);
         gp.fx_ld = fa->ldx;
         gp.f_mult = w->inv_s;
-        gp.f_codes = const_cast<uint8_t*>(a_codes);
-        gp.f_scales = const_cast<uint8_t*>(a_scales);
-        gp.f_rows = (int32_t)M;
         gp.f_K = (int32_t)K;
-        gp.f_kb_pad = (int32_t)round_up(K / 32, 8);
-        gp.cta_flags = fa->flags;              // also the split-K zeroing flags
-        if (gp.epoch == 0) gp.epoch = next_epoch();
     }
     CUtensorMap my;
     std::memset(&my, 0, sizeof(my));
@@ -512,29 +474,27 @@ macaq_status run_gemm(const uint8_t* a_codes, const uint8_t* a_scales, int64_t M
 
     if (go) {
         switch (g.bn) {
-            case 16: st = launch_gemm_bn<16, 8, true>(mp, mq, my, gp, grid, stream); break;
-            case 32: st = launch_gemm_bn<32, 8, true>(mp, mq, my, gp, grid, stream); break;
-            case 64: st = launch_gemm_bn<64, 8, true>(mp, mq, my, gp, grid, stream); break;
-            case 128: st = launch_gemm_bn<128, 6, true>(mp, mq, my, gp, grid, stream); break;
-            default: st = launch_gemm_bn<192, 5, true>(mp, mq, my, gp, grid, stream); break;
+            case 16: st = launch_gemm_bn<16, 8, kVarGather>(mp, mq, my, gp, grid, stream); break;
+            case 32: st = launch_gemm_bn<32, 8, kVarGather>(mp, mq, my, gp, grid, stream); break;
+            case 64: st = launch_gemm_bn<64, 8, kVarGather>(mp, mq, my, gp, grid, stream); break;
+            case 128: st = launch_gemm_bn<128, 6, kVarGather>(mp, mq, my, gp, grid, stream); break;
+            default: st = launch_gemm_bn<192, 5, kVarGather>(mp, mq, my, gp, grid, stream); break;
         }
         return st;
     }
-    switch (g.bn) {
-        case 16: st = launch_gemm_bn<16, 8>(mp, mq, my, gp, grid, stream); break;
-        case 32: st = launch_gemm_bn<32, 8>(mp, mq, my, gp, grid, stream); break;
-        case 64: st = launch_gemm_bn<64, 8>(mp, mq, my, gp, grid, stream); break;
-        case 128: st = launch_gemm_bn<128, 6>(mp, mq, my, gp, grid, stream); break;
-        default: st = launch_gemm_bn<192, 5>(mp, mq, my, gp, grid, stream); break;
+    if (fa) {
+        st = g.bn == 16 ? launch_gemm_bn<16, 8, kVarFused>(mp, mq, my, gp, grid, stream)
+                        : launch_gemm_bn<32, 6, kVarFused>(mp, mq, my, gp, grid, stream);
+    } else {
+        switch (g.bn) {
+            case 16: st = launch_gemm_bn<16, 8>(mp, mq, my, gp, grid, stream); break;
+            case 32: st = launch_gemm_bn<32, 8>(mp, mq, my, gp, grid, stream); break;
+            case 64: st = launch_gemm_bn<64, 8>(mp, mq, my, gp, grid, stream); break;
+            case 128: st = launch_gemm_bn<128, 6>(mp, mq, my, gp, grid, stream); break;
+            default: st = launch_gemm_bn<192, 5>(mp, mq, my, gp, grid, stream); break;
+        }
     }
-    if (st != MACAQ_OK || g.splits == 1) return st;
-    // split K (planned only for M <= 65535, never with a gathered output): one grid row
-    // per output row
-    const dim3 fgrid((unsigned)cdiv(cdiv(N, 4), 256), (unsigned)M);
-    if (launch_pdl(finalize_kernel, fgrid, dim3(256), 0, stream, static_cast<const float*>(workspace), acc_ld(N),
-                   (int)N, y, ldy, out == MACAQ_OUT_BF16 ? 1 : 0, y_vec) != cudaSuccess)
-        return MACAQ_ERR_CUDA;
-    return MACAQ_OK;
+    return st;
 }
 
 macaq_status check_gemm_args(int64_t M, const macaq_weight* w, const void* y, int64_t ldy,
@@ -575,22 +535,21 @@ size_t macaq_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, macaq_out_dty
     return gemm_workspace(M, N, K, sms);
 }
 
-// macaq_linear_w4a4's workspace: activation codes | scales | per-CTA flags of the fused
-// transform | the GEMM's own workspace, each 256-byte aligned.
+// macaq_linear_w4a4's workspace: activation codes | scales | the GEMM's own workspace,
+// each 256-byte aligned.
 static size_t linear_ws_parts(int64_t M, int64_t N, int64_t K, macaq_out_dtype out, size_t* off_scales,
-                              size_t* off_flags, size_t* off_gemm) {
+                              size_t* off_gemm) {
     const size_t codes = (size_t)round_up((int64_t)macaq_codes_bytes(M, K), 256);
     const size_t scales = (size_t)round_up((int64_t)macaq_scales_bytes(M, K), 256);
     *off_scales = codes;
-    *off_flags = codes + scales;
-    *off_gemm = codes + scales + kFusedFlagBytes;
+    *off_gemm = codes + scales;
     return *off_gemm + macaq_gemm_workspace_bytes(M, N, K, out);
 }
 
 size_t macaq_linear_workspace_bytes(int64_t M, int64_t N, int64_t K, macaq_out_dtype out) {
     if (M < 1 || N < 1 || K < 32) return 0;
-    size_t a, b, c;
-    return linear_ws_parts(M, N, K, out, &a, &b, &c);
+    size_t a, b;
+    return linear_ws_parts(M, N, K, out, &a, &b);
 }
 
 macaq_status macaq_prepare_weight(const void* W_bf16, int64_t N, int64_t K, int64_t ldw, const float* s,
@@ -629,16 +588,17 @@ macaq_status macaq_linear_w4a4(const void* x_bf16, int64_t M, int64_t ldx, const
     if (!w->inv_s) return MACAQ_ERR_INVALID_ARG;
     st = check_quant_args(x_bf16, M, w->K, ldx, w->inv_s, w->codes, w->scales);
     if (st != MACAQ_OK) return st;
-    size_t off_scales, off_flags, off_gemm;
-    const size_t need = linear_ws_parts(M, w->N, w->K, out, &off_scales, &off_flags, &off_gemm);
+    size_t off_scales, off_gemm;
+    const size_t need = linear_ws_parts(M, w->N, w->K, out, &off_scales, &off_gemm);
     if (!workspace || ws_bytes < need) return MACAQ_ERR_WORKSPACE;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255) != 0) return MACAQ_ERR_MISALIGNED;
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     uint8_t* a_codes = ws;
     uint8_t* a_scales = ws + off_scales;
-    if (fused == 1 && M <= kFusedMaxRows) {
-        // one launch: the GEMM kernel quantises the activations itself
-        const FusedAct fa{x_bf16, ldx, reinterpret_cast<unsigned long long*>(ws + off_flags)};
+    if (fused == 1 && M <= kFusedMaxRows && fused_fits(M <= 16 ? 16 : 32, (int)cdiv(w->K, 256))) {
+        // one launch: the GEMM kernel makes the MXFP4 activations in shared memory itself
+        // (the activation part of the workspace is not touched)
+        const FusedAct fa{x_bf16, ldx};
         return run_gemm(a_codes, a_scales, M, w, y, ldy, out, ws + off_gemm, ws_bytes - off_gemm,
                         (cudaStream_t)stream, &fa);
     }
@@ -649,7 +609,7 @@ macaq_status macaq_linear_w4a4(const void* x_bf16, int64_t M, int64_t ldx, const
 
 size_t macaq_linear_gather_workspace_bytes(int64_t M, int64_t N, int64_t K, macaq_out_dtype out) {
     const size_t lin = macaq_linear_workspace_bytes(M, N, K, out);
-    return lin == 0 ? 0 : lin + (size_t)round_up(kMaxGatherDest * 8, 256);
+    return lin;
 }
 
 macaq_status macaq_linear_w4a4_gather(const void* x_bf16, int64_t M, int64_t ldx, const macaq_weight* w,
@@ -666,21 +626,15 @@ macaq_status macaq_linear_w4a4_gather(const void* x_bf16, int64_t M, int64_t ldx
     if (!w->inv_s) return MACAQ_ERR_INVALID_ARG;
     macaq_status st = check_quant_args(x_bf16, M, w->K, ldx, w->inv_s, w->codes, w->scales);
     if (st != MACAQ_OK) return st;
-    size_t off_scales, off_flags, off_gemm;
-    const size_t lin = linear_ws_parts(M, w->N, w->K, out, &off_scales, &off_flags, &off_gemm);
+    size_t off_scales, off_gemm;
+    const size_t lin = linear_ws_parts(M, w->N, w->K, out, &off_scales, &off_gemm);
     const size_t need = macaq_linear_gather_workspace_bytes(M, w->N, w->K, out);
     if (!workspace || ws_bytes < need) return MACAQ_ERR_WORKSPACE;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255) != 0) return MACAQ_ERR_MISALIGNED;
     uint8_t* ws = static_cast<uint8_t*>(workspace);
-    // the destination table goes after the layer's own workspace (a copy from pageable
-    // host memory waits for the stream's earlier work)
-    unsigned long long* table = reinterpret_cast<unsigned long long*>(ws + lin);
-    if (cudaMemcpyAsync(table, dest, (size_t)n_dest * 8, cudaMemcpyHostToDevice, (cudaStream_t)stream) !=
-        cudaSuccess)
-        return MACAQ_ERR_CUDA;
     st = launch_quant(x_bf16, M, w->K, ldx, w->inv_s, ws, ws + off_scales, nullptr, nullptr, (cudaStream_t)stream);
     if (st != MACAQ_OK) return st;
-    const GatherOut go{table, n_dest, vec};
+    const GatherOut go{dest, n_dest, vec};
     return run_gemm(ws, ws + off_scales, M, w, nullptr, ldy, out, ws + off_gemm, lin - off_gemm,
                     (cudaStream_t)stream, nullptr, &go);
 }
@@ -724,29 +678,75 @@ macaq_status macaq_linear_w4a4_noalloc(const void* x_bf16, int64_t M, int64_t ld
     return macaq_linear_w4a4(x_bf16, M, ldx, w, y, ldy, out, 0, scratch, MACAQ_NOALLOC_SCRATCH_BYTES, stream);
 }
 
-// ------------------------------------------------------------- grouped (MoE) ---
+}  // extern "C"
+
+// ------------------------------------------- grouped layers (MoE, shared input) ---
+
+namespace macaq {
+
+// Per-call tables (tensor maps, group descriptors) reach the device inside kernel
+// parameters: one small kernel per chunk writes its bytes to the workspace. Parameters
+// are copied when the kernel is enqueued, so the call neither waits for the stream nor
+// reads host memory after it returns.
+constexpr uint32_t kUploadChunkBytes = 16384;
+struct UploadChunk {
+    uint4* dst;
+    uint32_t words;                       // 16-byte words in data
+    uint4 data[kUploadChunkBytes / 16];
+};
+
+__global__ void __launch_bounds__(256) upload_kernel(const __grid_constant__ UploadChunk c) {
+    ptx::griddep_wait();                  // the stream's earlier kernels may still read dst
+    ptx::griddep_launch_dependents();
+    for (uint32_t i = threadIdx.x; i < c.words; i += blockDim.x) c.dst[i] = c.data[i];
+}
+
+// Enqueue the upload of `bytes` (a multiple of 16) from host memory to device `dst`.
+macaq_status upload(void* dst, const void* src, size_t bytes, cudaStream_t stream) {
+    const uint8_t* s = static_cast<const uint8_t*>(src);
+    for (size_t off = 0; off < bytes; off += kUploadChunkBytes) {
+        const size_t n = std::min<size_t>(kUploadChunkBytes, bytes - off);
+        UploadChunk c;
+        c.dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(dst) + off);
+        c.words = (uint32_t)(n / 16);
+        std::memcpy(c.data, s + off, n);
+        if (launch_pdl(upload_kernel, dim3(1), dim3(256), 0, stream, c) != cudaSuccess) return MACAQ_ERR_CUDA;
+    }
+    return MACAQ_OK;
+}
+
+}  // namespace macaq
 
 namespace {
 
-// Padded row layout of the grouped activations: group g's rows start at the multiple of
-// 128 after the previous group's, so every group owns whole scale slabs.
+// One group of a grouped layer: rows x_row .. x_row + rows - 1 of x through weight w into
+// rows row_y .. of y (row stride ldy).
+struct GroupSpec {
+    int64_t x_row, rows;
+    const macaq_weight* w;
+    void* y;
+    int64_t row_y, ldy;
+};
+
+// Workspace of a grouped layer: the activation codes and scales of every group, each
+// group padded to whole 128-row scale slabs, then the tables (tensor maps, group
+// descriptors, the quantiser's table), each part 256-byte aligned.
 struct GroupedLayout {
     int64_t rows_pad_total = 0;
     size_t off_scales = 0, off_tmaps = 0, off_desc = 0, off_qtab = 0, total = 0;
 };
 
-bool grouped_layout(const int64_t* offsets, int64_t G, int64_t K, GroupedLayout* L) {
-    if (!offsets || G < 1 || G > 4096 || K < 32 || K % 32 != 0) return false;
-    int64_t rows = 0;
+bool grouped_layout(const int64_t* rows, int64_t G, int64_t K, GroupedLayout* L) {
+    if (!rows || G < 1 || G > 4096 || K < 32 || K % 32 != 0) return false;
+    int64_t total = 0;
     for (int64_t g = 0; g < G; ++g) {
-        const int64_t m = offsets[g + 1] - offsets[g];
-        if (m < 0 || offsets[g] < 0) return false;
-        rows += round_up(m, 128);
+        if (rows[g] < 0) return false;
+        total += round_up(rows[g], 128);
     }
-    if (rows > kMaxRows) return false;
-    L->rows_pad_total = rows;
-    const size_t codes = (size_t)round_up(std::max<int64_t>(rows, 128) * (K / 2), 256);
-    const size_t scales = (size_t)round_up(std::max<int64_t>(rows, 128) * round_up(K / 32, 8), 256);
+    if (total > kMaxRows) return false;
+    L->rows_pad_total = total;
+    const size_t codes = (size_t)round_up(std::max<int64_t>(total, 128) * (K / 2), 256);
+    const size_t scales = (size_t)round_up(std::max<int64_t>(total, 128) * round_up(K / 32, 8), 256);
     L->off_scales = codes;
     L->off_tmaps = codes + scales;
     L->off_desc = L->off_tmaps + (size_t)round_up(G * (int64_t)sizeof(CUtensorMap), 256);
@@ -755,22 +755,132 @@ bool grouped_layout(const int64_t* offsets, int64_t G, int64_t K, GroupedLayout*
     return true;
 }
 
+// The grouped layer (arguments validated by the caller): one quantiser launch puts every
+// group's rows through the activation transform with its own weight's inv_s, one GEMM
+// launch covers every group's tiles (prefill orientation, 128- or 192-wide weight tiles,
+// direct stores). The tables reach the workspace through kernel parameters.
+macaq_status run_grouped(const void* x, int64_t ldx, int64_t K, const std::vector<GroupSpec>& gs,
+                         macaq_out_dtype out, const GroupedLayout& GL, uint8_t* ws, cudaStream_t cs) {
+    DeviceInfo* dev = nullptr;
+    macaq_status st = device_info(&dev);
+    if (st != MACAQ_OK) return st;
+    const int64_t G = (int64_t)gs.size();
+    const int64_t esz = out == MACAQ_OUT_BF16 ? 2 : 4;
+    int64_t n_max = 0;
+    for (const GroupSpec& g : gs) n_max = std::max(n_max, g.w->N);
+    // tile width: the fewer rounds of tiles over the SMs, then the narrower tiles' cost
+    int bn = 128;
+    if (n_max > 128) {
+        double best = 0.0;
+        for (int cand : {192, 128}) {
+            int64_t units = 0;
+            for (const GroupSpec& g : gs) units += cdiv(g.rows, 128) * cdiv(g.w->N, cand);
+            const double cost = (double)cdiv(units, dev->num_sms) * ktile_cycles(cand);
+            if (best == 0.0 || cost < best * 0.98) {
+                best = cost;
+                bn = cand;
+            }
+        }
+    }
+    std::vector<CUtensorMap> maps((size_t)G);
+    std::vector<GemmGroup> desc((size_t)G);
+    std::vector<QuantGroup> qtab;
+    int64_t units = 0, row_p = 0;
+    bool vec = true;
+    for (int64_t g = 0; g < G; ++g) {
+        const GroupSpec& q = gs[(size_t)g];
+        if (q.rows > 0) qtab.push_back(QuantGroup{q.x_row, (int32_t)q.rows, (int32_t)row_p, q.w->inv_s});
+        if (!encode_codes_map(&maps[g], q.w->codes, q.w->N, K, bn)) return MACAQ_ERR_CUDA;
+        GemmGroup& d = desc[(size_t)g];
+        d.unit_begin = (int32_t)units;
+        d.rows = (int32_t)q.rows;
+        d.row_p = (int32_t)row_p;
+        d.row_y = (int32_t)q.row_y;
+        d.q_rows = (int32_t)q.w->N;
+        d.tiles_q = (int32_t)cdiv(q.w->N, bn);
+        d.sf_q = q.w->scales;
+        d.out = q.y;
+        d.ldo = q.ldy;
+        vec = vec && aligned16(q.y) && (q.ldy * esz) % 16 == 0;
+        units += cdiv(q.rows, 128) * d.tiles_q;
+        row_p += round_up(q.rows, 128);
+    }
+    if (units > INT32_MAX) return MACAQ_ERR_UNSUPPORTED_SHAPE;
+    {
+        // one contiguous image of the three tables, in their workspace layout
+        std::vector<uint8_t> image(GL.total - GL.off_tmaps, 0);
+        std::memcpy(image.data(), maps.data(), maps.size() * sizeof(CUtensorMap));
+        std::memcpy(image.data() + (GL.off_desc - GL.off_tmaps), desc.data(), desc.size() * sizeof(GemmGroup));
+        std::memcpy(image.data() + (GL.off_qtab - GL.off_tmaps), qtab.data(), qtab.size() * sizeof(QuantGroup));
+        st = upload(ws + GL.off_tmaps, image.data(), image.size(), cs);
+        if (st != MACAQ_OK) return st;
+    }
+    uint8_t* a_codes = ws;
+    uint8_t* a_scales = ws + GL.off_scales;
+    if (!qtab.empty()) {
+        st = launch_quant_grouped(x, ldx, K, reinterpret_cast<const QuantGroup*>(ws + GL.off_qtab), (int)qtab.size(),
+                                  GL.rows_pad_total, a_codes, a_scales, cs);
+        if (st != MACAQ_OK) return st;
+    }
+    if (units == 0) return MACAQ_OK;
+    CUtensorMap mp, mq, my;
+    std::memset(&mq, 0, sizeof(mq));
+    std::memset(&my, 0, sizeof(my));
+    if (!encode_codes_map(&mp, a_codes, std::max<int64_t>(GL.rows_pad_total, 1), K, 128)) return MACAQ_ERR_CUDA;
+    GemmParams gp{};
+    gp.sf_p = a_scales;
+    gp.sf_q = gs[0].w->scales;
+    gp.out = gs[0].y;
+    gp.ldo = gs[0].ldy;
+    gp.p_rows = (int32_t)GL.rows_pad_total;
+    gp.q_rows = (int32_t)n_max;
+    gp.k_tiles = (int32_t)cdiv(K, 256);
+    gp.kb4_pad = (int32_t)(round_up(K / 32, 8) / 4);
+    gp.tiles_p = 1;
+    gp.tiles_q = (int32_t)cdiv(n_max, bn);
+    gp.total_units = (int32_t)units;
+    gp.sk_tile0 = (int32_t)units;
+    gp.group_p = 1;
+    gp.out_bf16 = out == MACAQ_OUT_BF16 ? 1 : 0;
+    gp.vec_ok = vec ? 1 : 0;
+    gp.err = dev->err_ptr;
+    gp.groups = (int32_t)G;
+    gp.g_desc = reinterpret_cast<const GemmGroup*>(ws + GL.off_desc);
+    gp.g_tmaps = reinterpret_cast<const CUtensorMap*>(ws + GL.off_tmaps);
+    const int grid = (int)std::min<int64_t>(units, dev->num_sms);
+    return bn == 128 ? launch_gemm_bn<128, 6>(mp, mq, my, gp, grid, cs) : launch_gemm_bn<192, 5>(mp, mq, my, gp, grid, cs);
+}
+
+// Group rows of the MoE layer from its offsets (false if they are not valid).
+bool moe_rows(const int64_t* offsets, int64_t G, std::vector<int64_t>* rows) {
+    if (!offsets || G < 1 || G > 4096 || offsets[0] != 0) return false;
+    rows->resize((size_t)G);
+    for (int64_t g = 0; g < G; ++g) {
+        (*rows)[(size_t)g] = offsets[g + 1] - offsets[g];
+        if ((*rows)[(size_t)g] < 0) return false;
+    }
+    return true;
+}
+
 }  // namespace
 
+extern "C" {
+
 size_t macaq_grouped_linear_workspace_bytes(const int64_t* offsets, int64_t G, int64_t K) {
+    std::vector<int64_t> rows;
     GroupedLayout L;
-    return grouped_layout(offsets, G, K, &L) ? L.total : 0;
+    return moe_rows(offsets, G, &rows) && grouped_layout(rows.data(), G, K, &L) ? L.total : 0;
 }
 
 macaq_status macaq_grouped_linear_w4a4(const void* x_bf16, int64_t ldx, const int64_t* offsets, int64_t G,
                                        const macaq_weight* weights, void* y, int64_t ldy, macaq_out_dtype out,
                                        void* workspace, size_t ws_bytes, macaq_stream stream) {
     if (!x_bf16 || !offsets || !weights || !y) return MACAQ_ERR_INVALID_ARG;
-    GroupedLayout GL;
     if (G < 1 || !weights[0].codes) return MACAQ_ERR_INVALID_ARG;
     const int64_t N = weights[0].N, K = weights[0].K;
-    if (offsets[0] != 0) return MACAQ_ERR_INVALID_ARG;
-    if (!grouped_layout(offsets, G, K, &GL)) return MACAQ_ERR_INVALID_ARG;
+    std::vector<int64_t> rows;
+    GroupedLayout GL;
+    if (!moe_rows(offsets, G, &rows) || !grouped_layout(rows.data(), G, K, &GL)) return MACAQ_ERR_INVALID_ARG;
     const int64_t M = offsets[G];
     if (M < 1) return MACAQ_ERR_INVALID_ARG;
     for (int64_t g = 0; g < G; ++g) {
@@ -785,80 +895,40 @@ macaq_status macaq_grouped_linear_w4a4(const void* x_bf16, int64_t ldx, const in
     if (st != MACAQ_OK) return st;
     if (!workspace || ws_bytes < GL.total) return MACAQ_ERR_WORKSPACE;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255) != 0) return MACAQ_ERR_MISALIGNED;
-    DeviceInfo* dev = nullptr;
-    st = device_info(&dev);
-    if (st != MACAQ_OK) return st;
-    cudaStream_t cs = (cudaStream_t)stream;
-    uint8_t* ws = static_cast<uint8_t*>(workspace);
-    uint8_t* a_codes = ws;
-    uint8_t* a_scales = ws + GL.off_scales;
-    const int64_t kb_pad = round_up(K / 32, 8);
+    std::vector<GroupSpec> gs((size_t)G);
+    for (int64_t g = 0; g < G; ++g)
+        gs[(size_t)g] = GroupSpec{offsets[g], rows[(size_t)g], &weights[g], y, offsets[g], ldy};
+    return run_grouped(x_bf16, ldx, K, gs, out, GL, static_cast<uint8_t*>(workspace), (cudaStream_t)stream);
+}
 
-    // the GEMM's group tables, copied from pageable host memory before any kernel is
-    // enqueued (such a copy first waits for the stream, then is staged before return)
-    const int bn = N <= 128 ? 128 : 192;
-    const int64_t tiles_q = cdiv(N, bn);
-    std::vector<CUtensorMap> maps((size_t)G);
-    std::vector<GemmGroup> desc((size_t)G);
-    std::vector<QuantGroup> qtab;
-    int64_t units = 0;
-    int64_t row_p = 0;
+size_t macaq_multi_linear_workspace_bytes(int64_t M, int64_t K, int64_t G) {
+    if (M < 1 || G < 1 || G > 4096) return 0;
+    std::vector<int64_t> rows((size_t)G, M);
+    GroupedLayout L;
+    return grouped_layout(rows.data(), G, K, &L) ? L.total : 0;
+}
+
+macaq_status macaq_multi_linear_w4a4(const void* x_bf16, int64_t M, int64_t ldx, const macaq_weight* weights,
+                                     int64_t G, void* const* y, const int64_t* ldy, macaq_out_dtype out,
+                                     void* workspace, size_t ws_bytes, macaq_stream stream) {
+    if (!x_bf16 || !weights || !y || !ldy || G < 1 || G > 4096 || M < 1) return MACAQ_ERR_INVALID_ARG;
+    const int64_t K = weights[0].K;
     for (int64_t g = 0; g < G; ++g) {
-        const int64_t m = offsets[g + 1] - offsets[g];
-        if (m > 0) qtab.push_back(QuantGroup{offsets[g], (int32_t)m, (int32_t)row_p, weights[g].inv_s});
-        if (!encode_codes_map(&maps[g], weights[g].codes, N, K, bn)) return MACAQ_ERR_CUDA;
-        desc[g].unit_begin = (int32_t)units;
-        desc[g].rows = (int32_t)m;
-        desc[g].row_p = (int32_t)row_p;
-        desc[g].row_y = (int32_t)offsets[g];
-        desc[g].sf_q = weights[g].scales;
-        desc[g].pad = 0;
-        units += cdiv(m, 128) * tiles_q;
-        row_p += round_up(m, 128);
+        macaq_status st = check_gemm_args(M, &weights[g], y[g], ldy[g], out);
+        if (st != MACAQ_OK) return st;
+        if (weights[g].K != K || !weights[g].inv_s) return MACAQ_ERR_INVALID_ARG;
+        if (!aligned16(weights[g].inv_s)) return MACAQ_ERR_MISALIGNED;
     }
-    if (units > INT32_MAX) return MACAQ_ERR_UNSUPPORTED_SHAPE;
-    if (cudaMemcpyAsync(ws + GL.off_tmaps, maps.data(), maps.size() * sizeof(CUtensorMap), cudaMemcpyHostToDevice,
-                        cs) != cudaSuccess ||
-        cudaMemcpyAsync(ws + GL.off_desc, desc.data(), desc.size() * sizeof(GemmGroup), cudaMemcpyHostToDevice,
-                        cs) != cudaSuccess ||
-        cudaMemcpyAsync(ws + GL.off_qtab, qtab.data(), qtab.size() * sizeof(QuantGroup), cudaMemcpyHostToDevice,
-                        cs) != cudaSuccess)
-        return MACAQ_ERR_CUDA;
-    // every expert's rows through the activation transform with its own inv_s: one launch
-    st = launch_quant_grouped(x_bf16, ldx, K, reinterpret_cast<const QuantGroup*>(ws + GL.off_qtab),
-                              (int)qtab.size(), GL.rows_pad_total, a_codes, a_scales, cs);
+    macaq_status st = check_quant_args(x_bf16, M, K, ldx, weights[0].inv_s, weights[0].codes, weights[0].scales);
     if (st != MACAQ_OK) return st;
-
-    // the GEMM: one launch over every group's units
-    CUtensorMap mp, mq, my;
-    std::memset(&mq, 0, sizeof(mq));
-    std::memset(&my, 0, sizeof(my));
-    if (!encode_codes_map(&mp, a_codes, std::max<int64_t>(GL.rows_pad_total, 1), K, 128)) return MACAQ_ERR_CUDA;
-    GemmParams gp{};
-    gp.sf_p = a_scales;
-    gp.sf_q = weights[0].scales;
-    gp.out = y;
-    gp.ldo = ldy;
-    gp.p_rows = (int32_t)GL.rows_pad_total;
-    gp.q_rows = (int32_t)N;
-    gp.k_tiles = (int32_t)cdiv(K, 256);
-    gp.kb4_pad = (int32_t)(kb_pad / 4);
-    gp.tiles_p = 1;
-    gp.tiles_q = (int32_t)tiles_q;
-    gp.splits = 1;
-    gp.k_tiles_per_split = gp.k_tiles;
-    gp.total_units = (int32_t)units;
-    gp.group_p = 1;
-    gp.out_bf16 = out == MACAQ_OUT_BF16 ? 1 : 0;
-    const int64_t esz = out == MACAQ_OUT_BF16 ? 2 : 4;
-    gp.vec_ok = (aligned16(y) && (ldy * esz) % 16 == 0) ? 1 : 0;
-    gp.err = dev->err_ptr;
-    gp.groups = (int32_t)G;
-    gp.g_desc = reinterpret_cast<const GemmGroup*>(ws + GL.off_desc);
-    gp.g_tmaps = reinterpret_cast<const CUtensorMap*>(ws + GL.off_tmaps);
-    if (units == 0) return MACAQ_OK;
-    const int grid = (int)std::min<int64_t>(units, dev->num_sms);
-    return bn == 128 ? launch_gemm_bn<128, 6>(mp, mq, my, gp, grid, cs) : launch_gemm_bn<192, 5>(mp, mq, my, gp, grid, cs);
+    std::vector<int64_t> rows((size_t)G, M);
+    GroupedLayout GL;
+    if (!grouped_layout(rows.data(), G, K, &GL)) return MACAQ_ERR_UNSUPPORTED_SHAPE;
+    if (!workspace || ws_bytes < GL.total) return MACAQ_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255) != 0) return MACAQ_ERR_MISALIGNED;
+    std::vector<GroupSpec> gs((size_t)G);
+    for (int64_t g = 0; g < G; ++g) gs[(size_t)g] = GroupSpec{0, M, &weights[g], y[g], 0, ldy[g]};
+    return run_grouped(x_bf16, ldx, K, gs, out, GL, static_cast<uint8_t*>(workspace), (cudaStream_t)stream);
 }
 
 size_t macaq_hessian_bytes(int64_t K) {
@@ -982,9 +1052,8 @@ macaq_status macaq_flip_refine(const void* W_bf16, int64_t N, int64_t K, int64_t
 }  // extern "C"
 
 namespace {
-// Results and flags of macaq_selftest_wait_timeout (the device error word is not used).
+// Results of macaq_selftest_wait_timeout (the device error word is not used).
 __device__ long long g_selftest_out[macaq::kSelftestWords];
-__device__ unsigned long long g_selftest_flags[2];
 }  // namespace
 
 extern "C" {
@@ -995,13 +1064,8 @@ macaq_status macaq_selftest_wait_timeout(uint32_t limit_us, int64_t* result, mac
     const macaq_status st = device_info(&dev);
     if (st != MACAQ_OK) return st;
     void* out = nullptr;
-    void* flags = nullptr;
-    if (cudaGetSymbolAddress(&out, g_selftest_out) != cudaSuccess ||
-        cudaGetSymbolAddress(&flags, g_selftest_flags) != cudaSuccess)
-        return MACAQ_ERR_CUDA;
-    wait_selftest_kernel<<<2, 96, 0, stream>>>((uint64_t)limit_us * 1000u,
-                                               static_cast<unsigned long long*>(flags),
-                                               static_cast<long long*>(out));
+    if (cudaGetSymbolAddress(&out, g_selftest_out) != cudaSuccess) return MACAQ_ERR_CUDA;
+    wait_selftest_kernel<<<2, 96, 0, stream>>>((uint64_t)limit_us * 1000u, static_cast<long long*>(out));
     if (cudaGetLastError() != cudaSuccess) return MACAQ_ERR_CUDA;
     long long host[kSelftestWords];
     if (cudaMemcpyAsync(host, out, sizeof host, cudaMemcpyDeviceToHost, stream) != cudaSuccess ||

@@ -6,6 +6,7 @@ the ncu captures that back them.
                                           [--warmup W] [--fused] [--calib T] [--rounds R]
     python -m mxfp4_w4a4_post_b200.timing moe [--experts G] [--tokens T] [--n N] [--k K]
     python -m mxfp4_w4a4_post_b200.timing tp WORKLOAD [--world G]
+    python -m mxfp4_w4a4_post_b200.timing layerset
 
 Inputs are the workload's seeded synthetic tensors (workloads.py), resident on the
 device. Before every timed call L2 is flushed by a 256 MiB write and a read of the same
@@ -21,6 +22,8 @@ printed, one line per measured call:
              macaq_linear_w4a4 calls
     tp       one rank's macaq_linear_w4a4 under a column- and a row-parallel cut into G
              pieces (the collective that follows needs several GPUs and is not timed)
+    layerset the seven projections of a decoder layer at 256 rows: seven layer calls,
+             and by role (q/k/v and gate/up each one macaq_multi_linear_w4a4 call)
     flip     macaq_hessian_full on T calibration rows, then macaq_flip_refine of the
              prepared weight (each timed call starts again from the round-to-nearest
              codes, restored before the flush); also prints the moves per row
@@ -118,6 +121,73 @@ def moe(a):
     return 1 if mq.device_error() != 0 else 0
 
 
+def layerset(a):
+    """The seven projections of a Qwen3-32B-shaped decoder layer at 256 rows, each with its
+    own seeded input, weight and s: as seven macaq_linear_w4a4 calls, and by role, with
+    the layers that share an input in one macaq_multi_linear_w4a4 call (q/k/v; gate/up)
+    and o and down on their own (four calls)."""
+    import ctypes
+    import torch
+    import mxfp4_w4a4_post_b200 as mq
+    dev = torch.device("cuda", torch.cuda.current_device())
+    layers = wl.qwen3_32b_layer_decode(256)
+    by = {L.name.split("_")[2]: L for L in layers}          # q, k, v, o, gate, up, down
+    pws, xs = {}, {}
+    for k, L in by.items():
+        pws[k] = mq.prepare_weight(_bf16(torch, wl.draw_W(L), dev), torch.from_numpy(wl.draw_s(L)).to(dev))
+        xs[k] = _bf16(torch, wl.draw_x(L), dev)
+    ys = {k: torch.empty((L.M, L.N), dtype=torch.bfloat16, device=dev) for k, L in by.items()}
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    lib = mq.lib()
+    stream = ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+    cws = {k: pw.c_struct() for k, pw in pws.items()}
+    lws = torch.empty(max(mq.linear_workspace_bytes(L.M, L.N, L.K, torch.bfloat16) for L in layers),
+                      dtype=torch.uint8, device=dev)
+
+    def lin_args(k):
+        L = by[k]
+        return (xs[k].data_ptr(), L.M, xs[k].stride(0), ctypes.byref(cws[k]), ys[k].data_ptr(), ys[k].stride(0),
+                mq.OUT_BF16, 0, lws.data_ptr(), lws.numel(), stream)
+
+    def multi_args(keys, x, ws_t):
+        G = len(keys)
+        wts = (mq.MacaqWeight * G)(*[cws[k] for k in keys])
+        yp = (ctypes.c_void_p * G)(*[ys[k].data_ptr() for k in keys])
+        lds = (ctypes.c_int64 * G)(*[ys[k].stride(0) for k in keys])
+        return (x.data_ptr(), 256, x.stride(0), wts, G, yp, lds, mq.OUT_BF16, ws_t.data_ptr(), ws_t.numel(), stream)
+
+    # the layers that share an input take one input (q/k/v: q's, gate/up: gate's)
+    mws1 = torch.empty(lib.macaq_multi_linear_workspace_bytes(256, 5120, 3), dtype=torch.uint8, device=dev)
+    mws2 = torch.empty(lib.macaq_multi_linear_workspace_bytes(256, 5120, 2), dtype=torch.uint8, device=dev)
+    calls_sep = [(lib.macaq_linear_w4a4, lin_args(k)) for k in ("q", "k", "v", "o", "gate", "up", "down")]
+    calls_role = [(lib.macaq_multi_linear_w4a4, multi_args(("q", "k", "v"), xs["q"], mws1)),
+                  (lib.macaq_linear_w4a4, lin_args("o")),
+                  (lib.macaq_multi_linear_w4a4, multi_args(("gate", "up"), xs["gate"], mws2)),
+                  (lib.macaq_linear_w4a4, lin_args("down"))]
+
+    def run(calls):
+        def f():
+            for fn, args in calls:
+                st = fn(*args)
+                if st != 0:
+                    raise mq.MacaqError(st, fn.__name__)
+        return f
+
+    flops = sum(2.0 * L.M * L.N * L.K for L in layers)
+    wbytes = sum(L.N * L.K * 0.53125 for L in layers)
+    for label, calls in (("seven linear_w4a4 calls", calls_sep), ("by role (4 calls)", calls_role)):
+        t = _time(torch, run(calls), flush, a.reps, a.warmup)
+        print(f"qwen3_32b decoder-layer set, 256 rows, {label}: {t * 1e6:.1f} us {flops / t / 1e12:.1f} TFLOP/s "
+              f"{wbytes / t / 1e9:.0f} GB/s of weights")
+    for k in ("q", "k", "v", "o", "gate", "up", "down"):
+        t = _time(torch, run([(lib.macaq_linear_w4a4, lin_args(k))]), flush, a.reps, a.warmup)
+        print(f"  {by[k].name} linear_w4a4 {t * 1e6:.1f} us")
+    for keys, x, ws_t in ((("q", "k", "v"), xs["q"], mws1), (("gate", "up"), xs["gate"], mws2)):
+        t = _time(torch, run([(lib.macaq_multi_linear_w4a4, multi_args(keys, x, ws_t))]), flush, a.reps, a.warmup)
+        print(f"  multi_linear_w4a4 {'/'.join(keys)} {t * 1e6:.1f} us")
+    return 1 if mq.device_error() != 0 else 0
+
+
 def tp(a, L):
     """One rank's layer call under column- and row-parallel cuts of the workload's weight
     into `--world` pieces (the rank with the largest piece), with the bytes its single
@@ -166,7 +236,7 @@ def tp(a, L):
 
 def main(argv=None):
     p = argparse.ArgumentParser()
-    p.add_argument("what", choices=["list", "quant", "gemm", "linear", "hessian", "flip", "moe", "tp"])
+    p.add_argument("what", choices=["list", "quant", "gemm", "linear", "hessian", "flip", "moe", "tp", "layerset"])
     p.add_argument("workload", nargs="?")
     p.add_argument("--reps", type=int, default=20)
     p.add_argument("--warmup", type=int, default=3)
@@ -185,6 +255,8 @@ def main(argv=None):
         return 0
     if a.what == "moe":
         return moe(a)
+    if a.what == "layerset":
+        return layerset(a)
     if a.workload not in ws:
         p.error(f"unknown workload {a.workload!r}; see `list`")
     L = ws[a.workload]

@@ -97,7 +97,27 @@ def test_validation_rejects_bad_arguments(L):
     assert L.macaq_linear_w4a4_gather(a, 4, 256, ctypes.byref(w), d_many, 65, 128, 0, a, 1 << 20, None) == 1
     assert L.macaq_linear_w4a4_gather(a, 4, 256, ctypes.byref(w), d_mis, 1, 128, 0, a, 1 << 20, None) == 2
     assert L.macaq_linear_w4a4_gather(a, 4, 256, ctypes.byref(w), d_ok, 2, 64, 0, a, 1 << 20, None) == 1  # ldy < N
-    assert L.macaq_linear_gather_workspace_bytes(4, 128, 256, 0) == L.macaq_linear_workspace_bytes(4, 128, 256, 0) + 512
+    assert L.macaq_linear_gather_workspace_bytes(4, 128, 256, 0) == L.macaq_linear_workspace_bytes(4, 128, 256, 0)
+
+
+def test_multi_linear_validation(L):
+    """The shared-input layer checks its arguments before anything is launched."""
+    a = ctypes.c_void_p(0x1000)
+    ok = mq.MacaqWeight(0x1000, 0x1000, 0x1000, 128, 256)
+    ws2 = (mq.MacaqWeight * 2)(ok, mq.MacaqWeight(0x1000, 0x1000, 0x1000, 64, 256))
+    ys = (ctypes.c_void_p * 2)(0x2000, 0x3000)
+    lds = (ctypes.c_int64 * 2)(128, 64)
+    assert L.macaq_multi_linear_workspace_bytes(4, 256, 2) == L.macaq_multi_linear_workspace_bytes(100, 256, 2)
+    assert L.macaq_multi_linear_workspace_bytes(0, 256, 2) == 0
+    assert L.macaq_multi_linear_w4a4(None, 4, 256, ws2, 2, ys, lds, 0, a, 1 << 24, None) == 1
+    assert L.macaq_multi_linear_w4a4(a, 4, 256, ws2, 0, ys, lds, 0, a, 1 << 24, None) == 1
+    other_k = (mq.MacaqWeight * 2)(ok, mq.MacaqWeight(0x1000, 0x1000, 0x1000, 64, 512))
+    assert L.macaq_multi_linear_w4a4(a, 4, 256, other_k, 2, ys, lds, 0, a, 1 << 24, None) == 1
+    bad_inv = (mq.MacaqWeight * 2)(ok, mq.MacaqWeight(0x1000, 0x1000, 0x1004, 64, 256))
+    assert L.macaq_multi_linear_w4a4(a, 4, 256, bad_inv, 2, ys, lds, 0, a, 1 << 24, None) == 2
+    short_ld = (ctypes.c_int64 * 2)(128, 32)
+    assert L.macaq_multi_linear_w4a4(a, 4, 256, ws2, 2, ys, short_ld, 0, a, 1 << 24, None) == 1
+    assert L.macaq_multi_linear_w4a4(a, 4, 256, ws2, 2, ys, lds, 0, a, 1024, None) == 7
 
 
 def test_no_usable_device_is_a_status_not_a_crash(L):
@@ -116,5 +136,12 @@ def test_no_usable_device_is_a_status_not_a_crash(L):
     assert L.macaq_gemm_mxfp4(a, a, 4, ctypes.byref(w), a, 128, 0, None, 0, None) == 5
     assert L.macaq_linear_w4a4(a, 4, 256, ctypes.byref(w), a, 128, 0, 0, a, 1 << 24, None) == 5
     assert L.macaq_linear_w4a4_gather(a, 4, 256, ctypes.byref(w), d, 1, 128, 0, a, 1 << 24, None) == 5
+    ws2 = (mq.MacaqWeight * 2)(mq.MacaqWeight(0x1000, 0x1000, 0x1000, 128, 256),
+                               mq.MacaqWeight(0x1000, 0x1000, 0x1000, 64, 256))
+    ys = (ctypes.c_void_p * 2)(0x2000, 0x3000)
+    lds = (ctypes.c_int64 * 2)(128, 64)
+    assert L.macaq_multi_linear_w4a4(a, 4, 256, ws2, 2, ys, lds, 0, a, 1 << 24, None) == 5
+    offs = (ctypes.c_int64 * 3)(0, 3, 4)
+    assert L.macaq_grouped_linear_w4a4(a, 256, offs, 2, (mq.MacaqWeight * 2)(w, w), a, 128, 0, a, 1 << 24, None) == 5
     assert L.macaq_selftest_wait_timeout(100, res, None) == 5
     assert L.macaq_get_device_error() == 5

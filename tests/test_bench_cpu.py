@@ -23,7 +23,7 @@ def test_reference_arm_json_line():
                 "scaling", "vs_baseline", "dtype", "data", "config", "impl", "cpu_baseline", "e2e"):
         assert key in d, key
     assert d["impl"] == "reference" and d["value"] > 0 and d["steps"] == 1
-    assert d["config"]["workload"] == "llama3_8b_gate_up_prefill_4096x14336x4096"
+    assert d["config"]["workload"].startswith("llama3_8b_gate_up_prefill_4096x14336x4096 (sampled")
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"]
 

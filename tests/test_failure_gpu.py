@@ -1,9 +1,10 @@
 """Failure detection on the GPU without a fault: the GEMM kernel's bounded wait routines
 are run by a self-test kernel against waits that cannot succeed (an mbarrier nothing
-arrives at, a split-K flag that holds another epoch) with a short limit. Each wait must
-give up after the limit, record its code and raise the CTA abort flag; a second wait in
-the same CTA must leave on that flag; waits that can succeed must succeed. Afterwards
-the context must still run the layer correctly."""
+arrives at) with a short limit. Each wait must give up after the limit, record its code
+and raise the CTA abort flag; a second wait in the same CTA must leave on that flag;
+waits that can succeed must succeed; and a group of warps whose member gave up must
+agree to leave together at its named barrier instead of holding the others there.
+Afterwards the context must still run the layer correctly."""
 import numpy as np
 import pytest
 
@@ -14,7 +15,7 @@ from mxfp4_w4a4_post_b200 import workloads as wl
 pytestmark = pytest.mark.gpu
 
 ERR_TIMEOUT_PRODUCER = 1
-ERR_TIMEOUT_SPLIT = 5
+ERR_TIMEOUT_SET = 5
 
 
 @pytest.fixture(scope="module")
@@ -38,11 +39,12 @@ def test_bounded_waits_give_up(mq, limit_us):
     assert r["bar_abort_ns"] < 1_000_000_000
     # a barrier that completes is seen completing
     assert r["bar_done_ok"] == 1
-    # split-K flag wait: gives up with the flag code; a flag already set is accepted
-    assert r["flag_timeout_ok"] == 0
-    assert r["flag_err"] == ERR_TIMEOUT_SPLIT
-    assert limit_ns <= r["flag_timeout_ns"] < limit_ns + 500_000_000
-    assert r["flag_done_ok"] == 1
+    # a warp group whose member gave up agrees to leave; the member's wait took the
+    # limit and recorded its code, the others' own waits completed, and none was held
+    assert r["set_agreed_ok"] == 0
+    assert r["set_err"] == ERR_TIMEOUT_SET
+    assert limit_ns <= r["set_timeout_ns"] < limit_ns + 500_000_000
+    assert r["set_member_ok"] == 1
     # the layer's own error word is untouched
     assert mq.device_error() == 0
 

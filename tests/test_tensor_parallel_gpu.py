@@ -108,7 +108,7 @@ def test_module_with_nccl_one_rank(mq):
 
 
 # (M, N, K, shards): prefill tiles, decode (swapped) tiles, and a shape for which the
-# ordinary layer splits K (the gathered output never does)
+# ordinary layer runs on the stream-K schedule (the gathered output never does)
 GATHER_CASES = [(200, 520, 1024, 2), (5, 300, 512, 3), (16, 256, 16384, 2)]
 
 
@@ -148,7 +148,7 @@ def test_gathered_column_cut(mq, M, N, K, shards, dt):
     if dt == "f32":
         assert_gemm_close(y0, ref, f"gathered column cut {M}x{N}x{K}")
     # each shard's columns equal the ordinary layer's output for that shard whenever
-    # that one does not split K (same tiles, same MMAs, another store path)
+    # that one gives every tile to one CTA (same tiles, same MMAs, another store path)
     for n0, n1, w in shard_out:
         y_lin = mq.linear(xd, w, out_dtype=dtype)
         if mq.gemm_workspace_bytes(M, n1 - n0, K, dtype) == 0:
@@ -156,7 +156,7 @@ def test_gathered_column_cut(mq, M, N, K, shards, dt):
         else:
             y32 = mq.linear(xd, w, out_dtype=torch.float32)
             if dt == "f32":
-                assert_gemm_close(host(ys[0][:, n0:n1]), host(y32).astype(np.float64), "split shard")
+                assert_gemm_close(host(ys[0][:, n0:n1]), host(y32).astype(np.float64), "stream-K shard")
             else:
-                assert_bf16_matches_f32(ys[0][:, n0:n1], y32, "split shard")
+                assert_bf16_matches_f32(ys[0][:, n0:n1], y32, "stream-K shard")
     assert mq.device_error() == 0

@@ -47,7 +47,7 @@ def noalloc_linear(mq, x, pw, out_dtype):
 @pytest.mark.parametrize("M,N,K", [(16, 512, 16384), (300, 1000, 1024)])
 def test_noalloc_matches_workspace_entry_point(mq, M, N, K):
     """Two calls in a row with different activations (the second call must not see the
-    first call's split-K partial sums), each against macaq_linear_w4a4."""
+    first call's stream-K partial tiles or counts), each against macaq_linear_w4a4."""
     import torch
     base = wl.with_shape(wl.tiny_layer(), M=M, N=N, K=K)
     assert mq.linear_workspace_bytes(M, N, K, torch.float32) <= NOALLOC_SCRATCH_BYTES
