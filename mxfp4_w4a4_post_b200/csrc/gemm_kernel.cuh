@@ -459,7 +459,6 @@ __device__ __forceinline__ void tmem_load_chunk<16>(uint32_t taddr, uint32_t (&r
 }
 
 constexpr int kSfWarpSets = 2;                                // scale-writer sets
-constexpr int kPrefetchAhead = 4;                             // K tiles of L2 prefetch beyond the copies
 constexpr int kGemmThreads = 32 * (6 + 4 * kSfWarpSets);
 
 // Kernel variants, each its own instantiation so that the ordinary kernels keep their
@@ -496,27 +495,42 @@ __device__ __forceinline__ void fused_transform(const GemmParams& p, uint8_t* sm
     for (int i = tt; i < p.k_tiles * S::kSfChunkBytes / 16; i += kFusedThreads) ptx::sts128(sp + 16 * i, 0u, 0u, 0u, 0u);
     asm volatile("bar.sync 2, %0;" ::"n"(kFusedThreads) : "memory");   // zeros before scale words
     const int total = p.k_tiles * rows * 8;
+    // item i -> (K tile, row, block); the activation load of a thread's next item is
+    // issued before its current item is encoded, so its latency overlaps the encoding
+    auto item = [&](int i, int& kt, int& r, int& j) {
+        kt = i / (rows * 8);
+        const int rem = i - kt * rows * 8;
+        r = rem >> 3;
+        j = rem & 7;
+    };
+    auto load_x = [&](int i, uint4 (&xv)[4]) {
+        int kt, r, j;
+        item(i, kt, r, j);
+        const int b = kt * 8 + j;
+        if (i < total && b < kb) {
+            const uint4* xs = reinterpret_cast<const uint4*>(p.fx + (int64_t)r * p.fx_ld + (int64_t)b * 32);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) xv[c] = __ldg(xs + c);
+        }
+    };
+    uint4 nx[4];
+    load_x(tt, nx);
     for (int base = 0; base < total; base += kFusedThreads) {
         const int i = base + tt;
         const bool live = i < total;
         int kt = 0, r = 0, j = 0;
-        if (live) {
-            kt = i / (rows * 8);
-            const int rem = i - kt * rows * 8;
-            r = rem >> 3;
-            j = rem & 7;
-        }
+        if (live) item(i, kt, r, j);
+        uint4 xv[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) xv[c] = nx[c];
+        load_x(i + kFusedThreads, nx);
         const int b = kt * 8 + j;
         uint32_t sbyte = 0;
         if (live) {
             uint32_t packed[4] = {0u, 0u, 0u, 0u};
             if (b < kb) {
-                const uint4* xs = reinterpret_cast<const uint4*>(p.fx + (int64_t)r * p.fx_ld + (int64_t)b * 32);
                 const float4* ms = reinterpret_cast<const float4*>(p.f_mult + (int64_t)b * 32);
-                uint4 xv[4];
                 float4 mv[8];
-#pragma unroll
-                for (int c = 0; c < 4; ++c) xv[c] = __ldg(xs + c);
 #pragma unroll
                 for (int c = 0; c < 8; ++c) mv[c] = __ldg(ms + c);
                 uint64_t T[16];
@@ -624,23 +638,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                                t.sf_q + ((int64_t)(slab0 + c) * p.kb4_pad + 2 * kt) * 512, S::kSfChunkBytes,
                                &full[st]);
         };
-        // L2 prefetch of the K tile kPrefetchAhead positions further along this CTA's
-        // schedule, so that the copy of it later finds its lines in L2
-        auto prefetch = [&](const Unit& t, int kt) {
-            const int q0 = t.tq * BN;
-            ptx::tma_prefetch_2d(&tmap_p, kt * S::kBKBytes, t.p_row0);
-            ptx::bulk_prefetch_l2(p.sf_p + ((int64_t)(t.p_row0 >> 7) * p.kb4_pad + 2 * kt) * 512, S::kSfChunkBytes);
-            if constexpr (!FUSED) {
-                ptx::tma_prefetch_2d(t.tmap_q, kt * S::kBKBytes, q0);
-                ptx::bulk_prefetch_l2(t.sf_q + ((int64_t)(q0 / 128) * p.kb4_pad + 2 * kt) * 512, S::kSfChunkBytes);
-            }
-        };
         for (int uj = 0; uj < sc.n_units; ++uj) {
             const int u = sc.unit(uj);
             if (cta_aborted(abort)) break;
             const Unit t = decode_unit(p, u, &tmap_q, sc);
-            const bool has_next = uj + 1 < sc.n_units;
-            const Unit tn = has_next ? decode_unit(p, sc.unit(uj + 1), &tmap_q, sc) : t;
             const int q0 = t.tq * BN;
             const int slab0 = q0 / 128;
             const int nchunks = min(S::kQChunks, (t.q_rows + 127) / 128 - slab0);   // scale slabs of the Q rows
@@ -658,11 +659,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                                    p.sf_p + ((int64_t)(t.p_row0 >> 7) * p.kb4_pad + 2 * kt) * 512,
                                    S::kSfChunkBytes, &full[stage]);
                     if constexpr (!FUSED) issue_q(t, stage, kt, q0, slab0, nchunks);
-                    const int pk = kt + kPrefetchAhead;
-                    if (pk < t.kt_end)
-                        prefetch(t, pk);
-                    else if (has_next && tn.kt_begin + (pk - t.kt_end) < tn.kt_end)
-                        prefetch(tn, tn.kt_begin + (pk - t.kt_end));
                 }
                 __syncwarp();
                 issued_mask |= 1u << stage;

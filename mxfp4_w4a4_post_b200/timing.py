@@ -3,7 +3,7 @@ the ncu captures that back them.
 
     python -m mxfp4_w4a4_post_b200.timing list
     python -m mxfp4_w4a4_post_b200.timing {quant,gemm,linear,hessian,flip} WORKLOAD [--reps R]
-                                          [--warmup W] [--fused] [--calib T] [--rounds R]
+                                          [--warmup W] [--fused] [--rows M] [--calib T] [--rounds R]
     python -m mxfp4_w4a4_post_b200.timing moe [--experts G] [--tokens T] [--n N] [--k K]
     python -m mxfp4_w4a4_post_b200.timing tp WORKLOAD [--world G]
     python -m mxfp4_w4a4_post_b200.timing layerset
@@ -241,6 +241,8 @@ def main(argv=None):
     p.add_argument("--reps", type=int, default=20)
     p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--fused", action="store_true")
+    p.add_argument("--rows", type=int, default=None,
+                   help="run the workload's layer on this many rows of x (its first rows), e.g. a capture-sized slice")
     p.add_argument("--calib", type=int, default=2048, help="calibration rows for `hessian` and `flip`")
     p.add_argument("--rounds", type=int, default=256, help="move cap per row for `flip`")
     p.add_argument("--experts", type=int, default=8)
@@ -260,6 +262,9 @@ def main(argv=None):
     if a.workload not in ws:
         p.error(f"unknown workload {a.workload!r}; see `list`")
     L = ws[a.workload]
+    if a.rows is not None:
+        from dataclasses import replace
+        L = replace(L, M=a.rows, name=f"{L.name}[rows={a.rows}]")
     if a.what == "tp":
         return tp(a, L)
     import torch
