@@ -159,13 +159,17 @@ macaq_status macaq_gemm_mxfp4(const uint8_t* a_codes, const uint8_t* a_scales, i
 /* The whole online layer: the activation transform of macaq_quant_act into the
  * workspace, then the GEMM of macaq_gemm_mxfp4.
  *   fused     0: two launches (macaq_quant_act's kernel, then the GEMM).
- *             1: for M <= 32 (decode) one launch: the GEMM kernel makes the MXFP4
- *             activations itself, K tile by K tile, in the shared memory its tensor-core
- *             MMAs read them from (the per-channel multiplier, block Hadamard, E8M0
- *             exponent and E2M1 encoding of macaq_quant_act, bit for bit), while the
- *             weight tiles stream in; y is bit-identical to fused = 0. The activation
- *             part of the workspace is then not written. For M > 32 as 0 (there every
- *             CTA would repeat the transform of too many activation rows).
+ *             1: one launch where that is the faster form: for M <= 2 (decode) the GEMM
+ *             kernel makes the MXFP4 activations itself, before its main loop, in the
+ *             shared memory its tensor-core MMAs read them from (the per-channel
+ *             multiplier, block Hadamard, E8M0 exponent and E2M1 encoding of
+ *             macaq_quant_act, bit for bit), while the weight tiles stream in; every CTA
+ *             repeats that transform, so for more rows two launches are faster and are
+ *             used. y is bit-identical to fused = 0, and the activation part of the
+ *             workspace is not written.
+ *             2: as 1, for every M <= 32 whose MXFP4 activations fit in shared memory
+ *             beside the weight ring (K <= 7680 for M <= 16, K <= 6400 for M <= 32);
+ *             for callers that want a single launch whatever it costs. Other shapes as 0.
  *             Other values return MACAQ_ERR_INVALID_ARG.
  *   workspace device, >= macaq_linear_workspace_bytes(M, N, K, out), 256-byte aligned;
  *             it starts with the activation codes (macaq_codes_bytes(M, K) bytes) and,

@@ -333,8 +333,9 @@ def gemm_mxfp4(a_codes, a_scales, M, w, out_dtype=None, y=None, workspace=None):
 
 def linear(x, w, out_dtype=None, y=None, workspace=None, fused=False):
     """The MACaQ W4A4 layer: y = x W^T computed as (x diag(s)^-1 Hb)(Hb diag(s) W^T) in MXFP4.
-    fused=True: for M <= 128 the activation transform runs inside the GEMM kernel (one
-    launch); the quantised activations are left at the start of the workspace."""
+    fused: False (two launches), True (one launch where that is faster: M <= 2), or
+    "always" (one launch for every M <= 32 the kernel takes); in one launch the GEMM
+    kernel makes the MXFP4 activations in shared memory itself."""
     torch = _torch()
     _require(x, torch.bfloat16, "x")
     out_dtype = out_dtype or torch.bfloat16
@@ -348,7 +349,8 @@ def linear(x, w, out_dtype=None, y=None, workspace=None, fused=False):
     ws, ws_bytes = _workspace(need, dev, workspace)
     cw = w.c_struct()
     st = lib().macaq_linear_w4a4(x.data_ptr(), M, x.stride(0), ctypes.byref(cw), y.data_ptr(), y.stride(0),
-                                 _out_code(y.dtype), 1 if fused else 0, ws.data_ptr(), ws_bytes, _stream_ptr(dev))
+                                 _out_code(y.dtype), 2 if fused == "always" else 1 if fused else 0, ws.data_ptr(),
+                                 ws_bytes, _stream_ptr(dev))
     _check(st, "macaq_linear_w4a4")
     return y
 

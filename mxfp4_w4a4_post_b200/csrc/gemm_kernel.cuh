@@ -365,7 +365,8 @@ __device__ __forceinline__ Unit decode_unit(const GemmParams& p, int u, const CU
 // arrival (1 for the first arrival of the call). Lock-free: the compare-and-swap loop
 // only retries when another contributor of the same tile arrived in between.
 __device__ __forceinline__ uint32_t sk_arrive(unsigned long long* ctr, unsigned long long tag) {
-    unsigned long long cur = *reinterpret_cast<volatile unsigned long long*>(ctr);
+    // first guess: no arrival of this call yet (saves a read before the swap)
+    unsigned long long cur = tag << 16;
     for (;;) {
         const uint32_t n = (cur >> 16) == tag ? (uint32_t)(cur & 0xFFFFu) : 0u;
         const unsigned long long next = (tag << 16) | (unsigned long long)(n + 1);
@@ -814,7 +815,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const bool via_tma = S::kStagingBytes > 0 && p.tma_store;
         const uint32_t staging = ptx::smem_u32(smem + L::kOffStaging) + quad * S::kStageBoxBytes;
         volatile int* sk_last = reinterpret_cast<volatile int*>(smem + L::kOffMisc + 8);
-        constexpr bool kSkWidth = BN <= 64 && !GATHER;
+        constexpr bool kSkWidth = BN <= 32 && !GATHER;
         // The four epilogue warps leave the loop together: a stream-K tile synchronises
         // them on a named barrier, which a warp that had left alone would hold forever.
         for (int uj = 0; uj < sc.n_units; ++uj) {
@@ -825,7 +826,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const int prow = t.out_row0 + quad * 32 + lane;      // output row (transposed: column)
             const bool row_ok = quad * 32 + lane < t.rows;
             const uint32_t taddr = tmem + acc * S::kAccStride + ((uint32_t)(quad * 32) << 16);
-            // stream-K (planned for decode tiles of width <= 64 only): this CTA holds only
+            // stream-K (planned for decode tiles of width <= 32 only): this CTA holds only
             // part of the tile's K range
             const bool partial = kSkWidth && (t.kt_begin > 0 || t.kt_end < p.k_tiles);
             // write chunk c of y from registers: staged TMA store or direct stores

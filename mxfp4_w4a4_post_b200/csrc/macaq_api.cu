@@ -217,10 +217,6 @@ struct GemmPlan {
 // barriers and issue however narrow it is.
 inline double ktile_cycles(int bn) { return std::max(400.0, 2.42 * bn); }
 
-// Stream-K (decode orientation): a CTA takes at least this many K tiles, and a tile is
-// shared by at most this many CTAs (its finisher reads every contributor's partial).
-constexpr int64_t kSkMinIters = 3;
-constexpr int64_t kSkMaxContributors = 8;
 
 GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, int num_sms, bool allow_sk = true) {
     GemmPlan best{};
@@ -258,21 +254,22 @@ GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, int num_sms, bool allow_sk =
         }
     }
     // Decode: a weight-streaming product whose last round of tiles would leave SMs idle.
-    // Every CTA takes an even share of that round's K tiles first (stream-K), then its
-    // whole tiles; with fewer tiles than SMs, every tile is shared.
+    // Each tile of that round is split in two halves of its K range, taken by two CTAs
+    // before their whole tiles, so no CTA shares more than one tile and its fixup (one
+    // exchange of partial tiles through L2) overlaps the MMAs of its whole tile. Needs
+    // at most two halves per CTA: rest <= SMs / 2. Tiles up to 32 wide only: a wider
+    // tile's exchange (its finisher reads the partner's partial tile 16 columns at a
+    // time, each read an L2 round trip under a saturated HBM) costs more than the
+    // balance buys (64 wide: 32.7 against 29.0 us on the 64 x 25600 x 5120 product).
     const int64_t tiles = (int64_t)best.tiles_p * best.tiles_q;
-    if (allow_sk && best.swap && best.bn <= 64 && tiles % num_sms != 0 && best.k_tiles >= 2) {
+    if (allow_sk && best.swap && best.bn <= 32 && best.k_tiles >= 2) {
         const int64_t whole_rounds = tiles / num_sms;
         const int64_t rest = tiles - whole_rounds * num_sms;
-        int64_t grid = num_sms;
-        if (whole_rounds == 0)
-            grid = std::max<int64_t>(1, std::min<int64_t>({(int64_t)num_sms, tiles * best.k_tiles / kSkMinIters,
-                                                           tiles * kSkMaxContributors}));
-        if (grid > 1 && (whole_rounds > 0 || grid > tiles)) {
+        if (whole_rounds > 0 && rest > 0 && 2 * rest <= num_sms) {
             best.sk_tile0 = (int)(whole_rounds * num_sms);
             best.sk_iters = rest * best.k_tiles;
-            best.grid = (int)grid;
-            best.sk_ctas = (int)std::min<int64_t>(grid, best.sk_iters);
+            best.grid = num_sms;
+            best.sk_ctas = (int)(2 * rest);
         }
     }
     best.group_p = std::min(best.tiles_p, 16);
@@ -388,10 +385,13 @@ struct FusedAct {
     const void* x;
     int64_t ldx;
 };
-// Largest M the fused transform takes: the activation's MXFP4 form for every K tile
-// stays in shared memory beside the weight ring (one 16- or 32-row tile); larger M, or a
-// K whose tiles do not fit, runs the transform as its own kernel.
-constexpr int64_t kFusedMaxRows = 32;
+// Largest M the fused transform takes by default: every CTA repeats the transform of the
+// whole activation, which costs less than the separate launch only for a row or two
+// (measured on the Qwen3-32B up projection: fused 28.1 / 28.2 / 31.0 / 33.4 us against
+// 29.3 / 29.7 / 29.2 / 29.6 us for M = 1 / 2 / 4 / 8). The kernel itself takes up to 32
+// rows where their MXFP4 form fits in shared memory beside the weight ring.
+constexpr int64_t kFusedMaxRows = 2;
+constexpr int64_t kFusedKernelRows = 32;
 
 // Output written to several destinations (the gathered output of a column-parallel
 // layer): a device table of destination addresses, and whether all of them allow
@@ -584,7 +584,7 @@ macaq_status macaq_linear_w4a4(const void* x_bf16, int64_t M, int64_t ldx, const
                                macaq_stream stream) {
     macaq_status st = check_gemm_args(M, w, y, ldy, out);
     if (st != MACAQ_OK) return st;
-    if (fused != 0 && fused != 1) return MACAQ_ERR_INVALID_ARG;
+    if (fused < 0 || fused > 2) return MACAQ_ERR_INVALID_ARG;
     if (!w->inv_s) return MACAQ_ERR_INVALID_ARG;
     st = check_quant_args(x_bf16, M, w->K, ldx, w->inv_s, w->codes, w->scales);
     if (st != MACAQ_OK) return st;
@@ -595,7 +595,8 @@ macaq_status macaq_linear_w4a4(const void* x_bf16, int64_t M, int64_t ldx, const
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     uint8_t* a_codes = ws;
     uint8_t* a_scales = ws + off_scales;
-    if (fused == 1 && M <= kFusedMaxRows && fused_fits(M <= 16 ? 16 : 32, (int)cdiv(w->K, 256))) {
+    const int64_t fused_rows = fused == 2 ? kFusedKernelRows : fused == 1 ? kFusedMaxRows : 0;
+    if (M <= fused_rows && fused_fits(M <= 16 ? 16 : 32, (int)cdiv(w->K, 256))) {
         // one launch: the GEMM kernel makes the MXFP4 activations in shared memory itself
         // (the activation part of the workspace is not touched)
         const FusedAct fa{x_bf16, ldx};

@@ -14,7 +14,7 @@ buffer; each call is timed with CUDA events on the current stream and the mean i
 printed, one line per measured call:
     quant    macaq_quant_act on x (weights prepared first)
     gemm     macaq_gemm_mxfp4 on the quantised x and the prepared weight
-    linear   macaq_linear_w4a4 (fused = 0, or 1 with --fused)
+    linear   macaq_linear_w4a4 (fused = 0, or 2 with --fused: one launch whenever possible)
     hessian  macaq_hessian_blocks on T calibration rows (the workload's activation model
              with another seed) and macaq_prepare_weight_hessian on the weight
     moe      macaq_grouped_linear_w4a4 on T tokens routed over G experts (seeded skewed
@@ -308,9 +308,9 @@ def main(argv=None):
         else:
             ws_t = torch.empty(mq.linear_workspace_bytes(M, N, K, out), dtype=torch.uint8, device=dev)
             args = (x.data_ptr(), M, x.stride(0), ctypes.byref(cw), y.data_ptr(), y.stride(0), oc,
-                    1 if a.fused else 0, ws_t.data_ptr(), ws_t.numel(), stream)
+                    2 if a.fused else 0, ws_t.data_ptr(), ws_t.numel(), stream)
             t = _time(torch, lambda: call(lib.macaq_linear_w4a4, *args), flush, a.reps, a.warmup)
-            print(f"{line} linear_w4a4 fused={int(a.fused)} {t * 1e6:.2f} us {2.0 * M * N * K / t / 1e12:.1f} TFLOP/s")
+            print(f"{line} linear_w4a4 fused={2 if a.fused else 0} {t * 1e6:.2f} us {2.0 * M * N * K / t / 1e12:.1f} TFLOP/s")
     elif a.what == "flip":
         from dataclasses import replace
         xc = _bf16(torch, wl.draw_x(replace(L, M=a.calib, seed=L.seed + 100)), dev)

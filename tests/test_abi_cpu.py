@@ -82,7 +82,8 @@ def test_validation_rejects_bad_arguments(L):
     assert L.macaq_gemm_mxfp4(mis, a, 4, ctypes.byref(w), a, 128, 0, null, 0, None) == 2   # codes
     bad = mq.MacaqWeight(0x1000, 0x1000, 0x1000, 128, 250)
     assert L.macaq_gemm_mxfp4(a, a, 4, ctypes.byref(bad), a, 128, 0, null, 0, None) == 3
-    assert L.macaq_linear_w4a4(a, 4, 256, ctypes.byref(w), a, 128, 0, 2, a, 1 << 20, None) == 1  # fused not 0/1
+    assert L.macaq_linear_w4a4(a, 4, 256, ctypes.byref(w), a, 128, 0, 3, a, 1 << 20, None) == 1  # fused not 0..2
+    assert L.macaq_linear_w4a4(a, 4, 256, ctypes.byref(w), a, 128, 0, -1, a, 1 << 20, None) == 1
     # wait self-test: limit outside [1 us, 1 s] or no result array
     res = (ctypes.c_int64 * 10)()
     assert L.macaq_selftest_wait_timeout(0, res, None) == 1

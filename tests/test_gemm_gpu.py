@@ -122,7 +122,8 @@ def test_extreme_scales(mq):
 OUTPUT_CASES = [
     (300, 200, 512, "bf16", 0), (300, 200, 512, "f32", 0), (257, 333, 256, "bf16", 0),
     (300, 200, 512, "bf16", 24), (300, 200, 512, "f32", 12), (640, 1000, 768, "bf16", 0),
-    (16, 256, 25600, "bf16", 8), (64, 640, 12288, "f32", 3),     # stream-K, tiles shared by many CTAs
+    (16, 256, 25600, "bf16", 8), (64, 640, 12288, "f32", 3),     # deep K over few tiles
+    (1, 25600, 5120, "bf16", 8), (16, 19000, 5376, "f32", 4),    # stream-K: shared tiles
 ]
 
 
@@ -152,13 +153,13 @@ def test_output_paths(mq, M, N, K, dt, pad):
         assert np.array_equal(host(y).view(np.uint32), y32.view(np.uint32)), f"f32 {M}x{N}x{K} pad {pad}"
 
 
-@pytest.mark.parametrize("M,N,K", [(16, 256, 25600), (40, 1000, 8192), (64, 640, 12288), (1, 25600, 5120),
-                                   (32, 19200, 1024)])
+@pytest.mark.parametrize("M,N,K", [(1, 25600, 5120), (32, 19200, 1024), (24, 25600, 512), (16, 20000, 4096),
+                                   (5, 19000, 5376)])
 def test_stream_k_workspace_reuse(mq, M, N, K):
-    """Decode shapes on the stream-K schedule (the last round of output tiles, or all of
-    them when there are fewer tiles than SMs, dealt out K tile by K tile; a tile shared by
-    several CTAs is finished by the last to arrive from the partial tiles in the
-    workspace): two calls with different activations share one workspace that starts
+    """Decode shapes on the stream-K schedule (each tile of the last, partial round of
+    output tiles split in two K halves taken by two CTAs; a shared tile is finished by the
+    later of the two from the partial tiles in the workspace), odd K-tile counts
+    included: two calls with different activations share one workspace that starts
     filled with 0xFF bytes; both must match the oracle."""
     import torch
     rng = np.random.default_rng(M + N + K)

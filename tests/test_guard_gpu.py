@@ -86,18 +86,20 @@ def test_prepare_weight_guards(mq, N, K):
 
 
 # (M, N, K, out dtype, row stride of y): ragged rows and widths, narrow and wide tiles,
-# a stream-K case (small M, long K) whose partial tiles and counters live in the workspace
+# deep K over few tiles, and a stream-K case whose partial tiles and counters live in the
+# workspace
 GEMM_CASES = [
     (1, 16, 64, "f32", 20),
     (5, 200, 512, "bf16", 208),
     (200, 384, 512, "bf16", 392),
     (130, 136, 256, "f32", 140),
     (16, 256, 16384, "bf16", 264),
+    (8, 19100, 768, "f32", 19104),
 ]
 
 
 @pytest.mark.parametrize("M,N,K,dt,ld", GEMM_CASES)
-@pytest.mark.parametrize("fused", [False, True])
+@pytest.mark.parametrize("fused", [False, "always"])
 def test_linear_guards(mq, M, N, K, dt, ld, fused):
     import torch
     dtype = torch.float32 if dt == "f32" else torch.bfloat16

@@ -136,16 +136,18 @@ def test_device_error_word_is_clear(mq):
 
 
 # (M, N, K): decode shapes for the fused transform (one launch; the GEMM kernel makes
-# the MXFP4 activations in shared memory), a split-K shape, a K whose block count needs
-# scale padding and a partial last K tile, and two shapes above the fused row limit
-# (the call then runs the two-launch path).
-FUSED_CASES = [(1, 25600, 5120), (16, 25600, 5120), (32, 4096, 5120), (7, 300, 800), (16, 256, 25600),
-               (5, 1000, 96), (20, 700, 4128), (64, 4096, 5120), (128, 1024, 768)]
+# the MXFP4 activations in shared memory; also on the stream-K schedule), a K whose block
+# count needs scale padding and a partial last K tile, shapes beyond the default row
+# limit of the fused path, and two above what the kernel takes (the call then runs the
+# two-launch path).
+FUSED_CASES = [(1, 25600, 5120), (2, 19000, 4096), (1, 300, 800), (2, 1000, 96), (1, 700, 4128),
+               (16, 25600, 5120), (32, 4096, 5120), (7, 300, 800), (64, 4096, 5120), (128, 1024, 768)]
 
 
 @pytest.mark.parametrize("M,N,K", FUSED_CASES)
 def test_fused_transform(mq, M, N, K):
-    """macaq_linear_w4a4 with fused = 1: y is bit-identical to the two-launch layer
+    """macaq_linear_w4a4 with fused = 2 (one launch wherever the kernel takes the shape) and
+    fused = 1 (one launch where it is faster): y is bit-identical to the two-launch layer
     (fused = 0: the quantiser kernel, then the GEMM with the same tile plan), for fp32 and
     bf16 output, on two inputs in a row through one workspace, and within the GEMM
     tolerance of the oracle."""
@@ -159,12 +161,14 @@ def test_fused_transform(mq, M, N, K):
     for seed in (21, 22):
         x = wl.draw_x(wl.with_shape(L, seed=seed))
         xd = bf16_dev(x)
-        y = mq.linear(xd, pw, out_dtype=torch.float32, workspace=ws, fused=True)
+        y = mq.linear(xd, pw, out_dtype=torch.float32, workspace=ws, fused="always")
         y_two = mq.linear(xd, pw, out_dtype=torch.float32, fused=False)
-        y16 = mq.linear(xd, pw, out_dtype=torch.bfloat16, workspace=ws, fused=True)
+        y_auto = mq.linear(xd, pw, out_dtype=torch.float32, fused=True)
+        y16 = mq.linear(xd, pw, out_dtype=torch.bfloat16, workspace=ws, fused="always")
         y16_two = mq.linear(xd, pw, out_dtype=torch.bfloat16, fused=False)
         torch.cuda.synchronize()
         assert np.array_equal(host(y).view(np.uint32), host(y_two).view(np.uint32)), f"fused {M}x{N}x{K} fp32"
+        assert np.array_equal(host(y_auto).view(np.uint32), host(y_two).view(np.uint32)), f"fused=1 {M}x{N}x{K}"
         assert torch.equal(y16.view(torch.int16), y16_two.view(torch.int16)), f"fused {M}x{N}x{K} bf16"
         rac, ras = oracle.quant_rows(x, rinv)
         assert_gemm_close(host(y), oracle.gemm_fp64(rac, ras, rwc, rws, K), f"fused {M}x{N}x{K} seed {seed}")
@@ -181,7 +185,7 @@ def test_fused_transform_strided(mq):
     wide[:, :K] = x
     xd = bf16_dev(wide)[:, :K]
     pw = mq.prepare_weight(bf16_dev(W), f32_dev(s))
-    y = mq.linear(xd, pw, out_dtype=torch.float32, fused=True)
+    y = mq.linear(xd, pw, out_dtype=torch.float32, fused="always")
     y_two = mq.linear(bf16_dev(x), pw, out_dtype=torch.float32, fused=False)
     torch.cuda.synchronize()
     assert np.array_equal(host(y).view(np.uint32), host(y_two).view(np.uint32))
