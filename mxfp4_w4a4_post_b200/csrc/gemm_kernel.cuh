@@ -164,15 +164,17 @@ struct GemmShape {
     static constexpr int kStagingBytes = BN >= 128 ? 4 * kStageBoxBytes : 0;
 };
 
-template <int BN, int STAGES, bool FUSED = false>
+template <int BN, int STAGES, bool FUSED = false, bool PAIR = false>
 struct GemmSmem {
     using S = GemmShape<BN, STAGES>;
     // the fused variant keeps its Q operand for every K tile in one persistent region
     // after the fixed layout instead of in the stage ring
     static constexpr int kQRing = FUSED ? 0 : 1;
+    // a CTA of a pair holds half of the Q tile's rows (and the scales of all of them)
+    static constexpr int kQStageBytes = PAIR ? S::kQTileBytes / 2 : S::kQTileBytes;
     static constexpr int kOffP = 0;
     static constexpr int kOffQ = kOffP + STAGES * S::kPTileBytes;
-    static constexpr int kOffSfP = kOffQ + kQRing * STAGES * S::kQTileBytes;
+    static constexpr int kOffSfP = kOffQ + kQRing * STAGES * kQStageBytes;
     static constexpr int kOffSfQ = kOffSfP + STAGES * S::kSfChunkBytes;
     static constexpr int kOffStaging = kOffSfQ + kQRing * STAGES * S::kQChunks * S::kSfChunkBytes;   // 1 KB aligned
     static constexpr int kOffBar = kOffStaging + S::kStagingBytes;
@@ -269,9 +271,10 @@ struct Unit {
 // .. below sk_tile0 (grouped GEMM: every tile is whole).
 struct Sched {
     int n_sk, sk_first, n_units;
+    int base, stride;            // whole tiles base, base + stride, ..
     int64_t i0, i1;
     __device__ __forceinline__ int unit(int j) const {
-        return j < n_sk ? sk_first + j : (int)blockIdx.x + (j - n_sk) * (int)gridDim.x;
+        return j < n_sk ? sk_first + j : base + (j - n_sk) * stride;
     }
 };
 
@@ -279,9 +282,12 @@ __device__ __forceinline__ int64_t sk_start(const GemmParams& p, int c) {
     return (int64_t)c * p.sk_iters / p.sk_ctas;
 }
 
-__device__ __forceinline__ Sched cta_sched(const GemmParams& p) {
+// pair: the two CTAs of a cluster work through the same units (G = gridDim.x / 2).
+__device__ __forceinline__ Sched cta_sched(const GemmParams& p, bool pair = false) {
     Sched s;
     const int whole = p.groups > 0 ? p.total_units : p.sk_tile0;
+    s.base = pair ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+    s.stride = pair ? (int)(gridDim.x >> 1) : (int)gridDim.x;
     s.i0 = 0;
     s.i1 = 0;
     s.n_sk = 0;
@@ -294,7 +300,7 @@ __device__ __forceinline__ Sched cta_sched(const GemmParams& p) {
             s.n_sk = p.sk_tile0 + (int)((s.i1 - 1) / p.k_tiles) + 1 - s.sk_first;
         }
     }
-    const int n_whole = (int)blockIdx.x < whole ? (whole - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+    const int n_whole = s.base < whole ? (whole - 1 - s.base) / s.stride + 1 : 0;
     s.n_units = s.n_sk + n_whole;
     return s;
 }
@@ -306,7 +312,10 @@ __device__ __forceinline__ int sk_cta_of(const GemmParams& p, int64_t j) {
     return (int)(((j + 1) * p.sk_ctas - 1) / p.sk_iters);
 }
 
-__device__ __forceinline__ Unit decode_unit(const GemmParams& p, int u, const CUtensorMap* tmap_q, const Sched& sc) {
+// rank >= 0: CTA `rank` of a pair, whose unit is a 256-row tile (tp counts 256 rows) of
+// which this CTA holds rows 128 rank .. 128 rank + 127.
+__device__ __forceinline__ Unit decode_unit(const GemmParams& p, int u, const CUtensorMap* tmap_q, const Sched& sc,
+                                            int rank = -1) {
     if (p.groups > 0) {
         // the group whose units contain u: binary search over the unit offsets
         int lo = 0, hi = p.groups - 1;
@@ -350,9 +359,9 @@ __device__ __forceinline__ Unit decode_unit(const GemmParams& p, int u, const CU
         x.kt_begin = (int)(max(sc.i0, t0) - t0);
         x.kt_end = (int)(min(sc.i1, t0 + p.k_tiles) - t0);
     }
-    x.p_row0 = x.tp * 128;
-    x.out_row0 = x.tp * 128;
-    x.rows = p.p_rows - x.tp * 128;
+    x.p_row0 = rank >= 0 ? x.tp * 256 + rank * 128 : x.tp * 128;
+    x.out_row0 = x.p_row0;
+    x.rows = p.p_rows - x.p_row0;
     x.q_rows = p.q_rows;
     x.tmap_q = tmap_q;
     x.sf_q = p.sf_q;
@@ -464,8 +473,9 @@ constexpr int kGemmThreads = 32 * (6 + 4 * kSfWarpSets);
 
 // Kernel variants, each its own instantiation so that the ordinary kernels keep their
 // registers: kVarGather writes the output to p.dest[0 .. p.n_dest - 1]; kVarFused makes
-// the Q operand (the activations) from bf16 inside the kernel.
-enum : int { kVarPlain = 0, kVarGather = 1, kVarFused = 2 };
+// the Q operand (the activations) from bf16 inside the kernel; kVarPair runs on clusters
+// of two CTAs, each pair computing 256 x BN tiles with cta_group::2 MMAs (prefill).
+enum : int { kVarPlain = 0, kVarGather = 1, kVarFused = 2, kVarPair = 3 };
 
 // The fused variant's Q operand, made once per CTA before its main loop by warps 2-13
 // (the epilogue and scale-factor warps; the producer starts streaming the weight tiles
@@ -569,10 +579,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                      const __grid_constant__ CUtensorMap tmap_y, const GemmParams p) {
     constexpr bool GATHER = VAR == kVarGather;
     constexpr bool FUSED = VAR == kVarFused;
+    constexpr bool PAIR = VAR == kVarPair;
     // The fused variant covers Q tiles of at most 32 rows (one 128-row scale slab).
     static_assert(!FUSED || BN <= 32, "fused transform tile");
+    // A pair splits its Q tile in two halves of whole 8-row swizzle atoms; prefill only.
+    static_assert(!PAIR || BN == 128 || BN == 192, "pair tile");
     using S = GemmShape<BN, STAGES>;
-    using L = GemmSmem<BN, STAGES, FUSED>;
+    using L = GemmSmem<BN, STAGES, FUSED, PAIR>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -588,6 +601,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    // CTA pair: rank 0 issues the MMAs of both; rank 1's scale-factor writers and
+    // epilogue signal rank 0's sf_full and acc_empty barriers remotely, and rank 0's
+    // commits arrive on both CTAs' stage and accumulator barriers.
+    const int rank = PAIR ? (int)ptx::cluster_ctarank() : -1;
+    constexpr uint32_t kPeerArrivals = PAIR ? 2 : 1;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -596,10 +614,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         for (int a = 0; a < 2; ++a) {
             ptx::mbar_init(&acc_full[a], 1);
-            ptx::mbar_init(&acc_empty[a], 4);
+            ptx::mbar_init(&acc_empty[a], 4 * kPeerArrivals);
         }
         ptx::mbar_init(drain, 1);
-        for (int s = 0; s < STAGES; ++s) ptx::mbar_init(&sf_full[s], 4);
+        for (int s = 0; s < STAGES; ++s) ptx::mbar_init(&sf_full[s], 4 * kPeerArrivals);
         *abort = 0;
         ptx::fence_mbar_init();
         ptx::fence_proxy_async_smem();
@@ -608,14 +626,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (S::kStagingBytes > 0 && p.tma_store) ptx::prefetch_tensormap(&tmap_y);
     }
     if (warp == 1) {
-        ptx::tmem_alloc(tmem_slot, S::kTmemCols);
-        ptx::tmem_relinquish();
+        if constexpr (PAIR) {
+            ptx::tmem_alloc_pair(tmem_slot, S::kTmemCols);
+            ptx::tmem_relinquish_pair();
+        } else {
+            ptx::tmem_alloc(tmem_slot, S::kTmemCols);
+            ptx::tmem_relinquish();
+        }
     }
     ptx::tc_fence_before();
     __syncthreads();
+    // the other CTA of a pair signals this CTA's barriers only after they are set up
+    if constexpr (PAIR) ptx::cluster_sync();
     ptx::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const Sched sc = cta_sched(p);
+    const Sched sc = cta_sched(p, PAIR);
     // Set-up above overlaps the previous kernel's tail; operands are read only after it.
     ptx::griddep_wait();
     ptx::griddep_launch_dependents();
@@ -633,7 +658,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         uint32_t issued_mask = 0, issued_phase = 0;
         // Q side of one fill: codes tile and scale chunks
         auto issue_q = [&](const Unit& t, int st, int kt, int q0, int slab0, int nchunks) {
-            ptx::tma_load_2d(smem + L::kOffQ + st * S::kQTileBytes, t.tmap_q, &full[st], kt * S::kBKBytes, q0);
+            // a pair's CTA copies its half of the Q tile's rows, and the scales of all
+            ptx::tma_load_2d(smem + L::kOffQ + st * L::kQStageBytes, t.tmap_q, &full[st], kt * S::kBKBytes,
+                             PAIR ? q0 + rank * (BN / 2) : q0);
             for (int c = 0; c < nchunks; ++c)
                 ptx::bulk_load(smem + L::kOffSfQ + (st * S::kQChunks + c) * S::kSfChunkBytes,
                                t.sf_q + ((int64_t)(slab0 + c) * p.kb4_pad + 2 * kt) * 512, S::kSfChunkBytes,
@@ -642,13 +669,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         for (int uj = 0; uj < sc.n_units; ++uj) {
             const int u = sc.unit(uj);
             if (cta_aborted(abort)) break;
-            const Unit t = decode_unit(p, u, &tmap_q, sc);
+            const Unit t = decode_unit(p, u, &tmap_q, sc, rank);
             const int q0 = t.tq * BN;
             const int slab0 = q0 / 128;
             const int nchunks = min(S::kQChunks, (t.q_rows + 127) / 128 - slab0);   // scale slabs of the Q rows
+            // P scale slab of the tile; a pair's second CTA past the last P row (its rows
+            // are all zero-filled codes, and their results are never stored) reads slab 0
+            const int slab_p = t.rows > 0 ? (t.p_row0 >> 7) : 0;
             // the fused variant copies only the weight side; its Q side is made in place
             const uint32_t bytes = FUSED ? S::kPTileBytes + S::kSfChunkBytes
-                                         : S::kPTileBytes + S::kQTileBytes + S::kSfChunkBytes * (1 + nchunks);
+                                         : S::kPTileBytes + L::kQStageBytes + S::kSfChunkBytes * (1 + nchunks);
             bool ok = true;
             for (int kt = t.kt_begin; kt < t.kt_end; ++kt) {
                 if (!warp_wait(&empty[stage], phase ^ 1, abort, p.err, kErrTimeoutProducer)) { ok = false; break; }
@@ -657,8 +687,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     ptx::tma_load_2d(smem + L::kOffP + stage * S::kPTileBytes, &tmap_p, &full[stage],
                                      kt * S::kBKBytes, t.p_row0);
                     ptx::bulk_load(smem + L::kOffSfP + stage * S::kSfChunkBytes,
-                                   p.sf_p + ((int64_t)(t.p_row0 >> 7) * p.kb4_pad + 2 * kt) * 512,
-                                   S::kSfChunkBytes, &full[stage]);
+                                   p.sf_p + ((int64_t)slab_p * p.kb4_pad + 2 * kt) * 512, S::kSfChunkBytes,
+                                   &full[stage]);
                     if constexpr (!FUSED) issue_q(t, stage, kt, q0, slab0, nchunks);
                 }
                 __syncwarp();
@@ -680,8 +710,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             }
         }
         __syncwarp();
-    } else if (warp == 1) {
+    } else if (warp == 1 && rank <= 0) {
         // -------------------------------------------------------------- MMA -----
+        // (a pair's MMAs are issued by its rank-0 CTA alone; they wait for both CTAs'
+        // scale slots and accumulators, and their commits arrive in both CTAs)
         // Whole-warp loop with warp-uniform descriptors; the elected lane issues the
         // MMAs and the commits (a commit tracks the MMAs of the thread that issues it).
         // A K tile is ready once its scale-factor slot is: the scale-factor warps arrive
@@ -695,7 +727,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         for (int uj = 0; uj < sc.n_units; ++uj) {
             const int u = sc.unit(uj);
             if (cta_aborted(abort)) break;
-            const Unit t = decode_unit(p, u, &tmap_q, sc);
+            const Unit t = decode_unit(p, u, &tmap_q, sc, rank);
             const uint32_t q_off = (uint32_t)((t.tq * BN) % 128) / 32;
             if ((q_off & 1) != 0 || q_off * 32 + (BN < 32 ? 32 : BN) > 128 * S::kQChunks) {
                 // never planned: a scale-factor column offset the MMA is not given
@@ -716,7 +748,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 const uint32_t sf_base = tmem + S::kSfBase + stage * S::kSfCols;
                 const uint64_t adesc = ptx::smem_desc_sw128(ptx::smem_u32(smem + L::kOffP + stage * S::kPTileBytes));
                 const uint64_t bdesc = ptx::smem_desc_sw128(ptx::smem_u32(
-                    FUSED ? smem + L::kOffPersist + kt * S::kQTileBytes : smem + L::kOffQ + stage * S::kQTileBytes));
+                    FUSED ? smem + L::kOffPersist + kt * S::kQTileBytes : smem + L::kOffQ + stage * L::kQStageBytes));
                 if (leader) {
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk) {
@@ -724,18 +756,26 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         const uint32_t sfid = (kk & 1) * 2;
                         const uint32_t sfa = (sf_base + 4 * a) | (sfid << 30);
                         const uint32_t sfb = (sf_base + 8 + a * 4 * S::kQChunks + q_off) | (sfid << 30);
-                        ptx::mma_mxf4(d_tmem + (kk % S::kSub) * BN, adesc + 2 * kk, bdesc + 2 * kk,
-                                      ptx::idesc_mxf4(BN, sfid, sfid), sfa, sfb,
-                                      (kt > t.kt_begin || kk >= S::kSub) ? 1u : 0u);
+                        const uint32_t acc_in = (kt > t.kt_begin || kk >= S::kSub) ? 1u : 0u;
+                        if constexpr (PAIR)
+                            ptx::mma_mxf4_pair(d_tmem, adesc + 2 * kk, bdesc + 2 * kk,
+                                               ptx::idesc_mxf4(BN, sfid, sfid, 256), sfa, sfb, acc_in);
+                        else
+                            ptx::mma_mxf4(d_tmem + (kk % S::kSub) * BN, adesc + 2 * kk, bdesc + 2 * kk,
+                                          ptx::idesc_mxf4(BN, sfid, sfid), sfa, sfb, acc_in);
                     }
-                    ptx::tc_commit(&empty[stage]);
+                    if constexpr (PAIR) ptx::tc_commit_pair(&empty[stage], 3);
+                    else ptx::tc_commit(&empty[stage]);
                 }
                 __syncwarp();
                 issued = true;
                 if (++stage == STAGES) { stage = 0; phase ^= 1; }
             }
             if (!ok) break;
-            if (leader) ptx::tc_commit(&acc_full[acc]);
+            if (leader) {
+                if constexpr (PAIR) ptx::tc_commit_pair(&acc_full[acc], 3);
+                else ptx::tc_commit(&acc_full[acc]);
+            }
             __syncwarp();
             if (S::kNumAcc == 2) {
                 acc ^= 1;
@@ -746,12 +786,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         if (cta_aborted(abort) && issued && leader) {
             // wait (bounded) for every MMA this thread issued before TMEM is freed
-            ptx::tc_commit(drain);
+            if constexpr (PAIR) ptx::tc_commit_pair(drain, 1);
+            else ptx::tc_commit(drain);
             const uint64_t t0 = global_timer_ns();
             while (!ptx::mbar_try_wait(drain, 0) && global_timer_ns() - t0 < 100000000ull) {
             }
         }
         __syncwarp();
+    } else if (warp == 1) {
+        // rank 1 of a pair: no MMAs of its own to issue
     } else if (warp >= 6) {
         // ------------------------------------------------- scale-factor writers ---
         // Warp q' (= warp % 4) owns TMEM lanes 32q'..32q'+31. In the 128x4 scale atom,
@@ -767,7 +810,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         uint32_t kt_count = 0;
         for (int uj = 0; uj < sc.n_units && !*abort; ++uj) {
             const int u = sc.unit(uj);
-            const Unit t = decode_unit(p, u, &tmap_q, sc);
+            const Unit t = decode_unit(p, u, &tmap_q, sc, rank);
             bool ok = true;
             for (int kt = t.kt_begin; kt < t.kt_end; ++kt, ++kt_count) {
                 // Every set waits for every fill, in order, even those it does not
@@ -800,7 +843,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 ptx::tmem_st_wait();
                 ptx::tc_fence_before();
                 __syncwarp();
-                if (lane == 0) ptx::mbar_arrive(&sf_full[stage]);
+                if (lane == 0) {
+                    if (rank > 0) ptx::mbar_arrive_remote(ptx::mapa_shared(&sf_full[stage], 0));
+                    else ptx::mbar_arrive(&sf_full[stage]);
+                }
                 if (++stage == STAGES) { stage = 0; phase ^= 1; }
             }
             if (!ok) break;
@@ -820,7 +866,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         // them on a named barrier, which a warp that had left alone would hold forever.
         for (int uj = 0; uj < sc.n_units; ++uj) {
             const int u = sc.unit(uj);
-            const Unit t = decode_unit(p, u, &tmap_q, sc);
+            const Unit t = decode_unit(p, u, &tmap_q, sc, rank);
             if (!bar_and(1, 128, wait_or_abort(&acc_full[acc], acc_phase, abort, p.err, kErrTimeoutEpilogue))) break;
             ptx::tc_fence_after();
             const int prow = t.out_row0 + quad * 32 + lane;      // output row (transposed: column)
@@ -905,7 +951,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     // the accumulator is in registers: hand it back to the MMA warp now
                     ptx::tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) ptx::mbar_arrive(&acc_empty[acc]);
+                    if (lane == 0) {
+                        if (rank > 0) ptx::mbar_arrive_remote(ptx::mapa_shared(&acc_empty[acc], 0));
+                        else ptx::mbar_arrive(&acc_empty[acc]);
+                    }
                 }
                 if (!partial) {
                     emit(c, r);
@@ -981,9 +1030,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
     ptx::tc_fence_before();
     __syncthreads();
+    // a pair's CTAs leave together: neither frees its TMEM or shared memory while the
+    // other may still signal it or its MMAs may still write there
+    if constexpr (PAIR) ptx::cluster_sync();
     if (warp == 1) {
         ptx::tc_fence_after();
-        ptx::tmem_dealloc(tmem, S::kTmemCols);
+        if constexpr (PAIR) ptx::tmem_dealloc_pair(tmem, S::kTmemCols);
+        else ptx::tmem_dealloc(tmem, S::kTmemCols);
     }
 }
 

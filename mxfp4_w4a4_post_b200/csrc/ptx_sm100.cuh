@@ -77,6 +77,37 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
+// ------------------------------------------------------------------ cluster -----
+// (the CTA pair of the kernel's two-SM instantiation: clusters of two CTAs)
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+// Shared-memory address, in the cluster window, of `p`'s counterpart in CTA `rank`.
+__device__ __forceinline__ uint32_t mapa_shared(const void* p, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+    return r;
+}
+
+// Arrive on an mbarrier of another CTA of the cluster (address from mapa_shared). The
+// waiter uses an ordinary try_wait: what it orders are tcgen05 operations, which the
+// arriving thread completes (tcgen05.wait) and fences (tcgen05.fence::before_thread_sync)
+// before it arrives, and the waiter fences (tcgen05.fence::after_thread_sync) after.
+// (Release and acquire at cluster scope on these barriers made every K tile of the pair
+// kernel ~0.23 us slower: 170 against 102 us for 4096 x 14336 x 4096.)
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+// Every thread of both CTAs of the cluster: arrive, then wait for all.
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
 // --------------------------------------------------------------------- TMA ------
 
 __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* map, uint64_t* bar,
@@ -146,6 +177,24 @@ __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
                  : "memory");
 }
 
+// The same three for a CTA pair (cta_group::2): the warp with the same index in both CTAs
+// of the cluster issues them together, and gets the same TMEM address in each.
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* smem_result, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(smem_result)),
+                 "r"(ncols)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_relinquish_pair() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+                 : "memory");
+}
+
 __device__ __forceinline__ void tc_fence_before() {
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
 }
@@ -163,6 +212,16 @@ __device__ __forceinline__ void tc_commit(uint64_t* bar) {
         : "memory");
 }
 
+// CTA pair: arrive on the mbarrier at `bar`'s offset in every CTA of `cta_mask` once
+// every tcgen05 async operation this thread issued so far has completed.
+__device__ __forceinline__ void tc_commit_pair(uint64_t* bar, uint16_t cta_mask) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+            smem_u32(bar)),
+        "h"(cta_mask)
+        : "memory");
+}
+
 // Block-scaled FP4 MMA, D[tmem] (+)= A[smem] * B[smem]^T with E8M0 scales from TMEM,
 // K = 64 per instruction, one scale per 32 elements (two per row per instruction).
 __device__ __forceinline__ void mma_mxf4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
@@ -172,6 +231,22 @@ __device__ __forceinline__ void mma_mxf4(uint32_t d_tmem, uint64_t a_desc, uint6
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.scale_vec::2X"
+        " [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+        : "memory");
+}
+
+// The same over a CTA pair (issued by the even CTA): M = 256, the A rows of CTA r at
+// rows 128 r .. 128 r + 127, the B rows of CTA r at rows r N/2 .. (r + 1) N/2 - 1, each
+// CTA's operands at the same shared-memory offsets; each CTA's TMEM holds its 128 rows of
+// D, the scales of its A rows and the scales of all N B rows, at the same addresses.
+__device__ __forceinline__ void mma_mxf4_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                              uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
+                                              uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::mxf4.block_scale.scale_vec::2X"
         " [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
         : "memory");
@@ -255,14 +330,14 @@ __device__ __forceinline__ uint64_t smem_desc_sf(uint32_t saddr) {
 }
 
 // Instruction descriptor of kind::mxf4 block-scaled MMA: E2M1 x E2M1, E8M0 scales,
-// fp32 accumulate, both operands K-major, M = 128, N = n.
-__host__ __device__ constexpr uint32_t idesc_mxf4(int n, uint32_t a_sf_id, uint32_t b_sf_id) {
+// fp32 accumulate, both operands K-major, M = m (128, or 256 over a CTA pair), N = n.
+__host__ __device__ constexpr uint32_t idesc_mxf4(int n, uint32_t a_sf_id, uint32_t b_sf_id, int m = 128) {
     return (b_sf_id << 4)                 // B scale-factor byte id
            | (1u << 7)                    // A format: E2M1
            | (1u << 10)                   // B format: E2M1
            | ((uint32_t)(n >> 3) << 17)   // N / 8
            | (1u << 23)                   // scale format: E8M0
-           | ((uint32_t)(128 >> 4) << 24) // M / 16
+           | ((uint32_t)(m >> 4) << 24)   // M / 16
            | (a_sf_id << 29);             // A scale-factor byte id
 }
 

@@ -1,9 +1,9 @@
 """Parity of the block-scaled FP4 GEMM (tcgen05 kind::mxf4) with the oracle's fp64 sum
 of decoded products. One-hot operands pin the nibble order and the scale layout;
 random codes and scales cover every tile path (swapped decode tiles of width 16..128,
-prefill tiles of width 128/192, the stream-K schedule whose shared tiles are finished by
-their last contributor, ragged M/N/K) and every output path (TMA tensor stores of staged
-boxes, direct stores, transposed stores)."""
+prefill tiles of width 128/192, 256 x 192 tiles of CTA pairs, the stream-K schedule
+whose shared tiles are finished by their last contributor, ragged M/N/K) and every
+output path (TMA tensor stores of staged boxes, direct stores, transposed stores)."""
 import numpy as np
 import pytest
 
@@ -52,7 +52,9 @@ def one_hot_operands(M, N, K, picks):
     return pack(a), sa, pack(w), sw
 
 
-@pytest.mark.parametrize("M,N,K", [(16, 128, 256), (300, 448, 512), (200, 130, 768)])
+# the last shape runs on CTA pairs (rows 128..255 of each 256-row tile, and weight rows
+# 96..191 of each 192-row tile, in the second CTA of the pair)
+@pytest.mark.parametrize("M,N,K", [(16, 128, 256), (300, 448, 512), (200, 130, 768), (700, 4200, 768)])
 def test_one_hot_layout(mq, M, N, K):
     rng = np.random.default_rng(M + N + K)
     picks, used_k, used_m, used_n = [], set(), set(), set()
@@ -80,6 +82,10 @@ SHAPES = [
     (1, 128, 256), (3, 300, 512), (16, 1000, 1024), (17, 256, 5120), (32, 2000, 2048),
     (64, 640, 4096), (100, 384, 1280), (128, 512, 768),
     (129, 224, 256), (256, 1024, 5120), (300, 700, 800), (512, 2240, 2048), (1000, 130, 1536),
+    # CTA pairs: a 256-row tile whose second CTA has no rows (M % 256 = 44) or 8 of 128
+    # rows in the first, and a last weight tile whose second half is empty (N % 192 = 88)
+    # or partly filled (N % 192 = 168)
+    (300, 7000, 768), (520, 4200, 768),
 ]
 
 
@@ -124,6 +130,8 @@ OUTPUT_CASES = [
     (300, 200, 512, "bf16", 24), (300, 200, 512, "f32", 12), (640, 1000, 768, "bf16", 0),
     (16, 256, 25600, "bf16", 8), (64, 640, 12288, "f32", 3),     # deep K over few tiles
     (1, 25600, 5120, "bf16", 8), (16, 19000, 5376, "f32", 4),    # stream-K: shared tiles
+    (700, 4200, 256, "bf16", 0), (300, 7000, 768, "f32", 4),     # CTA pairs
+    (1000, 6100, 768, "bf16", 8),                                # CTA pairs, unaligned rows
 ]
 
 

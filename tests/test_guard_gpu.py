@@ -95,6 +95,7 @@ GEMM_CASES = [
     (130, 136, 256, "f32", 140),
     (16, 256, 16384, "bf16", 264),
     (8, 19100, 768, "f32", 19104),
+    (700, 4200, 256, "bf16", 4216),          # CTA pairs, ragged second CTA and weight half
 ]
 
 

@@ -109,7 +109,7 @@ def test_module_with_nccl_one_rank(mq):
 
 # (M, N, K, shards): prefill tiles, decode (swapped) tiles, and a shape for which the
 # ordinary layer runs on the stream-K schedule (the gathered output never does)
-GATHER_CASES = [(200, 520, 1024, 2), (5, 300, 512, 3), (16, 256, 16384, 2)]
+GATHER_CASES = [(200, 520, 1024, 2), (5, 300, 512, 3), (16, 256, 16384, 2), (8, 40000, 512, 2)]
 
 
 @pytest.mark.parametrize("M,N,K,shards", GATHER_CASES)
