@@ -93,10 +93,11 @@ size_t macaq_codes_bytes(int64_t rows, int64_t K);
 size_t macaq_scales_bytes(int64_t rows, int64_t K);
 
 /* Device workspace macaq_gemm_mxfp4 needs for an M x N x K product with output
- * `out`: when the library runs the product on a stream-K schedule (shapes with few
- * output tiles per SM: the K tiles of all output tiles are dealt out evenly over the
- * CTAs, so a tile may be shared by several), two fp32 partial tiles per CTA and an
- * arrival counter per output tile; 0 otherwise. Its contents need no clearing. */
+ * `out`: when the library runs the product on its stream-K schedule (decode shapes,
+ * M <= 32, whose last round of weight tiles would leave SMs idle: each tile of that
+ * round is split in two halves of its K range taken by two CTAs), two fp32 partial
+ * tiles per CTA and an arrival counter per output tile; 0 otherwise. Its contents need
+ * no clearing. */
 size_t macaq_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, macaq_out_dtype out);
 
 /* Device workspace macaq_linear_w4a4 needs: the activation codes and scales, then the
@@ -138,7 +139,9 @@ macaq_status macaq_quant_act(const void* x_bf16, int64_t M, int64_t K, int64_t l
  * that follows the activation transform; W4A4 definition in the openai-hub.com
  * article):
  *   y[m, n] = sum_b 2^(ea[m,b] + ew[n,b]) * sum_{k in b} dec(a[m,k]) * dec(w[n,k]),
- * fp32 accumulation on the tensor cores (tcgen05 kind::mxf4).
+ * fp32 accumulation on the tensor cores (tcgen05 kind::mxf4). Large prefill products
+ * run on clusters of two CTAs (256-row tiles, cta_group::2 MMAs), the rest on single
+ * CTAs; the choice is the library's and does not change the result's tolerance.
  *   a_codes/a_scales device, as written by macaq_quant_act for M rows
  *   w        prepared weight (inv_s unused here)
  *   y        device [M x N] fp32 or bf16, row stride ldy elements (ldy >= N), aligned
