@@ -119,6 +119,14 @@ struct GemmParams {
     // in the kernel's parameters.
     int32_t n_dest;
     unsigned long long dest[kMaxGatherDest];
+    // 1: the producer may copy the weight side of its first fills before waiting for the
+    // previous kernel on the stream (set by the layer entry points, which launch their
+    // own activation transform just before the GEMM)
+    int32_t w_early;
+    // K split over a cluster (the kernel's SPLIT instantiation): `split` CTAs per cluster,
+    // one output tile per cluster, CTA r accumulating K tiles [r k / split, (r + 1) k /
+    // split) of it; CTA 0 adds the others' partial tiles, read from their shared memory.
+    int32_t split;
 };
 
 enum : int {
@@ -126,7 +134,8 @@ enum : int {
     kErrTimeoutMma = 2,
     kErrTimeoutEpilogue = 3,
     kErrSfOffset = 4,
-    kErrTimeoutSet = 5
+    kErrTimeoutSet = 5,
+    kErrPlan = 6              // a cluster launch the K-split kernel is not planned for
 };
 
 template <int BN, int STAGES>
@@ -178,7 +187,7 @@ struct GemmSmem {
     static constexpr int kOffSfQ = kOffSfP + STAGES * S::kSfChunkBytes;
     static constexpr int kOffStaging = kOffSfQ + kQRing * STAGES * S::kQChunks * S::kSfChunkBytes;   // 1 KB aligned
     static constexpr int kOffBar = kOffStaging + S::kStagingBytes;
-    static constexpr int kNumBars = 3 * STAGES + 4 + 1;
+    static constexpr int kNumBars = 3 * STAGES + 4 + 1 + 2;    // ..., sf_full[STAGES], part_full, ring_free
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;
     static constexpr int kBytes = kOffMisc + 16;
     // fused: Q codes of K tile kt at kOffPersist + kt * BN * 128 (128-byte swizzle, as the
@@ -282,12 +291,13 @@ __device__ __forceinline__ int64_t sk_start(const GemmParams& p, int c) {
     return (int64_t)c * p.sk_iters / p.sk_ctas;
 }
 
-// pair: the two CTAs of a cluster work through the same units (G = gridDim.x / 2).
-__device__ __forceinline__ Sched cta_sched(const GemmParams& p, bool pair = false) {
+// cluster > 1: the CTAs of a cluster work through the same units (G = gridDim.x /
+// cluster).
+__device__ __forceinline__ Sched cta_sched(const GemmParams& p, int cluster = 1) {
     Sched s;
     const int whole = p.groups > 0 ? p.total_units : p.sk_tile0;
-    s.base = pair ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
-    s.stride = pair ? (int)(gridDim.x >> 1) : (int)gridDim.x;
+    s.base = (int)blockIdx.x / cluster;
+    s.stride = (int)gridDim.x / cluster;
     s.i0 = 0;
     s.i1 = 0;
     s.n_sk = 0;
@@ -313,7 +323,8 @@ __device__ __forceinline__ int sk_cta_of(const GemmParams& p, int64_t j) {
 }
 
 // rank >= 0: CTA `rank` of a pair, whose unit is a 256-row tile (tp counts 256 rows) of
-// which this CTA holds rows 128 rank .. 128 rank + 127.
+// which this CTA holds rows 128 rank .. 128 rank + 127; or, with p.split > 1, CTA `rank`
+// of a K-split cluster, which has the whole tile and its share of the K tiles.
 __device__ __forceinline__ Unit decode_unit(const GemmParams& p, int u, const CUtensorMap* tmap_q, const Sched& sc,
                                             int rank = -1) {
     if (p.groups > 0) {
@@ -340,6 +351,10 @@ __device__ __forceinline__ Unit decode_unit(const GemmParams& p, int u, const CU
         x.sf_q = gd.sf_q;
         x.out = gd.out;
         x.ldo = gd.ldo;
+        if (p.split > 1 && rank >= 0) {
+            x.kt_begin = rank * p.k_tiles / p.split;
+            x.kt_end = (rank + 1) * p.k_tiles / p.split;
+        }
         return x;
     }
     const int tile = u;
@@ -358,6 +373,12 @@ __device__ __forceinline__ Unit decode_unit(const GemmParams& p, int u, const CU
         const int64_t t0 = (int64_t)(tile - p.sk_tile0) * p.k_tiles;
         x.kt_begin = (int)(max(sc.i0, t0) - t0);
         x.kt_end = (int)(min(sc.i1, t0 + p.k_tiles) - t0);
+    }
+    if (p.split > 1 && rank >= 0) {
+        // a K-split cluster: every CTA has the whole tile, and its share of the K range
+        x.kt_begin = rank * p.k_tiles / p.split;
+        x.kt_end = (rank + 1) * p.k_tiles / p.split;
+        rank = -1;
     }
     x.p_row0 = rank >= 0 ? x.tp * 256 + rank * 128 : x.tp * 128;
     x.out_row0 = x.p_row0;
@@ -474,8 +495,21 @@ constexpr int kGemmThreads = 32 * (6 + 4 * kSfWarpSets);
 // Kernel variants, each its own instantiation so that the ordinary kernels keep their
 // registers: kVarGather writes the output to p.dest[0 .. p.n_dest - 1]; kVarFused makes
 // the Q operand (the activations) from bf16 inside the kernel; kVarPair runs on clusters
-// of two CTAs, each pair computing 256 x BN tiles with cta_group::2 MMAs (prefill).
-enum : int { kVarPlain = 0, kVarGather = 1, kVarFused = 2, kVarPair = 3 };
+// of two CTAs, each pair computing 256 x BN tiles with cta_group::2 MMAs (prefill);
+// kVarSplit runs on clusters of p.split CTAs that share one tile's K range.
+enum : int { kVarPlain = 0, kVarGather = 1, kVarFused = 2, kVarPair = 3, kVarSplit = 4 };
+
+// Largest K split over a cluster.
+constexpr int kMaxSplit = 4;
+
+// Whether a ring of `ring_bytes` holds what a K-split CTA keeps there: its parked partial
+// tile (128 x BN fp32) and the other split - 1 CTAs' slices of its own output chunks
+// (ceil(NCH / split) chunks of 128 x 32 fp32 at most).
+template <int BN>
+__host__ __device__ constexpr bool split_ring_fits(int split, int ring_bytes) {
+    constexpr int kChunks = BN / 32;
+    return split >= 2 && 128 * BN * 4 + (split - 1) * ((kChunks + split - 1) / split) * 128 * 32 * 4 <= ring_bytes;
+}
 
 // The fused variant's Q operand, made once per CTA before its main loop by warps 2-13
 // (the epilogue and scale-factor warps; the producer starts streaming the weight tiles
@@ -580,12 +614,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     constexpr bool GATHER = VAR == kVarGather;
     constexpr bool FUSED = VAR == kVarFused;
     constexpr bool PAIR = VAR == kVarPair;
+    constexpr bool SPLIT = VAR == kVarSplit;
     // The fused variant covers Q tiles of at most 32 rows (one 128-row scale slab).
     static_assert(!FUSED || BN <= 32, "fused transform tile");
     // A pair splits its Q tile in two halves of whole 8-row swizzle atoms; prefill only.
     static_assert(!PAIR || BN == 128 || BN == 192, "pair tile");
     using S = GemmShape<BN, STAGES>;
     using L = GemmSmem<BN, STAGES, FUSED, PAIR>;
+    // A K-split CTA parks its fp32 partial tile in its pipeline ring once its MMAs are done
+    // (wide tiles only: one accumulator per tile, no partial sums to add first).
+    static_assert(!SPLIT || (BN >= 128 && 128 * BN * 4 <= STAGES * (S::kPTileBytes + S::kQTileBytes)),
+                  "split partial tile");
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -596,6 +635,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint64_t* acc_empty = bars + 2 * STAGES + 2;
     uint64_t* drain = bars + 2 * STAGES + 4;
     uint64_t* sf_full = bars + 2 * STAGES + 5;    // [STAGES]: scale-factor slot written
+    uint64_t* part_full = bars + 3 * STAGES + 5;  // K split: the other CTAs' slices of this CTA's columns in
+    uint64_t* ring_free = bars + 3 * STAGES + 6;  // K split: every other CTA's ring may take slices
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kOffMisc);
     volatile int* abort = reinterpret_cast<volatile int*>(smem + L::kOffMisc + 4);
 
@@ -604,7 +645,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // CTA pair: rank 0 issues the MMAs of both; rank 1's scale-factor writers and
     // epilogue signal rank 0's sf_full and acc_empty barriers remotely, and rank 0's
     // commits arrive on both CTAs' stage and accumulator barriers.
-    const int rank = PAIR ? (int)ptx::cluster_ctarank() : -1;
+    const int rank = PAIR || SPLIT ? (int)ptx::cluster_ctarank() : -1;
     constexpr uint32_t kPeerArrivals = PAIR ? 2 : 1;
 
     if (threadIdx.x == 0) {
@@ -618,6 +659,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         ptx::mbar_init(drain, 1);
         for (int s = 0; s < STAGES; ++s) ptx::mbar_init(&sf_full[s], 4 * kPeerArrivals);
+        // K split: a CTA arrives once on its own part_full (with the bytes the others copy
+        // in), and once on every other CTA's ring_free
+        ptx::mbar_init(part_full, 1);
+        ptx::mbar_init(ring_free, SPLIT && p.split > 1 ? p.split - 1 : 1);
         *abort = 0;
         ptx::fence_mbar_init();
         ptx::fence_proxy_async_smem();
@@ -636,13 +681,25 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     ptx::tc_fence_before();
     __syncthreads();
-    // the other CTA of a pair signals this CTA's barriers only after they are set up
-    if constexpr (PAIR) ptx::cluster_sync();
+    // the other CTAs of a cluster signal this CTA's barriers only after they are set up
+    if constexpr (PAIR || SPLIT) ptx::cluster_sync();
     ptx::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const Sched sc = cta_sched(p, PAIR);
+    Sched sc = cta_sched(p, PAIR ? 2 : SPLIT ? p.split : 1);
+    if constexpr (SPLIT) {
+        // planned: clusters of p.split CTAs (<= kMaxSplit), at most one tile per cluster
+        // (partial tiles live in the rings after the MMAs), CTA 0's ring large enough for
+        // the others' partial tiles; otherwise do nothing
+        if ((int)ptx::cluster_nctarank() != p.split || p.split < 2 || p.split > kMaxSplit || sc.n_units > 1 ||
+            !split_ring_fits<BN>(p.split, STAGES * (S::kPTileBytes + S::kQTileBytes))) {
+            if (threadIdx.x == 0) atomicExch(p.err, kErrPlan);
+            sc.n_units = 0;
+        }
+    }
     // Set-up above overlaps the previous kernel's tail; operands are read only after it.
-    ptx::griddep_wait();
+    // (With w_early the producer copies the weight side of its first fills first and
+    // waits after that.)
+    if (warp != 0 || !p.w_early) ptx::griddep_wait();
     ptx::griddep_launch_dependents();
     if constexpr (FUSED) {
         if (warp >= 2) fused_transform<BN, STAGES>(p, smem);
@@ -666,30 +723,67 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                                t.sf_q + ((int64_t)(slab0 + c) * p.kb4_pad + 2 * kt) * 512, S::kSfChunkBytes,
                                &full[st]);
         };
-        for (int uj = 0; uj < sc.n_units; ++uj) {
-            const int u = sc.unit(uj);
-            if (cta_aborted(abort)) break;
-            const Unit t = decode_unit(p, u, &tmap_q, sc, rank);
+        // The copies of one fill: its P side (codes tile and scale chunk) and/or its Q side.
+        // `weight` / `act` select the side that holds the weight / the activations (P for
+        // decode's swapped tiles, Q otherwise; the fused variant has no Q copies).
+        const bool p_is_weight = p.transpose_out != 0;
+        auto unit_bytes = [&](const Unit& t) -> uint32_t {
+            const int nchunks = min(S::kQChunks, (t.q_rows + 127) / 128 - (t.tq * BN) / 128);
+            return FUSED ? S::kPTileBytes + S::kSfChunkBytes
+                         : S::kPTileBytes + L::kQStageBytes + S::kSfChunkBytes * (1 + nchunks);
+        };
+        auto issue_fill = [&](const Unit& t, int st, int kt, bool weight, bool act) {
             const int q0 = t.tq * BN;
             const int slab0 = q0 / 128;
             const int nchunks = min(S::kQChunks, (t.q_rows + 127) / 128 - slab0);   // scale slabs of the Q rows
             // P scale slab of the tile; a pair's second CTA past the last P row (its rows
             // are all zero-filled codes, and their results are never stored) reads slab 0
             const int slab_p = t.rows > 0 ? (t.p_row0 >> 7) : 0;
-            // the fused variant copies only the weight side; its Q side is made in place
-            const uint32_t bytes = FUSED ? S::kPTileBytes + S::kSfChunkBytes
-                                         : S::kPTileBytes + L::kQStageBytes + S::kSfChunkBytes * (1 + nchunks);
+            if (p_is_weight ? weight : act) {
+                ptx::tma_load_2d(smem + L::kOffP + st * S::kPTileBytes, &tmap_p, &full[st], kt * S::kBKBytes,
+                                 t.p_row0);
+                ptx::bulk_load(smem + L::kOffSfP + st * S::kSfChunkBytes,
+                               p.sf_p + ((int64_t)slab_p * p.kb4_pad + 2 * kt) * 512, S::kSfChunkBytes, &full[st]);
+            }
+            if constexpr (!FUSED) {
+                if (p_is_weight ? act : weight) issue_q(t, st, kt, q0, slab0, nchunks);
+            }
+        };
+        // w_early: no kernel still running on the stream writes the weight (the library
+        // launched its own activation transform just before, and that kernel starts its
+        // work only after everything before it has completed), so the weight side of the
+        // first fills, whose stages are still free, is copied before the wait for the
+        // previous kernel; their activation side follows in the loop below.
+        int n_early = 0;
+        if (p.w_early) {
+            for (int uj = 0; uj < sc.n_units && n_early < STAGES; ++uj) {
+                const Unit t = decode_unit(p, sc.unit(uj), &tmap_q, sc, rank);
+                for (int kt = t.kt_begin; kt < t.kt_end && n_early < STAGES; ++kt, ++n_early) {
+                    if (leader) {
+                        ptx::mbar_arrive_expect_tx(&full[n_early], unit_bytes(t));
+                        issue_fill(t, n_early, kt, true, false);
+                    }
+                    __syncwarp();
+                }
+            }
+            ptx::griddep_wait();
+        }
+        int fills = 0;
+        for (int uj = 0; uj < sc.n_units; ++uj) {
+            const int u = sc.unit(uj);
+            if (cta_aborted(abort)) break;
+            const Unit t = decode_unit(p, u, &tmap_q, sc, rank);
+            const uint32_t bytes = unit_bytes(t);
             bool ok = true;
-            for (int kt = t.kt_begin; kt < t.kt_end; ++kt) {
-                if (!warp_wait(&empty[stage], phase ^ 1, abort, p.err, kErrTimeoutProducer)) { ok = false; break; }
-                if (leader) {
-                    ptx::mbar_arrive_expect_tx(&full[stage], bytes);
-                    ptx::tma_load_2d(smem + L::kOffP + stage * S::kPTileBytes, &tmap_p, &full[stage],
-                                     kt * S::kBKBytes, t.p_row0);
-                    ptx::bulk_load(smem + L::kOffSfP + stage * S::kSfChunkBytes,
-                                   p.sf_p + ((int64_t)slab_p * p.kb4_pad + 2 * kt) * 512, S::kSfChunkBytes,
-                                   &full[stage]);
-                    if constexpr (!FUSED) issue_q(t, stage, kt, q0, slab0, nchunks);
+            for (int kt = t.kt_begin; kt < t.kt_end; ++kt, ++fills) {
+                if (fills < n_early) {
+                    if (leader) issue_fill(t, stage, kt, false, true);
+                } else {
+                    if (!warp_wait(&empty[stage], phase ^ 1, abort, p.err, kErrTimeoutProducer)) { ok = false; break; }
+                    if (leader) {
+                        ptx::mbar_arrive_expect_tx(&full[stage], bytes);
+                        issue_fill(t, stage, kt, true, true);
+                    }
                 }
                 __syncwarp();
                 issued_mask |= 1u << stage;
@@ -710,7 +804,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             }
         }
         __syncwarp();
-    } else if (warp == 1 && rank <= 0) {
+    } else if (warp == 1 && (!PAIR || rank == 0)) {
         // -------------------------------------------------------------- MMA -----
         // (a pair's MMAs are issued by its rank-0 CTA alone; they wait for both CTAs'
         // scale slots and accumulators, and their commits arrive in both CTAs)
@@ -794,7 +888,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         __syncwarp();
     } else if (warp == 1) {
-        // rank 1 of a pair: no MMAs of its own to issue
+        // rank 1 of a pair: no MMAs of its own to issue (rank 0 issues the pair's)
     } else if (warp >= 6) {
         // ------------------------------------------------- scale-factor writers ---
         // Warp q' (= warp % 4) owns TMEM lanes 32q'..32q'+31. In the 128x4 scale atom,
@@ -844,7 +938,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 ptx::tc_fence_before();
                 __syncwarp();
                 if (lane == 0) {
-                    if (rank > 0) ptx::mbar_arrive_remote(ptx::mapa_shared(&sf_full[stage], 0));
+                    if (PAIR && rank > 0) ptx::mbar_arrive_remote(ptx::mapa_shared(&sf_full[stage], 0));
                     else ptx::mbar_arrive(&sf_full[stage]);
                 }
                 if (++stage == STAGES) { stage = 0; phase ^= 1; }
@@ -927,6 +1021,98 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 }
                 store_chunk<CW>(p, t.out, t.ldo, t.q_rows, prow, row_ok, t.tq * BN + c * CW, r);
             };
+            if constexpr (SPLIT) {
+                // K split over the cluster, finished as a reduce-scatter by columns: CTA s owns
+                // output chunks [s NCH / split, (s + 1) NCH / split). Every CTA parks, in its
+                // own ring (its MMAs have read their last stage, and it has no further tile),
+                // the chunks of its partial tile that other CTAs own, as float4 columns of
+                // 128 rows (columns 4j .. 4j + 3 of row i at float4 j * 128 + i: chunk c is
+                // 16 KB at 16 KB c, and a warp's accesses are 512 contiguous bytes); once
+                // every other CTA's MMAs are done too (ring_free), it copies each CTA's chunks
+                // into that CTA's ring after the parked tile (bulk copies completing on that
+                // CTA's part_full). Each CTA then adds, for its own chunks, the partial tiles
+                // of all CTAs in the order of their K ranges (its own from TMEM) and writes
+                // them to y. The CTAs leave together (cluster barrier at the end), so no
+                // CTA's shared memory goes while a copy may still read or write it.
+                constexpr uint32_t kChunkBytes = 128 * CW * 4;
+                constexpr uint32_t kPartBytes = NCH * kChunkBytes;
+                const int nsplit = p.split;
+                auto chunk0 = [&](int q) { return q * NCH / nsplit; };     // first chunk CTA q owns
+                const int my0 = chunk0(rank), my1 = chunk0(rank + 1);
+                const int row = quad * 32 + lane;
+                float4* part = reinterpret_cast<float4*>(smem);
+#pragma unroll 1
+                for (int c = 0; c < NCH; ++c) {
+                    if (c >= my0 && c < my1) continue;
+                    uint32_t r[CW];
+                    tmem_load_chunk<CW>(taddr + c * CW, r);
+                    ptx::tmem_ld_wait();
+#pragma unroll
+                    for (int j = 0; j < CW; j += 4)
+                        part[((c * CW + j) >> 2) * 128 + row] =
+                            make_float4(__uint_as_float(r[j]), __uint_as_float(r[j + 1]), __uint_as_float(r[j + 2]),
+                                        __uint_as_float(r[j + 3]));
+                }
+                ptx::fence_proxy_async_smem();             // the copies read through the async proxy
+                asm volatile("bar.sync 1, 128;" ::: "memory");
+                if (threadIdx.x == 64) {
+                    // the slices of this CTA's chunks that the others send: expected bytes,
+                    // then this CTA's ring is free for them
+                    ptx::mbar_arrive_expect_tx(part_full, (uint32_t)(nsplit - 1) * (my1 - my0) * kChunkBytes);
+                    for (int q = 0; q < nsplit; ++q)
+                        if (q != rank) ptx::mbar_arrive_remote(ptx::mapa_shared(ring_free, (uint32_t)q));
+                    if (wait_or_abort(ring_free, 0, abort, p.err, kErrTimeoutEpilogue)) {
+                        // CTA q's chunks go to its ring, slot of this CTA among its senders
+                        for (int q = 0; q < nsplit; ++q) {
+                            if (q == rank) continue;
+                            const int q0 = chunk0(q), q1 = chunk0(q + 1);
+                            const uint32_t slot = (uint32_t)(rank < q ? rank : rank - 1);
+                            const uint32_t dst = kPartBytes + slot * (uint32_t)(q1 - q0) * kChunkBytes;
+                            const uint32_t mbar = ptx::mapa_shared(part_full, (uint32_t)q);
+                            for (int c = q0; c < q1; ++c)
+                                ptx::bulk_copy_to_cluster(
+                                    ptx::mapa_shared(smem + dst + (uint32_t)(c - q0) * kChunkBytes, (uint32_t)q),
+                                    smem + (uint32_t)c * kChunkBytes, kChunkBytes, mbar);
+                        }
+                    }
+                }
+                if (!bar_and(1, 128, wait_or_abort(part_full, 0, abort, p.err, kErrTimeoutEpilogue))) break;
+#pragma unroll 1
+                for (int c = my0; c < my1; ++c) {
+                    uint32_t r[CW];
+#pragma unroll 1
+                    for (int q = 0; q < nsplit; ++q) {
+                        // partial of CTA q (K order): this CTA's from TMEM, others from the ring
+                        uint32_t v[CW];
+                        if (q == rank) {
+                            tmem_load_chunk<CW>(taddr + c * CW, v);
+                            ptx::tmem_ld_wait();
+                        } else {
+                            const uint32_t slot = (uint32_t)(q < rank ? q : q - 1);
+                            const float4* src = part + (kPartBytes + slot * (uint32_t)(my1 - my0) * kChunkBytes +
+                                                        (uint32_t)(c - my0) * kChunkBytes) / 16 + row;
+#pragma unroll
+                            for (int j = 0; j < CW / 4; ++j) {
+                                const float4 f = src[j * 128];
+                                v[4 * j] = __float_as_uint(f.x);
+                                v[4 * j + 1] = __float_as_uint(f.y);
+                                v[4 * j + 2] = __float_as_uint(f.z);
+                                v[4 * j + 3] = __float_as_uint(f.w);
+                            }
+                        }
+#pragma unroll
+                        for (int j = 0; j < CW; ++j)
+                            r[j] = q == 0 ? v[j] : __float_as_uint(__fadd_rn(__uint_as_float(r[j]), __uint_as_float(v[j])));
+                    }
+                    emit(c, r);
+                }
+                ptx::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(&acc_empty[acc]);
+                acc ^= 1;
+                if (acc == 0) acc_phase ^= 1;
+                continue;
+            }
             // this thread's row of the CTA's partial-tile slot (the first or the last tile of
             // its stream-K range)
             const int64_t slot_row = ((int64_t)blockIdx.x * 2 + (u == sc.sk_first ? 0 : 1)) * (128 * BN) +
@@ -952,7 +1138,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     ptx::tc_fence_before();
                     __syncwarp();
                     if (lane == 0) {
-                        if (rank > 0) ptx::mbar_arrive_remote(ptx::mapa_shared(&acc_empty[acc], 0));
+                        if (PAIR && rank > 0) ptx::mbar_arrive_remote(ptx::mapa_shared(&acc_empty[acc], 0));
                         else ptx::mbar_arrive(&acc_empty[acc]);
                     }
                 }
@@ -1030,9 +1216,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
     ptx::tc_fence_before();
     __syncthreads();
-    // a pair's CTAs leave together: neither frees its TMEM or shared memory while the
-    // other may still signal it or its MMAs may still write there
-    if constexpr (PAIR) ptx::cluster_sync();
+    // a cluster's CTAs leave together: none frees its TMEM or shared memory while another
+    // may still signal it, read it or (pair) write there with its MMAs
+    if constexpr (PAIR || SPLIT) ptx::cluster_sync();
     if (warp == 1) {
         ptx::tc_fence_after();
         if constexpr (PAIR) ptx::tmem_dealloc_pair(tmem, S::kTmemCols);

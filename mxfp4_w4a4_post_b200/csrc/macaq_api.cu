@@ -203,6 +203,7 @@ macaq_status check_quant_args(const void* x, int64_t rows, int64_t K, int64_t ld
 struct GemmPlan {
     bool swap;        // P = weight, Q = activations, output written transposed
     bool pair;        // clusters of two CTAs, 256 x bn tiles (cta_group::2 MMAs)
+    int split;        // > 1: clusters of `split` CTAs sharing each tile's K range
     int bn;
     int tiles_p, tiles_q, k_tiles;
     int sk_tile0;     // tiles below are whole units dealt round robin; the rest stream-K
@@ -226,6 +227,22 @@ inline double ktile_cycles(int bn) { return std::max(400.0, 2.42 * bn); }
 // (4096 x 14336 x 4096, the same 17 rounds of tiles either way: 102.1 against 107.2 us).
 // A pair's tile is 256 rows, so ragged M costs it more rounds; the planner weighs both.
 constexpr bool kPairPrefill = true;
+// Largest K split over a cluster (the kernel's kMaxSplit), and the planner's estimate of
+// what a split costs beside its share of the K tiles: a fixed part (the cluster launch
+// and the exchange of partial slices: measured ~2-3 us more than one CTA per tile,
+// outside the work itself) and a part per extra CTA. Measured at 256 rows: 5120 x 25600,
+// split 2: 31.4 against 36.3 us; 1024 x 5120, split 4: 16.3 against 14.4 us; 5120 x 8192,
+// split 2: 20.6 against 18.5 us.
+constexpr int kSplitMax = kMaxSplit;
+constexpr double kSplitFixedCycles = 6000.0;
+constexpr double kSplitExchangeCycles = 600.0;
+
+// Whether the ring of the K-split kernel of width bn (the instantiations launched:
+// <128, 6>, <192, 5>) holds a CTA's parked partial tile and the slices it receives.
+bool split_fits(int bn, int split) {
+    return bn == 128 ? split_ring_fits<128>(split, 6 * (GemmShape<128, 6>::kPTileBytes + GemmShape<128, 6>::kQTileBytes))
+                     : split_ring_fits<192>(split, 5 * (GemmShape<192, 5>::kPTileBytes + GemmShape<192, 5>::kQTileBytes));
+}
 constexpr double kPairKtileFactor = 0.95;
 
 GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, int num_sms, bool allow_sk = true, bool allow_pair = true) {
@@ -247,26 +264,40 @@ GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, int num_sms, bool allow_sk =
     }
     const bool pair_ok = kPairPrefill && allow_pair && !swap && M > 128 && N > 128 && num_sms >= 2;
     for (int c = 0; c < 3; ++c) {
-        // candidates: single CTAs with widths[0], widths[1]; then a pair of width 192
+        // candidates: single CTAs with widths[0], widths[1] (each also with its K range
+        // split over a cluster of 2 .. kSplitMax CTAs where every tile's cluster fits on
+        // the SMs at once); then a pair of width 192
         const bool pair = c == 2;
         if (pair ? !pair_ok : widths[c] == 0) continue;
-        GemmPlan g{};
-        g.swap = swap;
-        g.pair = pair;
-        g.k_tiles = k_tiles;
-        g.bn = pair ? 192 : widths[c];
-        g.tiles_p = (int)cdiv(swap ? N : M, pair ? 256 : 128);
-        g.tiles_q = (int)cdiv(swap ? M : N, g.bn);
-        const int64_t tiles = (int64_t)g.tiles_p * g.tiles_q;
-        // time = rounds of tiles over the SMs (pairs) x K tiles per tile x cycles per K tile
-        const double cost = (double)cdiv(tiles, pair ? num_sms / 2 : num_sms) * k_tiles * ktile_cycles(g.bn) *
-                            (pair ? kPairKtileFactor : 1.0);
-        g.sk_tile0 = (int)tiles;
-        g.sk_iters = 0;
-        g.grid = pair ? 2 * (int)std::min<int64_t>(tiles, num_sms / 2) : (int)std::min<int64_t>(tiles, num_sms);
-        if (best.bn == 0 || cost < best_cost * 0.98) {
-            best = g;
-            best_cost = cost;
+        for (int split = 1; split <= (pair || swap ? 1 : kSplitMax); ++split) {
+            GemmPlan g{};
+            g.swap = swap;
+            g.pair = pair;
+            g.split = split;
+            g.k_tiles = k_tiles;
+            g.bn = pair ? 192 : widths[c];
+            g.tiles_p = (int)cdiv(swap ? N : M, pair ? 256 : 128);
+            g.tiles_q = (int)cdiv(swap ? M : N, g.bn);
+            const int64_t tiles = (int64_t)g.tiles_p * g.tiles_q;
+            if (split > 1 &&
+                (!allow_sk || g.bn < 128 || tiles * split > num_sms || k_tiles < 2 * split || !split_fits(g.bn, split)))
+                continue;
+            // time = rounds of tiles over the SMs (pairs) x K tiles per tile x cycles per K
+            // tile; a split tile takes its share of the K tiles plus the exchange of one
+            // partial tile per extra CTA through distributed shared memory
+            const double cost = split > 1 ? (double)cdiv(k_tiles, split) * ktile_cycles(g.bn) + kSplitFixedCycles +
+                                                (split - 1) * kSplitExchangeCycles
+                                          : (double)cdiv(tiles, pair ? num_sms / 2 : num_sms) * k_tiles *
+                                                ktile_cycles(g.bn) * (pair ? kPairKtileFactor : 1.0);
+            g.sk_tile0 = (int)tiles;
+            g.sk_iters = 0;
+            g.grid = split > 1 ? (int)(tiles * split)
+                     : pair    ? 2 * (int)std::min<int64_t>(tiles, num_sms / 2)
+                               : (int)std::min<int64_t>(tiles, num_sms);
+            if (best.bn == 0 || cost < best_cost * 0.98) {
+                best = g;
+                best_cost = cost;
+            }
         }
     }
     // Decode: a weight-streaming product whose last round of tiles would leave SMs idle.
@@ -423,6 +454,49 @@ macaq_status launch_gemm_pair(const CUtensorMap& mp, const CUtensorMap& mq, cons
     return cudaLaunchKernelEx(&cfg, kernel, mp, mq, my, gp) == cudaSuccess ? MACAQ_OK : MACAQ_ERR_CUDA;
 }
 
+// Launch of the K-split variant: one cluster of `split` CTAs per tile. MACAQ_ERR_UNSUPPORTED_SHAPE
+// (nothing launched) when not every tile's cluster fits on the device at once (looked up
+// once per device, tile width and split); the caller then runs single CTAs.
+template <int BN, int STAGES>
+macaq_status launch_gemm_split(const CUtensorMap& mp, const CUtensorMap& mq, const CUtensorMap& my,
+                               const GemmParams& gp, int units, int split, cudaStream_t stream) {
+    using L = GemmSmem<BN, STAGES>;
+    auto kernel = gemm_mxf4_kernel<BN, STAGES, kVarSplit>;
+    static std::mutex m;
+    static int clusters[kMaxDevices][kMaxSplit + 1] = {};
+    int dev = 0;
+    if (split < 2 || split > kMaxSplit) return MACAQ_ERR_UNSUPPORTED_SHAPE;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MACAQ_ERR_CUDA;
+    cudaLaunchConfig_t cfg{};
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)split;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.blockDim = dim3(kGemmThreads);
+    cfg.dynamicSmemBytes = L::kAlloc;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    {
+        std::lock_guard<std::mutex> lock(m);
+        if (clusters[dev][split] == 0) {
+            if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc) != cudaSuccess)
+                return MACAQ_ERR_CUDA;
+            int n = 0;
+            cfg.gridDim = dim3(split);
+            cfg.numAttrs = 1;
+            if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) != cudaSuccess) return MACAQ_ERR_CUDA;
+            clusters[dev][split] = n > 0 ? n : -1;
+        }
+    }
+    if (units > clusters[dev][split]) return MACAQ_ERR_UNSUPPORTED_SHAPE;
+    cfg.gridDim = dim3(units * split);
+    cfg.numAttrs = 2;
+    return cudaLaunchKernelEx(&cfg, kernel, mp, mq, my, gp) == cudaSuccess ? MACAQ_OK : MACAQ_ERR_CUDA;
+}
+
 // Whether the fused variant's persistent Q operand (every K tile of a bn-row tile) fits
 // in shared memory beside its weight ring.
 bool fused_fits(int bn, int k_tiles) {
@@ -464,7 +538,7 @@ struct GatherOut {
 macaq_status run_gemm(const uint8_t* a_codes, const uint8_t* a_scales, int64_t M,
                       const macaq_weight* w, void* y, int64_t ldy, macaq_out_dtype out,
                       void* workspace, size_t ws_bytes, cudaStream_t stream, const FusedAct* fa = nullptr,
-                      const GatherOut* go = nullptr) {
+                      const GatherOut* go = nullptr, bool after_own_quant = false) {
     DeviceInfo* dev = nullptr;
     macaq_status st = device_info(&dev);
     if (st != MACAQ_OK) return st;
@@ -502,8 +576,11 @@ macaq_status run_gemm(const uint8_t* a_codes, const uint8_t* a_scales, int64_t M
     gp.ldo = ldy;
     gp.out_bf16 = out == MACAQ_OUT_BF16 ? 1 : 0;
     gp.vec_ok = (aligned16(y) && (ldy * esz) % 16 == 0) ? 1 : 0;
-    // wide row-major tiles store through TMA (an aligned output is all it needs)
-    gp.tma_store = (!g.swap && g.bn >= 128 && gp.vec_ok) ? 1 : 0;
+    // wide row-major tiles store through TMA when the output is aligned and its rows end
+    // on a 16-byte boundary: a tensor store clips a box at the row's end only to whole
+    // 16-byte pieces (a bf16 output of N = 700 got columns 700..703 written), so other
+    // widths use direct stores, which check every column
+    gp.tma_store = (!g.swap && g.bn >= 128 && gp.vec_ok && (N * esz) % 16 == 0) ? 1 : 0;
     if (go) {
         gp.n_dest = go->n;
         for (int d = 0; d < go->n; ++d) gp.dest[d] = go->dest[d];
@@ -519,6 +596,9 @@ macaq_status run_gemm(const uint8_t* a_codes, const uint8_t* a_scales, int64_t M
         gp.sk_counters = reinterpret_cast<unsigned long long*>(static_cast<uint8_t*>(workspace) + sw.partial_bytes);
         gp.sk_tag = next_sk_tag();
     }
+    // after the library's own activation transform on this stream nothing still running
+    // writes the weight, so its first tiles may be copied before the previous kernel ends
+    gp.w_early = after_own_quant ? 1 : 0;
     const int grid = g.grid;
     if (fa) {
         // decode orientation only, one activation tile held whole in shared memory
@@ -547,6 +627,17 @@ macaq_status run_gemm(const uint8_t* a_codes, const uint8_t* a_scales, int64_t M
                         : launch_gemm_bn<32, 6, kVarFused>(mp, mq, my, gp, grid, stream);
     } else if (g.pair) {
         st = launch_gemm_pair<192, 5>(mp, mq, my, gp, gp.total_units, stream);
+    } else if (g.split > 1) {
+        gp.split = g.split;
+        st = g.bn == 128 ? launch_gemm_split<128, 6>(mp, mq, my, gp, gp.total_units, g.split, stream)
+                         : launch_gemm_split<192, 5>(mp, mq, my, gp, gp.total_units, g.split, stream);
+        if (st == MACAQ_ERR_UNSUPPORTED_SHAPE) {
+            // the clusters do not all fit at once: one CTA per tile
+            gp.split = 1;
+            const int grid1 = std::min(gp.total_units, dev->num_sms);
+            st = g.bn == 128 ? launch_gemm_bn<128, 6>(mp, mq, my, gp, grid1, stream)
+                             : launch_gemm_bn<192, 5>(mp, mq, my, gp, grid1, stream);
+        }
     } else {
         switch (g.bn) {
             case 16: st = launch_gemm_bn<16, 8>(mp, mq, my, gp, grid, stream); break;
@@ -667,7 +758,8 @@ macaq_status macaq_linear_w4a4(const void* x_bf16, int64_t M, int64_t ldx, const
     }
     st = launch_quant(x_bf16, M, w->K, ldx, w->inv_s, a_codes, a_scales, nullptr, nullptr, (cudaStream_t)stream);
     if (st != MACAQ_OK) return st;
-    return run_gemm(a_codes, a_scales, M, w, y, ldy, out, ws + off_gemm, ws_bytes - off_gemm, (cudaStream_t)stream);
+    return run_gemm(a_codes, a_scales, M, w, y, ldy, out, ws + off_gemm, ws_bytes - off_gemm, (cudaStream_t)stream,
+                    nullptr, nullptr, true);
 }
 
 size_t macaq_linear_gather_workspace_bytes(int64_t M, int64_t N, int64_t K, macaq_out_dtype out) {
@@ -699,7 +791,7 @@ macaq_status macaq_linear_w4a4_gather(const void* x_bf16, int64_t M, int64_t ldx
     if (st != MACAQ_OK) return st;
     const GatherOut go{dest, n_dest, vec};
     return run_gemm(ws, ws + off_scales, M, w, nullptr, ldy, out, ws + off_gemm, lin - off_gemm,
-                    (cudaStream_t)stream, nullptr, &go);
+                    (cudaStream_t)stream, nullptr, &go, true);
 }
 
 }  // extern "C"
@@ -910,6 +1002,30 @@ macaq_status run_grouped(const void* x, int64_t ldx, int64_t K, const std::vecto
     gp.groups = (int32_t)G;
     gp.g_desc = reinterpret_cast<const GemmGroup*>(ws + GL.off_desc);
     gp.g_tmaps = reinterpret_cast<const CUtensorMap*>(ws + GL.off_tmaps);
+    // the tables' upload kernels and the grouped quantiser run before this GEMM on the
+    // stream, each starting its work only after everything before it has completed: when
+    // the GEMM starts, the tables and every weight are final
+    gp.w_early = qtab.empty() ? 0 : 1;
+    // few tiles for the SMs (the shared-input q/k/v projections): K split over clusters,
+    // as for a single layer (plan_gemm)
+    const int k_tiles = (int)cdiv(K, 256);
+    // (by the same cost model: one round of the tiles' K tiles against a split's share plus
+    // its fixed and per-CTA costs)
+    if (2 * units <= dev->num_sms && k_tiles >= 4) {
+        int split = (int)std::min<int64_t>(std::min<int64_t>(kSplitMax, dev->num_sms / units), k_tiles / 2);
+        while (split >= 2 && (double)cdiv(k_tiles, split) * ktile_cycles(bn) + kSplitFixedCycles +
+                                     (split - 1) * kSplitExchangeCycles >=
+                                 0.98 * (double)k_tiles * ktile_cycles(bn))
+            --split;
+        while (split >= 2 && !split_fits(bn, split)) --split;
+        if (split >= 2) {
+            gp.split = split;
+            st = bn == 128 ? launch_gemm_split<128, 6>(mp, mq, my, gp, (int)units, split, cs)
+                           : launch_gemm_split<192, 5>(mp, mq, my, gp, (int)units, split, cs);
+            if (st != MACAQ_ERR_UNSUPPORTED_SHAPE) return st;
+            gp.split = 1;
+        }
+    }
     const int grid = (int)std::min<int64_t>(units, dev->num_sms);
     return bn == 128 ? launch_gemm_bn<128, 6>(mp, mq, my, gp, grid, cs) : launch_gemm_bn<192, 5>(mp, mq, my, gp, grid, cs);
 }

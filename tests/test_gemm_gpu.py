@@ -1,9 +1,11 @@
 """Parity of the block-scaled FP4 GEMM (tcgen05 kind::mxf4) with the oracle's fp64 sum
 of decoded products. One-hot operands pin the nibble order and the scale layout;
 random codes and scales cover every tile path (swapped decode tiles of width 16..128,
-prefill tiles of width 128/192, 256 x 192 tiles of CTA pairs, the stream-K schedule
-whose shared tiles are finished by their last contributor, ragged M/N/K) and every
-output path (TMA tensor stores of staged boxes, direct stores, transposed stores)."""
+prefill tiles of width 128/192, 256 x 192 tiles of CTA pairs, tiles whose K range is
+split over a cluster of 2..4 CTAs that finish them as a reduce-scatter of partial
+slices, the stream-K schedule whose shared tiles are finished by their last
+contributor, ragged M/N/K) and every output path (TMA tensor stores of staged boxes,
+direct stores, transposed stores)."""
 import numpy as np
 import pytest
 
@@ -52,9 +54,11 @@ def one_hot_operands(M, N, K, picks):
     return pack(a), sa, pack(w), sw
 
 
-# the last shape runs on CTA pairs (rows 128..255 of each 256-row tile, and weight rows
-# 96..191 of each 192-row tile, in the second CTA of the pair)
-@pytest.mark.parametrize("M,N,K", [(16, 128, 256), (300, 448, 512), (200, 130, 768), (700, 4200, 768)])
+# the last two shapes run on CTA pairs (rows 128..255 of each 256-row tile, and weight
+# rows 96..191 of each 192-row tile, in the second CTA of the pair) and with each tile's K
+# range split over a cluster of four CTAs (every product lands in one CTA's partial tile)
+@pytest.mark.parametrize("M,N,K", [(16, 128, 256), (300, 448, 512), (200, 130, 768), (700, 4200, 768),
+                                   (130, 300, 12288)])
 def test_one_hot_layout(mq, M, N, K):
     rng = np.random.default_rng(M + N + K)
     picks, used_k, used_m, used_n = [], set(), set(), set()
@@ -86,6 +90,8 @@ SHAPES = [
     # rows in the first, and a last weight tile whose second half is empty (N % 192 = 88)
     # or partly filled (N % 192 = 168)
     (300, 7000, 768), (520, 4200, 768),
+    # each tile's K range split over a cluster of 4 CTAs (tiles 128 and 192 wide), 3 and 2
+    (300, 700, 12288), (640, 1000, 12288), (1024, 1000, 8192), (1536, 1000, 12288),
 ]
 
 
@@ -132,6 +138,7 @@ OUTPUT_CASES = [
     (1, 25600, 5120, "bf16", 8), (16, 19000, 5376, "f32", 4),    # stream-K: shared tiles
     (700, 4200, 256, "bf16", 0), (300, 7000, 768, "f32", 4),     # CTA pairs
     (1000, 6100, 768, "bf16", 8),                                # CTA pairs, unaligned rows
+    (300, 700, 512, "bf16", 12),    # aligned row stride, rows not 16-byte multiples: no tensor store
 ]
 
 

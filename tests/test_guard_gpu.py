@@ -96,6 +96,7 @@ GEMM_CASES = [
     (16, 256, 16384, "bf16", 264),
     (8, 19100, 768, "f32", 19104),
     (700, 4200, 256, "bf16", 4216),          # CTA pairs, ragged second CTA and weight half
+    (300, 700, 12288, "bf16", 712),          # K split over clusters of four CTAs
 ]
 
 

@@ -65,6 +65,7 @@ def check_layers(mq, M, K, Ns, dt="f32", pad=0, seed=0):
     (300, 768, (384, 200), "bf16", 8),
     (129, 512, (1000,), "f32", 4),
     (256, 1024, (1024, 128, 128), "bf16", 0),
+    (256, 12288, (256, 128), "f32", 4),     # few tiles, long K: each tile's K range split over 4 CTAs
 ])
 def test_shared_input_layers(mq, M, K, Ns, dt, pad):
     check_layers(mq, M, K, Ns, dt, pad)
