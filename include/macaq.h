@@ -140,8 +140,10 @@ macaq_status macaq_quant_act(const void* x_bf16, int64_t M, int64_t K, int64_t l
  * article):
  *   y[m, n] = sum_b 2^(ea[m,b] + ew[n,b]) * sum_{k in b} dec(a[m,k]) * dec(w[n,k]),
  * fp32 accumulation on the tensor cores (tcgen05 kind::mxf4). Large prefill products
- * run on clusters of two CTAs (256-row tiles, cta_group::2 MMAs), the rest on single
- * CTAs; the choice is the library's and does not change the result's tolerance.
+ * run on clusters of two CTAs (256-row tiles, cta_group::2 MMAs), products with few
+ * long-K tiles on clusters of 2-4 CTAs that share each tile's K range, the rest on single
+ * CTAs; the choice is the library's and does not change the result's tolerance. Every
+ * plan gives the same y for the same inputs, call after call.
  *   a_codes/a_scales device, as written by macaq_quant_act for M rows
  *   w        prepared weight (inv_s unused here)
  *   y        device [M x N] fp32 or bf16, row stride ldy elements (ldy >= N), aligned

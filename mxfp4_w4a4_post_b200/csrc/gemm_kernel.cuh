@@ -37,6 +37,7 @@
 #pragma once
 
 #include <cstdint>
+#include <type_traits>
 #include <cuda.h>
 #include <cuda_bf16.h>
 
@@ -723,75 +724,100 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                                t.sf_q + ((int64_t)(slab0 + c) * p.kb4_pad + 2 * kt) * 512, S::kSfChunkBytes,
                                &full[st]);
         };
-        // The copies of one fill: its P side (codes tile and scale chunk) and/or its Q side.
-        // `weight` / `act` select the side that holds the weight / the activations (P for
-        // decode's swapped tiles, Q otherwise; the fused variant has no Q copies).
-        const bool p_is_weight = p.transpose_out != 0;
-        auto unit_bytes = [&](const Unit& t) -> uint32_t {
-            const int nchunks = min(S::kQChunks, (t.q_rows + 127) / 128 - (t.tq * BN) / 128);
-            return FUSED ? S::kPTileBytes + S::kSfChunkBytes
-                         : S::kPTileBytes + L::kQStageBytes + S::kSfChunkBytes * (1 + nchunks);
-        };
-        auto issue_fill = [&](const Unit& t, int st, int kt, bool weight, bool act) {
-            const int q0 = t.tq * BN;
-            const int slab0 = q0 / 128;
-            const int nchunks = min(S::kQChunks, (t.q_rows + 127) / 128 - slab0);   // scale slabs of the Q rows
-            // P scale slab of the tile; a pair's second CTA past the last P row (its rows
-            // are all zero-filled codes, and their results are never stored) reads slab 0
-            const int slab_p = t.rows > 0 ? (t.p_row0 >> 7) : 0;
-            if (p_is_weight ? weight : act) {
-                ptx::tma_load_2d(smem + L::kOffP + st * S::kPTileBytes, &tmap_p, &full[st], kt * S::kBKBytes,
-                                 t.p_row0);
-                ptx::bulk_load(smem + L::kOffSfP + st * S::kSfChunkBytes,
-                               p.sf_p + ((int64_t)slab_p * p.kb4_pad + 2 * kt) * 512, S::kSfChunkBytes, &full[st]);
-            }
-            if constexpr (!FUSED) {
-                if (p_is_weight ? act : weight) issue_q(t, st, kt, q0, slab0, nchunks);
-            }
-        };
         // w_early: no kernel still running on the stream writes the weight (the library
         // launched its own activation transform just before, and that kernel starts its
         // work only after everything before it has completed), so the weight side of the
         // first fills, whose stages are still free, is copied before the wait for the
-        // previous kernel; their activation side follows in the loop below.
+        // previous kernel; their activation side follows in the loop below. The weight is
+        // P for decode's swapped tiles, Q otherwise. The main loop is instantiated twice so
+        // that the one without early fills is the plain loop (a test per K tile in it cost
+        // ~4% of the prefill GEMM).
+        const bool p_is_weight = p.transpose_out != 0;
         int n_early = 0;
         if (p.w_early) {
             for (int uj = 0; uj < sc.n_units && n_early < STAGES; ++uj) {
                 const Unit t = decode_unit(p, sc.unit(uj), &tmap_q, sc, rank);
+                const int q0 = t.tq * BN;
+                const int slab0 = q0 / 128;
+                const int nchunks = min(S::kQChunks, (t.q_rows + 127) / 128 - slab0);
+                const int slab_p = t.rows > 0 ? (t.p_row0 >> 7) : 0;
+                const uint32_t bytes = FUSED ? S::kPTileBytes + S::kSfChunkBytes
+                                             : S::kPTileBytes + L::kQStageBytes + S::kSfChunkBytes * (1 + nchunks);
                 for (int kt = t.kt_begin; kt < t.kt_end && n_early < STAGES; ++kt, ++n_early) {
                     if (leader) {
-                        ptx::mbar_arrive_expect_tx(&full[n_early], unit_bytes(t));
-                        issue_fill(t, n_early, kt, true, false);
+                        ptx::mbar_arrive_expect_tx(&full[n_early], bytes);
+                        if (p_is_weight) {
+                            ptx::tma_load_2d(smem + L::kOffP + n_early * S::kPTileBytes, &tmap_p, &full[n_early],
+                                             kt * S::kBKBytes, t.p_row0);
+                            ptx::bulk_load(smem + L::kOffSfP + n_early * S::kSfChunkBytes,
+                                           p.sf_p + ((int64_t)slab_p * p.kb4_pad + 2 * kt) * 512, S::kSfChunkBytes,
+                                           &full[n_early]);
+                        } else if constexpr (!FUSED) {
+                            issue_q(t, n_early, kt, q0, slab0, nchunks);
+                        }
                     }
                     __syncwarp();
                 }
             }
             ptx::griddep_wait();
         }
-        int fills = 0;
-        for (int uj = 0; uj < sc.n_units; ++uj) {
-            const int u = sc.unit(uj);
-            if (cta_aborted(abort)) break;
-            const Unit t = decode_unit(p, u, &tmap_q, sc, rank);
-            const uint32_t bytes = unit_bytes(t);
-            bool ok = true;
-            for (int kt = t.kt_begin; kt < t.kt_end; ++kt, ++fills) {
-                if (fills < n_early) {
-                    if (leader) issue_fill(t, stage, kt, false, true);
-                } else {
-                    if (!warp_wait(&empty[stage], phase ^ 1, abort, p.err, kErrTimeoutProducer)) { ok = false; break; }
-                    if (leader) {
-                        ptx::mbar_arrive_expect_tx(&full[stage], bytes);
-                        issue_fill(t, stage, kt, true, true);
+        auto main_loop = [&](auto has_early) {
+            constexpr bool kEarly = decltype(has_early)::value;
+            int fills = 0;
+            for (int uj = 0; uj < sc.n_units; ++uj) {
+                const int u = sc.unit(uj);
+                if (cta_aborted(abort)) break;
+                const Unit t = decode_unit(p, u, &tmap_q, sc, rank);
+                const int q0 = t.tq * BN;
+                const int slab0 = q0 / 128;
+                const int nchunks = min(S::kQChunks, (t.q_rows + 127) / 128 - slab0);   // scale slabs of the Q rows
+                // P scale slab of the tile; a pair's second CTA past the last P row (its rows
+                // are all zero-filled codes, and their results are never stored) reads slab 0
+                const int slab_p = t.rows > 0 ? (t.p_row0 >> 7) : 0;
+                // the fused variant copies only the weight side; its Q side is made in place
+                const uint32_t bytes = FUSED ? S::kPTileBytes + S::kSfChunkBytes
+                                             : S::kPTileBytes + L::kQStageBytes + S::kSfChunkBytes * (1 + nchunks);
+                bool ok = true;
+                for (int kt = t.kt_begin; kt < t.kt_end; ++kt) {
+                    if (kEarly && fills < n_early) {
+                        // an early fill: its activation side
+                        if (leader) {
+                            if (!p_is_weight) {
+                                ptx::tma_load_2d(smem + L::kOffP + stage * S::kPTileBytes, &tmap_p, &full[stage],
+                                                 kt * S::kBKBytes, t.p_row0);
+                                ptx::bulk_load(smem + L::kOffSfP + stage * S::kSfChunkBytes,
+                                               p.sf_p + ((int64_t)slab_p * p.kb4_pad + 2 * kt) * 512,
+                                               S::kSfChunkBytes, &full[stage]);
+                            } else if constexpr (!FUSED) {
+                                issue_q(t, stage, kt, q0, slab0, nchunks);
+                            }
+                        }
+                    } else {
+                        if (!warp_wait(&empty[stage], phase ^ 1, abort, p.err, kErrTimeoutProducer)) {
+                            ok = false;
+                            break;
+                        }
+                        if (leader) {
+                            ptx::mbar_arrive_expect_tx(&full[stage], bytes);
+                            ptx::tma_load_2d(smem + L::kOffP + stage * S::kPTileBytes, &tmap_p, &full[stage],
+                                             kt * S::kBKBytes, t.p_row0);
+                            ptx::bulk_load(smem + L::kOffSfP + stage * S::kSfChunkBytes,
+                                           p.sf_p + ((int64_t)slab_p * p.kb4_pad + 2 * kt) * 512, S::kSfChunkBytes,
+                                           &full[stage]);
+                            if constexpr (!FUSED) issue_q(t, stage, kt, q0, slab0, nchunks);
+                        }
                     }
+                    __syncwarp();
+                    if constexpr (kEarly) ++fills;
+                    issued_mask |= 1u << stage;
+                    issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
+                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
                 }
-                __syncwarp();
-                issued_mask |= 1u << stage;
-                issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
-                if (++stage == STAGES) { stage = 0; phase ^= 1; }
+                if (!ok) break;
             }
-            if (!ok) break;
-        }
+        };
+        if (n_early > 0) main_loop(std::true_type{});
+        else main_loop(std::false_type{});
         if (cta_aborted(abort) && leader) {
             // let copies already in flight land before the CTA can exit: wait
             // (bounded) for the phase of the latest fill of every stage
