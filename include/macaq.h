@@ -374,7 +374,9 @@ macaq_status macaq_linear_w4a4_noalloc(const void* x_bf16, int64_t M, int64_t ld
 /* ------------------------------------------------------------ status ---------- */
 
 /* Every wait inside the GEMM kernel is bounded. A kernel that gives up a wait records
- * a code in a device-side word and returns early (its output is then undefined).
+ * a code in a device-side word and returns early (its output is then undefined); so does
+ * a kernel launched in a way it is not planned for (a scale-factor offset or a cluster
+ * size the plan never gives).
  * This call synchronises the current device, reads the word, clears it, and returns
  * MACAQ_ERR_DEVICE_TIMEOUT if it was set (MACAQ_OK otherwise, MACAQ_ERR_CUDA if the
  * read fails). */
