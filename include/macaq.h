@@ -201,8 +201,9 @@ macaq_status macaq_linear_w4a4(const void* x_bf16, int64_t M, int64_t ldx, const
  *             macaq_linear_w4a4's), 256-byte aligned. The destination addresses travel in
  *             the GEMM kernel's parameters.
  * Every destination receives the same values that macaq_linear_w4a4 (fused = 0) would
- * write to y, except that no output tile is shared between CTAs (no stream-K
- * schedule), so sums may round differently. Completion of the writes into another
+ * write to y, except that every output tile is computed by one CTA over its whole K
+ * range (no stream-K schedule, no K split over a cluster, no CTA pairs), so sums may
+ * round differently. Completion of the writes into another
  * GPU's memory is ordered for that GPU only by the caller (for example a barrier on
  * both streams after the call). */
 size_t macaq_linear_gather_workspace_bytes(int64_t M, int64_t N, int64_t K, macaq_out_dtype out);
