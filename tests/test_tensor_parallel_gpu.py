@@ -148,7 +148,10 @@ def test_gathered_column_cut(mq, M, N, K, shards, dt):
     if dt == "f32":
         assert_gemm_close(y0, ref, f"gathered column cut {M}x{N}x{K}")
     # each shard's columns equal the ordinary layer's output for that shard whenever
-    # that one gives every tile to one CTA (same tiles, same MMAs, another store path)
+    # that one computes every tile over its whole K range on one CTA or a CTA pair (same
+    # K order per tile, same MMAs, another store path): no stream-K workspace, and no K
+    # split over a cluster, which these shapes (K <= 1024 at prefill rows, or decode
+    # rows) never get
     for n0, n1, w in shard_out:
         y_lin = mq.linear(xd, w, out_dtype=dtype)
         if mq.gemm_workspace_bytes(M, n1 - n0, K, dtype) == 0:
